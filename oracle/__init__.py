@@ -1,0 +1,162 @@
+"""fp64 CPU oracle for the SSA block-sparse attention path (TEST INFRASTRUCTURE).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg may import this package.  It shares no code with the CUDA path; the C source
+``ssa_oracle.c`` is compiled with gcc/OpenMP into ``libssa_oracle.so`` beside it.
+
+Functions take/return numpy arrays laid out [BH, T, d] (batch and heads
+flattened) in float64, selections as int32 [BH, T, k].
+
+What each function computes (readings of "SSA: Sparse Sparse Attention by
+Aligning Full and Sparse Attention Outputs in Feature Space", paperlayer.ai
+summary of v4):
+  block_pool    section 3  mean-pooled block keys
+  block_select  section 3  current block + top-(k-1) preceding blocks by q.Kbar
+  attn_fwd      sections 3 full causal attention / attention over the selected
+                           blocks' tokens
+  attn_bwd      section 4.2 gradients; dropped keys get none
+  align_fwd/bwd section 5  bidirectional SmoothL1 output alignment
+  dropped_mass  section 4.2 / Appendix B  delta = 1 - exp(lse_s - lse_f)
+
+Parity pins: see tests/test_oracle_pins.py.  Every function there is pinned
+(brute force, library special cases, closed forms, invariants, finite
+differences); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssa_oracle.c")
+_LIB = os.path.join(_HERE, "libssa_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle's C source (gcc -O2 -fopenmp); return the library path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB)
+    i64, dbl, p = ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
+    lib.ora_num_threads.restype = ctypes.c_int
+    lib.ora_block_pool.argtypes = [i64, i64, i64, i64, p, p]
+    lib.ora_block_select.argtypes = [i64, i64, i64, i64, i64, p, p, p, p, p]
+    lib.ora_check_selection.argtypes = [i64, i64, i64, i64, p]
+    lib.ora_check_selection.restype = ctypes.c_int
+    lib.ora_attn_fwd.argtypes = [i64, i64, i64, i64, i64, dbl, p, p, p, p, i64, p, p, p]
+    lib.ora_attn_bwd.argtypes = [i64, i64, i64, i64, i64, dbl, p, p, p, p, p, i64, p, i64, p, p, p, p]
+    lib.ora_align_fwd.argtypes = [i64, p, p, dbl, dbl, dbl]
+    lib.ora_align_fwd.restype = dbl
+    lib.ora_align_bwd.argtypes = [i64, p, p, dbl, dbl, dbl, dbl, p, p]
+    _lib = lib
+    return lib
+
+
+def _f64(x) -> np.ndarray:
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _rows(rows) -> Optional[np.ndarray]:
+    return None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+
+
+def num_threads() -> int:
+    return int(_load().ora_num_threads())
+
+
+def block_pool(K: np.ndarray, s: int) -> np.ndarray:
+    """K [BH, T, d] -> Kbar [BH, T/s, d]."""
+    K = _f64(K)
+    BH, T, d = K.shape
+    out = np.empty((BH, T // s, d), dtype=np.float64)
+    _load().ora_block_pool(BH, T, d, s, _ptr(K), _ptr(out))
+    return out
+
+
+def block_select(Q: np.ndarray, Kbar: np.ndarray, s: int, k: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Q [BH, T, d], Kbar [BH, nb, d] -> (idx int32 [BH,T,k], r_(k-1) [BH,T], r_(k) [BH,T])."""
+    Q, Kbar = _f64(Q), _f64(Kbar)
+    BH, T, d = Q.shape
+    idx = np.empty((BH, T, k), dtype=np.int32)
+    r1 = np.empty((BH, T), dtype=np.float64)
+    r2 = np.empty((BH, T), dtype=np.float64)
+    _load().ora_block_select(BH, T, d, s, k, _ptr(Q), _ptr(Kbar), _ptr(idx), _ptr(r1), _ptr(r2))
+    return idx, r1, r2
+
+
+def check_selection(idx: np.ndarray, s: int) -> bool:
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    BH, T, k = idx.shape
+    return bool(_load().ora_check_selection(BH, T, s, k, _ptr(idx)))
+
+
+def attn_fwd(Q, K, V, s: int, scale: float, idx: Optional[np.ndarray] = None, rows=None):
+    """Full (idx None) or sparse attention forward -> (O [BH, n, d], lse [BH, n])."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    BH, T, d = Q.shape
+    k = 0 if idx is None else idx.shape[-1]
+    if idx is not None:
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+    rows = _rows(rows)
+    n = T if rows is None else rows.shape[0]
+    O = np.empty((BH, n, d), dtype=np.float64)
+    lse = np.empty((BH, n), dtype=np.float64)
+    _load().ora_attn_fwd(BH, T, d, s, k, float(scale), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
+                         n, _ptr(rows), _ptr(O), _ptr(lse))
+    return O, lse
+
+
+def attn_bwd(Q, K, V, dO, s: int, scale: float, idx: Optional[np.ndarray] = None, qrows=None, krows=None):
+    """Gradients of sum(dO * O) -> (dQ [BH, nq, d], dK [BH, nk, d], dV [BH, nk, d])."""
+    Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
+    BH, T, d = Q.shape
+    k = 0 if idx is None else idx.shape[-1]
+    if idx is not None:
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+    qrows, krows = _rows(qrows), _rows(krows)
+    nq = T if qrows is None else qrows.shape[0]
+    nk = T if krows is None else krows.shape[0]
+    dQ = np.empty((BH, nq, d), dtype=np.float64)
+    dK = np.empty((BH, nk, d), dtype=np.float64)
+    dV = np.empty((BH, nk, d), dtype=np.float64)
+    _load().ora_attn_bwd(BH, T, d, s, k, float(scale), _ptr(Q), _ptr(K), _ptr(V), _ptr(dO), _ptr(idx),
+                         nq, _ptr(qrows), nk, _ptr(krows), _ptr(dQ), _ptr(dK), _ptr(dV))
+    return dQ, dK, dV
+
+
+def align_fwd(Of, Os, beta: float = 1.0, w_sparsity: float = 1.0, w_commit: float = 1.0) -> float:
+    Of, Os = _f64(Of).ravel(), _f64(Os).ravel()
+    return float(_load().ora_align_fwd(Of.size, _ptr(Of), _ptr(Os), beta, w_sparsity, w_commit))
+
+
+def align_bwd(Of, Os, beta: float = 1.0, w_sparsity: float = 1.0, w_commit: float = 1.0, g: float = 1.0):
+    shape = np.shape(Of)
+    Of, Os = _f64(Of).ravel(), _f64(Os).ravel()
+    dOf = np.empty_like(Of)
+    dOs = np.empty_like(Os)
+    _load().ora_align_bwd(Of.size, _ptr(Of), _ptr(Os), beta, w_sparsity, w_commit, g, _ptr(dOf), _ptr(dOs))
+    return dOf.reshape(shape), dOs.reshape(shape)
+
+
+def dropped_mass(lse_sparse: np.ndarray, lse_full: np.ndarray) -> np.ndarray:
+    """Page section 4.2 / Appendix B: full-attention mass outside S(t), delta = 1 - exp(lse_s - lse_f)."""
+    return 1.0 - np.exp(_f64(lse_sparse) - _f64(lse_full))
