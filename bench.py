@@ -1,0 +1,356 @@
+#!/usr/bin/env python3
+"""Benchmark of the SSA block-sparse attention hot path on B200.
+
+One step = one pass of the whole path over one batch of the 32K-context
+workload (B=1, H=32, T=32768, d=128, s=128, k=16, bf16, sink block):
+  block pooling, causal top-k selection, full causal attention forward,
+  sparse attention forward, alignment loss forward, alignment backward (the
+  main stream -- full on even steps, sparse on odd steps -- also receives its
+  upstream gradient), full attention backward and sparse attention backward
+  accumulating into one set of dQ, dK, dV.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  N > 1 runs independent replicas, one per GPU
+(the path has no exchange step); value = tokens of all ranks / max-over-ranks time.
+``--impl reference`` times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload (see ``reference_arm``).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn fwd+bwd TFLOP/s & tokens/s at 32K ctx; % of bf16 tensor peak"
+WORKLOAD = "long"
+K_SEL = 16
+
+
+def flops(B, H, T, d, s, k):
+    """Algorithmic FLOPs: sparse fwd 4*B*H*d*sum_t min(k*s, t+1); full fwd 4*B*H*d*T(T+1)/2; bwd = 2.5 x fwd."""
+    t = np.arange(T, dtype=np.float64)
+    sparse_fwd = 4.0 * B * H * d * np.minimum(k * s, t + 1).sum()
+    full_fwd = 4.0 * B * H * d * T * (T + 1) / 2.0
+    return sparse_fwd, 2.5 * sparse_fwd, full_fwd, 2.5 * full_fwd
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index, self.proc = index, None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (getattr(self, "out", "") or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][1]) if rows[0][1].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def oracle_sample(T_sample: int, seed_rows: int = 0):
+    """Run the oracle's whole step on a prefix sample: head (0,0), first T_sample tokens.
+
+    Returns (seconds, sample FLOPs by the same algorithmic count, description)."""
+    import oracle
+    from block_top_sparse_b200 import inputs
+    wl = inputs.WORKLOADS[WORKLOAD]
+    g = inputs.generate(wl, H=1, T=T_sample)
+    f = {key: inputs.to_float64(g[key], "bf16").reshape(1, T_sample, wl.d) for key in ("Q", "K", "V", "dO")}
+    s, k, scale = wl.s, K_SEL, wl.d ** -0.5
+    t0 = time.perf_counter()
+    Kbar = oracle.block_pool(f["K"], s)
+    idx, _, _ = oracle.block_select(f["Q"], Kbar, s, k)
+    Of, lf = oracle.attn_fwd(f["Q"], f["K"], f["V"], s, scale)
+    Os, ls = oracle.attn_fwd(f["Q"], f["K"], f["V"], s, scale, idx)
+    oracle.align_fwd(Of, Os)
+    gf, gs = oracle.align_bwd(Of, Os)
+    oracle.attn_bwd(f["Q"], f["K"], f["V"], f["dO"] + gf, s, scale)
+    oracle.attn_bwd(f["Q"], f["K"], f["V"], gs, s, scale, idx)
+    dt = time.perf_counter() - t0
+    fl = sum(flops(1, 1, T_sample, wl.d, s, k))
+    return dt, fl, "head (b=0,h=0), first %d of %d tokens, whole step (pool, select, full+sparse fwd, align fwd/bwd, full+sparse bwd)" % (T_sample, wl.T)
+
+
+def reference_arm(args, rank):
+    """The oracle as it stands on the host cores; throughput scaled to the full workload by FLOPs."""
+    if rank != 0:
+        return
+    import oracle
+    from block_top_sparse_b200 import inputs
+    oracle.build()
+    wl = inputs.WORKLOADS[WORKLOAD]
+    full_fl = sum(flops(wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL))
+    T_sample = args.ref_tokens
+    for _ in range(args.warmup):
+        oracle_sample(T_sample)
+    times, fl, desc = [], None, None
+    for _ in range(args.steps):
+        dt, fl, desc = oracle_sample(T_sample)
+        times.append(dt)
+    est = sum(times) / len(times) * full_fl / fl  # seconds for one full step
+    tok_s = wl.B * wl.T / est
+    line = {"metric": METRIC, "value": tok_s, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_block(wl),
+            "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": desc + "; time per sample %.2f s, scaled to the full step by algorithmic FLOPs"
+                             % (sum(times) / len(times))},
+            "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_block(wl):
+    return {"workload": "long-context fwd+bwd, both streams + alignment: B=%d H=%d T=%d d=%d s=%d k=%d, sink block"
+                        % (wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL),
+            "B": wl.B, "H": wl.H, "T": wl.T, "d": wl.d, "s": wl.s, "k": K_SEL, "global_batch": wl.B, "seq_len": wl.T,
+            "parallelism": "replicas", "main_stream": "alternating full/sparse per step",
+            "l2": "inputs larger than L2 (Q, K, V, dO 268 MB each)"}
+
+
+def ours(args, rank, world, local_rank):
+    import torch
+    from block_top_sparse_b200 import _lib as L
+    from block_top_sparse_b200 import build, inputs, ops
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = inputs.WORKLOADS[WORKLOAD]
+    g = inputs.generate(wl)
+    host = {}
+    for key in ("Q", "K", "V", "dO"):
+        t = torch.from_numpy(g[key].view(np.int16)).view(torch.bfloat16)
+        host[key] = t.pin_memory()
+    d = {key: host[key].to(dev, non_blocking=False) for key in host}
+    dims = L.make_dims(wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL, dtype="bf16")
+    steps = [ops.SSAStep(dims, device=dev, main="full"), ops.SSAStep(dims, device=dev, main="sparse")]
+    # the two steps share no buffers: allocate once, reuse alternately
+    stream = torch.cuda.current_stream(dev)
+
+    ev = {name: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for name in ("pool", "select", "full_fwd", "sparse_fwd", "align_fwd", "align_bwd", "full_bwd", "sparse_bwd")}
+    per_op = {name: [] for name in ev}
+
+    def run_step(i, timed_ops=False):
+        st = steps[i % 2]
+        Q, K, V = d["Q"], d["K"], d["V"]
+        dd = st.dims
+
+        def rec(name, fn):
+            if timed_ops:
+                ev[name][0].record(stream)
+            fn()
+            if timed_ops:
+                ev[name][1].record(stream)
+
+        rec("pool", lambda: L.ssa_block_pool(dd, K, st.Kbar))
+        rec("select", lambda: L.ssa_block_select(dd, Q, st.Kbar, st.idx))
+        rec("full_fwd", lambda: L.ssa_full_attn_fwd(dd, Q, K, V, st.Of, st.lse_f, st.ws[L.SSA_OP_FULL_FWD]))
+        rec("sparse_fwd", lambda: L.ssa_sparse_attn_fwd(dd, Q, K, V, st.idx, st.Os, st.lse_s,
+                                                        st.ws[L.SSA_OP_SPARSE_FWD]))
+        rec("align_fwd", lambda: L.ssa_align_loss_fwd(dd, st.Of, st.Os, 1.0, 1.0, 1.0, st.loss,
+                                                      st.ws[L.SSA_OP_ALIGN_FWD]))
+        st.main_grad_buffer().copy_(d["dO"], non_blocking=True)  # upstream gradient of the main stream
+        acc = L.SSA_ACC_OF if st.main == "full" else L.SSA_ACC_OS
+        rec("align_bwd", lambda: L.ssa_align_loss_bwd(dd, st.Of, st.Os, 1.0, 1.0, 1.0, st.dloss, st.dOf, st.dOs,
+                                                      acc))
+        rec("full_bwd", lambda: L.ssa_full_attn_bwd(dd, Q, K, V, st.Of, st.lse_f, st.dOf, st.dQ, st.dK, st.dV, 0,
+                                                    st.ws[L.SSA_OP_FULL_BWD]))
+        rec("sparse_bwd", lambda: L.ssa_sparse_attn_bwd(dd, Q, K, V, st.Os, st.lse_s, st.dOs, st.idx, st.dQ, st.dK,
+                                                        st.dV, 1, st.ws[L.SSA_OP_SPARSE_BWD]))
+        if timed_ops:
+            torch.cuda.synchronize(dev)
+            for name, (a, b) in ev.items():
+                per_op[name].append(a.elapsed_time(b))
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        run_step(i)
+    torch.cuda.synchronize(dev)
+    if L.ssa_get_device_error() != L.SSA_OK:
+        raise RuntimeError("device error during warm-up")
+
+    # ---- timed region: K whole steps, inputs resident in HBM ----
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize(dev)
+        start.record(stream)
+        for i in range(args.steps):
+            run_step(i)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    ms = start.elapsed_time(end)
+    clocks = clk.summary()
+
+    # ---- per-op breakdown (separate, untimed-for-value pass) ----
+    for i in range(max(2, min(args.steps, 4))):
+        run_step(i, timed_ops=True)
+
+    # ---- end to end: pinned host inputs -> device, step, loss back to host ----
+    loss_host = torch.empty((), dtype=torch.float32).pin_memory()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e_start.record(stream)
+    for i in range(args.steps):
+        for key in ("Q", "K", "V", "dO"):
+            d[key].copy_(host[key], non_blocking=True)
+        run_step(i)
+        loss_host.copy_(steps[i % 2].loss, non_blocking=True)
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e_ms = e_start.elapsed_time(e_end)
+    if L.ssa_get_device_error() != L.SSA_OK:
+        raise RuntimeError("device error during timing")
+
+    if dist is not None:
+        t = torch.tensor([ms, e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e_ms = float(t[0]), float(t[1])
+    if rank != 0:
+        return
+
+    hbm, peak_burst, peak_sust, peak_kind = measured_peaks()
+    sf, sb, ff, fb = flops(wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL)
+    ms_step = ms / args.steps
+    tokens = wl.B * wl.T * world
+    value = tokens / (ms_step / 1e3)
+    op_ms = {name: statistics.median(v) for name, v in per_op.items()}
+    sparse_ms = op_ms["sparse_fwd"] + op_ms["sparse_bwd"]
+    full_ms = op_ms["full_fwd"] + op_ms["full_bwd"]
+    op_flops = {"full_fwd": ff, "full_bwd": fb, "sparse_fwd": sf, "sparse_bwd": sb}
+    dominant = max(op_ms, key=op_ms.get)
+    traffic = None
+    roof = {"kernel": "ssa_%s call" % dominant, "bound": "tensor",
+            "achieved": op_flops.get(dominant, 0.0) / (op_ms[dominant] / 1e3) / 1e12, "peak": peak_sust,
+            "unit": "TFLOP/s", "traffic": traffic,
+            "peak_basis": "%s bf16 dense, sustained (kernel timed inside a long step)" % peak_kind}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_block(wl),
+        "sparse_attn": {"fwd_bwd_ms": sparse_ms, "tflops": (sf + sb) / (sparse_ms / 1e3) / 1e12,
+                        "frac_of_peak": (sf + sb) / (sparse_ms / 1e3) / 1e12 / peak_sust,
+                        "frac_of_burst_peak": (sf + sb) / (sparse_ms / 1e3) / 1e12 / peak_burst,
+                        "tokens_per_s": wl.B * wl.T / (sparse_ms / 1e3), "flop_per_step": sf + sb},
+        "full_attn": {"fwd_bwd_ms": full_ms, "tflops": (ff + fb) / (full_ms / 1e3) / 1e12,
+                      "frac_of_peak": (ff + fb) / (full_ms / 1e3) / 1e12 / peak_sust},
+        "op_ms": op_ms,
+        "select_hbm": {"gbs": (wl.B * wl.H * wl.T * (2 * wl.d + 4 * K_SEL)) / (op_ms["select"] / 1e3) / 1e9,
+                       "frac": (wl.B * wl.H * wl.T * (2 * wl.d + 4 * K_SEL)) / (op_ms["select"] / 1e3) / 1e9 / hbm},
+        "pool_hbm": {"gbs": (wl.B * wl.H * wl.T * 2 * wl.d) / (op_ms["pool"] / 1e3) / 1e9,
+                     "frac": (wl.B * wl.H * wl.T * 2 * wl.d) / (op_ms["pool"] / 1e3) / 1e9 / hbm},
+        "roofline": roof,
+        "e2e": {"value": tokens / (e_ms / args.steps / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": sum(host[k].numel() * 2 for k in host), "d2h_bytes_per_step": 4},
+        "gpu_launches": args.steps * (ops.SSAStep.KERNELS_FWD + ops.SSAStep.KERNELS_BWD),
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        try:
+            import oracle
+            oracle.build()
+            dt, fl, desc = oracle_sample(args.ref_tokens)
+            full_fl = sf + sb + ff + fb
+            line["cpu_baseline"] = {"value": wl.B * wl.T / (dt * full_fl / fl), "unit": "tokens/s",
+                                    "cores": oracle.num_threads(), "kind": "oracle",
+                                    "sample": desc + "; %.2f s, scaled to the full step by algorithmic FLOPs" % dt}
+        except Exception as e:  # the baseline never blocks the GPU number
+            line["cpu_baseline"] = {"value": None, "unit": "tokens/s", "cores": None, "kind": "oracle",
+                                    "sample": "failed: %s" % e}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-tokens", type=int, default=4096, help="prefix length of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

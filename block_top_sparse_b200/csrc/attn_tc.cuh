@@ -1,0 +1,739 @@
+// attn_tc.cuh -- tcgen05 (5th-generation tensor core) attention kernels for
+// head dimension 128, bf16 inputs, fp32 accumulation in tensor memory.
+//
+//  full_fwd_kernel    full causal attention forward, query-major: one CTA per
+//                     128-query tile, loops over the causal key tiles with an
+//                     online softmax (paper section 3, full attention).
+//  sparse_fwd_kernel  block-major sparse forward: one CTA per (head, key block
+//                     j) processes, 128 at a time, the queries whose selection
+//                     holds j (gathered by row), and writes a normalised
+//                     partial output + log-sum-exp per (query, slot); a merge
+//                     kernel combines the k partials of each query.
+//  attn_bwd_kernel    backward for both streams, key-block-outer: one CTA per
+//                     key tile (full) or key block (sparse) keeps K_j, V_j and
+//                     the transposed dK_j, dV_j accumulators resident and loops
+//                     over the query rows that attend to it; dQ is accumulated
+//                     with fp32 vector atomics.
+//
+// Shared-memory operand tiles are "chunks" of R rows x 64 bf16 (128 B rows,
+// 128-byte swizzle), see smem_desc_sw128().  Warps 0..3 (128 threads) own one
+// tile row each (a query row, or in the backward epilogue a head-dim row);
+// warp 4 issues TMA and MMA.
+#pragma once
+
+#include "device.cuh"
+
+namespace ssa {
+
+constexpr int kD = 128;         // head dimension of the tensor-core path
+constexpr int kTileQ = 128;     // query rows per tile (MMA M)
+constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16
+
+struct Rows {
+    // Row source of a query tile: contiguous (full attention) or gathered from
+    // the inverse selection index (sparse attention).
+    const int32_t *list;  // entries t*k + slot, or nullptr for contiguous rows
+    int len;              // number of rows in the list / valid rows overall
+    int first;            // contiguous: first query position
+    int k;
+};
+
+// Query position and global selection entry of tile row r of tile `it`.
+__device__ __forceinline__ bool tile_row(const Rows &R, int T, int it, int r, int &t, int &entry) {
+    if (R.list) {
+        const int li = it * kTileQ + r;
+        if (li >= R.len) return false;
+        entry = __ldg(R.list + li);
+        t = entry / R.k;
+        return true;
+    }
+    t = R.first + it * kTileQ + r;
+    entry = -1;
+    return t < T;
+}
+
+// cp.async one 256-byte row (128 bf16) into row r of a 2-chunk swizzled tile.
+// Invalid rows are zero-filled (source size 0).
+__device__ __forceinline__ void gather_row(uint32_t tile, const __nv_bfloat16 *src, bool valid, int r) {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        const uint32_t dst = tile + (u >> 3) * kChunkBytes + r * 128 + ((((u & 7) ^ (r & 7)) & 7) << 4);
+        cp_async_16(dst, src + u * 8, valid ? 16u : 0u);
+    }
+}
+
+// Write 32 fp32 values as bf16 into row r, columns [c0, c0+32) of a swizzled
+// multi-chunk tile (chunk = 64 columns, chunk stride `cstride` bytes).
+__device__ __forceinline__ void store_row32_bf16(uint32_t tile, uint32_t cstride, int r, int c0, const float (&v)[32]) {
+    const uint32_t base = tile + (c0 >> 6) * cstride + r * 128;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        const uint32_t unit = ((c0 & 63) >> 3) + g;
+        const uint32_t addr = base + (((unit ^ (r & 7)) & 7) << 4);
+        st_shared_v4(addr, pack_bf16x2(v[8 * g + 0], v[8 * g + 1]), pack_bf16x2(v[8 * g + 2], v[8 * g + 3]),
+                     pack_bf16x2(v[8 * g + 4], v[8 * g + 5]), pack_bf16x2(v[8 * g + 6], v[8 * g + 7]));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// MMA sequences (issued by one thread).
+// ---------------------------------------------------------------------------
+
+// D[128 x N] = A[128 x 128] * B[N x 128]^T with A, B K-major over K = 128
+// (two 64-wide chunks each; A chunk stride 16 KB, B chunk stride b_cstride).
+__device__ __forceinline__ void mma_k128_kmajor(uint32_t d_tmem, uint32_t a, uint32_t b, uint32_t b_cstride,
+                                                uint32_t idesc) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t da = smem_desc_sw128(a + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16);
+        const uint64_t db = smem_desc_sw128(b + (kk >> 2) * b_cstride + (kk & 3) * 32, 16);
+        mma_bf16_ss(d_tmem, da, db, idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Full causal attention forward.
+// grid = (ceil(T/128), B*H); block = 192 threads.
+// smem: Q 32 KB | K[2] 64 KB | V[2] 64 KB | P 32 KB | barriers
+// tmem: S[2] at columns 0 / 128, O at 256 (512 allocated).
+// ---------------------------------------------------------------------------
+struct FullFwdSmem {
+    static constexpr int kQ = 0;
+    static constexpr int kK = kQ + 2 * kChunkBytes;
+    static constexpr int kV = kK + 2 * 2 * kChunkBytes;
+    static constexpr int kP = kV + 2 * 2 * kChunkBytes;
+    static constexpr int kBar = kP + 2 * kChunkBytes;
+    static constexpr int kTotal = kBar + 256;
+};
+
+__global__ void __launch_bounds__(192, 1)
+    full_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ O, float *__restrict__ lse,
+                    int T, float scale_log2) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + FullFwdSmem::kBar);
+    uint64_t *bar_q = bars + 0;
+    uint64_t *bar_kv_full = bars + 1;   // [2]
+    uint64_t *bar_kv_empty = bars + 3;  // [2]
+    uint64_t *bar_s_full = bars + 5;    // [2]
+    uint64_t *bar_p_full = bars + 7;
+    uint64_t *bar_o_full = bars + 8;
+    uint64_t *bar_final = bars + 9;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 12);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 13);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nq = (T + kTileQ - 1) / kTileQ;
+    const int m = nq - 1 - blockIdx.x;  // heaviest tiles first
+    const int bh = blockIdx.y;
+    const int row0 = bh * T;            // first tensor-map row of this head
+    const int nkv = m + 1;              // causal key tiles 0..m
+
+    const uint32_t sQ = smem_u32(smem + FullFwdSmem::kQ);
+    const uint32_t sK = smem_u32(smem + FullFwdSmem::kK);
+    const uint32_t sV = smem_u32(smem + FullFwdSmem::kV);
+    const uint32_t sP = smem_u32(smem + FullFwdSmem::kP);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_kv_full + i, 1);
+            mbar_init(bar_kv_empty + i, 1);
+            mbar_init(bar_s_full + i, 1);
+        }
+        mbar_init(bar_p_full, 128);
+        mbar_init(bar_o_full, 1);
+        mbar_init(bar_final, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS0 = tmem, tO = tmem + 256;
+
+    if (warp == 5) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar_q, 2 * kChunkBytes);
+            tma_load_2d(&tmQ, bar_q, smem + FullFwdSmem::kQ, 0, row0 + m * kTileQ);
+            tma_load_2d(&tmQ, bar_q, smem + FullFwdSmem::kQ + kChunkBytes, 64, row0 + m * kTileQ);
+            for (int n = 0; n < nkv; ++n) {
+                const int st = n & 1;
+                if (n >= 2 && !mbar_wait(bar_kv_empty + st, ((n >> 1) - 1) & 1, abort_flag, 0x101)) break;
+                mbar_arrive_expect_tx(bar_kv_full + st, 4 * kChunkBytes);
+                uint8_t *k = smem + FullFwdSmem::kK + st * 2 * kChunkBytes;
+                uint8_t *v = smem + FullFwdSmem::kV + st * 2 * kChunkBytes;
+                tma_load_2d(&tmK, bar_kv_full + st, k, 0, row0 + n * kTileQ);
+                tma_load_2d(&tmK, bar_kv_full + st, k + kChunkBytes, 64, row0 + n * kTileQ);
+                tma_load_2d(&tmV, bar_kv_full + st, v, 0, row0 + n * kTileQ);
+                tma_load_2d(&tmV, bar_kv_full + st, v + kChunkBytes, 64, row0 + n * kTileQ);
+            }
+        }
+    } else if (warp == 4) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t idS = idesc_bf16(128, 128, false, false);
+            const uint32_t idO = idesc_bf16(128, 128, false, true);
+            bool ok = mbar_wait(bar_q, 0, abort_flag, 0x102) && mbar_wait(bar_kv_full, 0, abort_flag, 0x103);
+            if (ok) {
+                tc_fence_after();
+                mma_k128_kmajor(tS0, sQ, sK, kChunkBytes, idS);
+                mma_commit(bar_s_full);
+            }
+            for (int n = 0; ok && n < nkv; ++n) {
+                const int st = n & 1;
+                if (n + 1 < nkv) {
+                    const int s1 = (n + 1) & 1;
+                    if (!mbar_wait(bar_kv_full + s1, ((n + 1) >> 1) & 1, abort_flag, 0x104)) break;
+                    tc_fence_after();
+                    mma_k128_kmajor(tmem + s1 * 128, sQ, sK + s1 * 2 * kChunkBytes, kChunkBytes, idS);
+                    mma_commit(bar_s_full + s1);
+                }
+                if (!mbar_wait(bar_p_full, n & 1, abort_flag, 0x105)) break;
+                tc_fence_after();
+                // O += P V : A = P [128 q x 128 kv] K-major, B = V [kv rows x d] MN-major.
+                const uint32_t vb = sV + st * 2 * kChunkBytes;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t da = smem_desc_sw128(sP + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16);
+                    const uint64_t db = smem_desc_sw128(vb + kk * 2048, kChunkBytes);
+                    mma_bf16_ss(tO, da, db, idO, (n > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bar_o_full);
+                mma_commit(bar_kv_empty + st);
+            }
+            mma_commit(bar_final);
+            mbar_wait(bar_final, 0, abort_flag, 0x106);
+        }
+    } else {
+        // ---------------- softmax warps (thread r <-> query row r) ----------------
+        const int r = threadIdx.x;
+        const int t = m * kTileQ + r;
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        float m_used = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int n = 0; n < nkv; ++n) {
+            const int sb = n & 1;
+            if (!mbar_wait(bar_s_full + sb, (n >> 1) & 1, abort_flag, 0x107)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tS = tmem + sb * 128 + lane_off;
+            const bool diag = (n == m);
+            // pass 1: row maximum (log2 domain)
+            float mx = -INFINITY;
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+                float v[32];
+                tmem_ld32(tS + c0, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int kv = n * kTileQ + c0 + i;
+                    const float x = (diag && kv > t) ? -INFINITY : v[i] * scale_log2;
+                    mx = fmaxf(mx, x);
+                }
+            }
+            float alpha = 1.f;
+            if (n == 0) {
+                m_used = mx;
+            } else if (mx > m_used + 8.f) {
+                alpha = fast_exp2(m_used - mx);
+                m_used = mx;
+            }
+            if (n > 0) {
+                // PV of the previous tile must be done before P is overwritten / O rescaled.
+                if (!mbar_wait(bar_o_full, (n - 1) & 1, abort_flag, 0x108)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                    for (int c0 = 0; c0 < 128; c0 += 32) {
+                        float o[32];
+                        tmem_ld32(tO + lane_off + c0, o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                        tmem_st32(tO + lane_off + c0, o);
+                    }
+                }
+            }
+            l *= alpha;
+            // pass 2: probabilities -> P (bf16) in shared memory
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+                float v[32];
+                tmem_ld32(tS + c0, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int kv = n * kTileQ + c0 + i;
+                    const float p = (diag && kv > t) ? 0.f : fast_exp2(v[i] * scale_log2 - m_used);
+                    l += p;
+                    v[i] = p;
+                }
+                store_row32_bf16(sP, kChunkBytes, r, c0, v);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar_p_full);
+        }
+        if (ok && mbar_wait(bar_o_full, (nkv - 1) & 1, abort_flag, 0x109)) {
+            tc_fence_after();
+            const float inv_l = 1.f / l;
+            const bool valid = t < T;
+            __nv_bfloat16 *dst = O + (static_cast<size_t>(row0) + (valid ? t : 0)) * kD;
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+                float o[32];
+                tmem_ld32(tO + lane_off + c0, o);  // warp-collective: outside the per-row branch
+                if (valid) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + c0);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        d4[g] = make_uint4(pack_bf16x2(o[8 * g] * inv_l, o[8 * g + 1] * inv_l),
+                                           pack_bf16x2(o[8 * g + 2] * inv_l, o[8 * g + 3] * inv_l),
+                                           pack_bf16x2(o[8 * g + 4] * inv_l, o[8 * g + 5] * inv_l),
+                                           pack_bf16x2(o[8 * g + 6] * inv_l, o[8 * g + 7] * inv_l));
+                }
+            }
+            if (valid) lse[static_cast<size_t>(row0) + t] = (m_used + __log2f(l)) * kLn2;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
+// Sparse forward, block-major.
+// grid = (B*H*nb): unit u -> block j = u / BH, head bh = u % BH.  block = 160.
+// For every tile of the block's query list: S = Q_g K_j^T, masked softmax over
+// the block's NKV keys, O = P V_j, partial (o / l, lse) stored per entry.
+// smem: Q 32 KB | K NKV*256 | V NKV*256 | P (NKV/64)*16 KB | barriers
+// tmem: S at 0, O at 128 (256 allocated).
+// ---------------------------------------------------------------------------
+template <int NKV>
+struct SparseFwdSmem {
+    static constexpr int kQ = 0;
+    static constexpr int kK = kQ + 2 * kChunkBytes;
+    static constexpr int kV = kK + 2 * NKV * 128;
+    static constexpr int kP = kV + 2 * NKV * 128;
+    static constexpr int kBar = kP + (NKV / 64) * kChunkBytes;
+    static constexpr int kTotal = kBar + 256;
+};
+
+template <int NKV>
+__global__ void __launch_bounds__(160, 1)
+    sparse_fwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      const __nv_bfloat16 *__restrict__ Q, const int32_t *__restrict__ entries,
+                      const int32_t *__restrict__ lstart, const int32_t *__restrict__ llen,
+                      __nv_bfloat16 *__restrict__ Opart, float *__restrict__ lsepart, int BH, int T, int k,
+                      int nb, float scale_log2) {
+    using L = SparseFwdSmem<NKV>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
+    uint64_t *bar_kv = bars + 0, *bar_q_full = bars + 1, *bar_s_full = bars + 2, *bar_p_full = bars + 3;
+    uint64_t *bar_o_full = bars + 4, *bar_o_empty = bars + 5, *bar_final = bars + 6;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 9);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j = blockIdx.x / BH, bh = blockIdx.x % BH;
+    const int kv0 = j * NKV;
+    const size_t head_rows = static_cast<size_t>(bh) * T;
+    Rows R;
+    R.list = entries + head_rows * k + lstart[bh * nb + j];
+    R.len = llen[bh * nb + j];
+    R.first = 0;
+    R.k = k;
+    const int ntiles = (R.len + kTileQ - 1) / kTileQ;
+
+    const uint32_t sQ = smem_u32(smem + L::kQ), sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV),
+                   sP = smem_u32(smem + L::kP);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_kv, 1);
+        mbar_init(bar_q_full, 128);
+        mbar_init(bar_s_full, 1);
+        mbar_init(bar_p_full, 128);
+        mbar_init(bar_o_full, 1);
+        mbar_init(bar_o_empty, 128);
+        mbar_init(bar_final, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tO = tmem + 128;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar_kv, 4 * NKV * 128);
+            tma_load_2d(&tmK, bar_kv, smem + L::kK, 0, static_cast<int>(head_rows) + kv0);
+            tma_load_2d(&tmK, bar_kv, smem + L::kK + NKV * 128, 64, static_cast<int>(head_rows) + kv0);
+            tma_load_2d(&tmV, bar_kv, smem + L::kV, 0, static_cast<int>(head_rows) + kv0);
+            tma_load_2d(&tmV, bar_kv, smem + L::kV + NKV * 128, 64, static_cast<int>(head_rows) + kv0);
+            const uint32_t idS = idesc_bf16(128, NKV, false, false);
+            const uint32_t idO = idesc_bf16(128, 128, false, true);
+            bool ok = mbar_wait(bar_kv, 0, abort_flag, 0x201);
+            for (int it = 0; ok && it < ntiles; ++it) {
+                if (!mbar_wait(bar_q_full, it & 1, abort_flag, 0x202)) break;
+                if (it > 0 && !mbar_wait(bar_o_empty, (it - 1) & 1, abort_flag, 0x203)) break;
+                tc_fence_after();
+                mma_k128_kmajor(tS, sQ, sK, NKV * 128, idS);
+                mma_commit(bar_s_full);
+                if (!mbar_wait(bar_p_full, it & 1, abort_flag, 0x204)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < NKV / 16; ++kk) {
+                    const uint64_t da = smem_desc_sw128(sP + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16);
+                    const uint64_t db = smem_desc_sw128(sV + kk * 2048, NKV * 128);
+                    mma_bf16_ss(tO, da, db, idO, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar_o_full);
+            }
+            mma_commit(bar_final);
+            mbar_wait(bar_final, 0, abort_flag, 0x205);
+        }
+    } else {
+        const int r = threadIdx.x;
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        int t = 0, e = 0;
+        bool valid = ntiles > 0 && tile_row(R, T, 0, r, t, e);
+        gather_row(sQ, Q + (head_rows + (valid ? t : 0)) * kD, valid, r);
+        cp_async_commit();
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        mbar_arrive(bar_q_full);
+        for (int it = 0; it < ntiles; ++it) {
+            if (!mbar_wait(bar_s_full, it & 1, abort_flag, 0x206)) break;
+            tc_fence_after();
+            float mx = -INFINITY;
+            for (int c0 = 0; c0 < NKV; c0 += 32) {
+                float v[32];
+                tmem_ld32(tS + lane_off + c0, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const bool keep = valid && (kv0 + c0 + i <= t);
+                    mx = fmaxf(mx, keep ? v[i] * scale_log2 : -INFINITY);
+                }
+            }
+            const float mref = (mx == -INFINITY) ? 0.f : mx;
+            float l = 0.f;
+            for (int c0 = 0; c0 < NKV; c0 += 32) {
+                float v[32];
+                tmem_ld32(tS + lane_off + c0, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const bool keep = valid && (kv0 + c0 + i <= t);
+                    const float p = keep ? fast_exp2(v[i] * scale_log2 - mref) : 0.f;
+                    l += p;
+                    v[i] = p;
+                }
+                store_row32_bf16(sP, kChunkBytes, r, c0, v);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar_p_full);
+            if (!mbar_wait(bar_o_full, it & 1, abort_flag, 0x207)) break;
+            tc_fence_after();
+            // prefetch the next tile's query rows (S of this tile is complete)
+            int t_next = 0, e_next = 0;
+            bool valid_next = false;
+            if (it + 1 < ntiles) {
+                valid_next = tile_row(R, T, it + 1, r, t_next, e_next);
+                gather_row(sQ, Q + (head_rows + (valid_next ? t_next : 0)) * kD, valid_next, r);
+                cp_async_commit();
+            }
+            const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+            __nv_bfloat16 *dst = Opart + (head_rows * k + (valid ? e : 0)) * kD;
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+                float o[32];
+                tmem_ld32(tO + lane_off + c0, o);
+                if (valid) {
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + c0);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        d4[g] = make_uint4(pack_bf16x2(o[8 * g] * inv_l, o[8 * g + 1] * inv_l),
+                                           pack_bf16x2(o[8 * g + 2] * inv_l, o[8 * g + 3] * inv_l),
+                                           pack_bf16x2(o[8 * g + 4] * inv_l, o[8 * g + 5] * inv_l),
+                                           pack_bf16x2(o[8 * g + 6] * inv_l, o[8 * g + 7] * inv_l));
+                }
+            }
+            if (valid) lsepart[head_rows * k + e] = (l > 0.f) ? (mref + __log2f(l)) * kLn2 : -INFINITY;
+            tc_fence_before();
+            mbar_arrive(bar_o_empty);
+            if (it + 1 < ntiles) {
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                mbar_arrive(bar_q_full);
+                t = t_next;
+                e = e_next;
+                valid = valid_next;
+            }
+        }
+        cp_async_wait_all();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------------------
+// Backward for full (NKV = 128, contiguous query tiles) and sparse (gathered
+// query rows of key block j) attention.
+// grid: full   -> (nkt * BH) units, u -> key tile n = u / BH, head bh = u % BH
+//       sparse -> (nb * BH) units,  u -> block j = u / BH,   head bh = u % BH
+// block = 160.  Per query tile:
+//   S = Q K^T, dP = dO V^T                       (thread r <-> query row r)
+//   P = exp(scale S - lse), dS = P (dP - D)      -> shared memory, bf16
+//   dV^T += dO^T P, dK^T += Q^T dS               (tensor memory, M = head dim)
+//   dQ = dS K  -> fp32 atomics into dQacc (scaled)
+// smem: Q 32 KB | dO 32 KB | K, V NKV*256 each | P, dS (NKV/64)*16 KB each
+// tmem: S / dQ at 0, dP at 128, dV^T at 256, dK^T at 384 (512 allocated).
+// ---------------------------------------------------------------------------
+template <int NKV>
+struct BwdSmem {
+    static constexpr int kQ = 0;
+    static constexpr int kdO = kQ + 2 * kChunkBytes;
+    static constexpr int kK = kdO + 2 * kChunkBytes;
+    static constexpr int kV = kK + 2 * NKV * 128;
+    static constexpr int kP = kV + 2 * NKV * 128;
+    static constexpr int kdS = kP + (NKV / 64) * kChunkBytes;
+    static constexpr int kBar = kdS + (NKV / 64) * kChunkBytes;
+    static constexpr int kTotal = kBar + 256;
+};
+
+struct BwdArgs {
+    const __nv_bfloat16 *Q, *dO;
+    const float *lse, *Dvec;
+    float *dQacc;
+    __nv_bfloat16 *dK, *dV;
+    const float *dK_in_f32;  // unused (reserved)
+    const int32_t *entries, *lstart, *llen;  // sparse only
+    int BH, T, k, nb, sparse, accumulate;
+    float scale, scale_log2;
+};
+
+template <int NKV>
+__global__ void __launch_bounds__(160, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const BwdArgs a) {
+    using L = BwdSmem<NKV>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
+    uint64_t *bar_kv = bars + 0, *bar_qdo_full = bars + 1, *bar_sdp_full = bars + 2, *bar_pds_full = bars + 3;
+    uint64_t *bar_dq_full = bars + 4, *bar_dq_empty = bars + 5, *bar_final = bars + 6;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 9);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = a.T;
+    const int kb = blockIdx.x / a.BH, bh = blockIdx.x % a.BH;
+    const int kv0 = kb * NKV;
+    const size_t head_rows = static_cast<size_t>(bh) * T;
+    Rows R;
+    int ntiles;
+    if (a.sparse) {
+        R.list = a.entries + head_rows * a.k + a.lstart[bh * a.nb + kb];
+        R.len = a.llen[bh * a.nb + kb];
+        R.first = 0;
+        ntiles = (R.len + kTileQ - 1) / kTileQ;
+    } else {
+        R.list = nullptr;
+        R.first = kv0;  // causal: query tiles from the key tile onward
+        R.len = T - kv0;
+        ntiles = (R.len + kTileQ - 1) / kTileQ;
+    }
+    R.k = a.k;
+
+    const uint32_t sQ = smem_u32(smem + L::kQ), sdO = smem_u32(smem + L::kdO), sK = smem_u32(smem + L::kK),
+                   sV = smem_u32(smem + L::kV), sP = smem_u32(smem + L::kP), sdS = smem_u32(smem + L::kdS);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_kv, 1);
+        mbar_init(bar_qdo_full, 128);
+        mbar_init(bar_sdp_full, 1);
+        mbar_init(bar_pds_full, 128);
+        mbar_init(bar_dq_full, 1);
+        mbar_init(bar_dq_empty, 128);
+        mbar_init(bar_final, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384, tdQ = tmem;
+
+    if (warp == 4) {
+        if (lane == 0) {
+            const int krow = static_cast<int>(head_rows) + kv0;
+            mbar_arrive_expect_tx(bar_kv, 4 * NKV * 128);
+            tma_load_2d(&tmK, bar_kv, smem + L::kK, 0, krow);
+            tma_load_2d(&tmK, bar_kv, smem + L::kK + NKV * 128, 64, krow);
+            tma_load_2d(&tmV, bar_kv, smem + L::kV, 0, krow);
+            tma_load_2d(&tmV, bar_kv, smem + L::kV + NKV * 128, 64, krow);
+            const uint32_t idS = idesc_bf16(128, NKV, false, false);   // S, dP
+            const uint32_t idT = idesc_bf16(128, NKV, true, true);     // dV^T, dK^T
+            const uint32_t idQ = idesc_bf16(128, 128, false, true);    // dQ
+            bool ok = mbar_wait(bar_kv, 0, abort_flag, 0x301);
+            for (int it = 0; ok && it < ntiles; ++it) {
+                if (!mbar_wait(bar_qdo_full, it & 1, abort_flag, 0x302)) break;
+                if (it > 0 && !mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x303)) break;
+                tc_fence_after();
+                mma_k128_kmajor(tS, sQ, sK, NKV * 128, idS);
+                mma_k128_kmajor(tdP, sdO, sV, NKV * 128, idS);
+                mma_commit(bar_sdp_full);
+                if (!mbar_wait(bar_pds_full, it & 1, abort_flag, 0x304)) break;
+                tc_fence_after();
+                // dV^T[d x kv] += dO^T P ; dK^T[d x kv] += Q^T dS   (K = 128 query rows)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t a_do = smem_desc_sw128(sdO + kk * 2048, kChunkBytes);
+                    const uint64_t b_p = smem_desc_sw128(sP + kk * 2048, kChunkBytes);
+                    mma_bf16_ss(tdV, a_do, b_p, idT, (it > 0 || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t a_q = smem_desc_sw128(sQ + kk * 2048, kChunkBytes);
+                    const uint64_t b_ds = smem_desc_sw128(sdS + kk * 2048, kChunkBytes);
+                    mma_bf16_ss(tdK, a_q, b_ds, idT, (it > 0 || kk > 0) ? 1u : 0u);
+                }
+                // dQ[q x d] = dS K   (K = NKV keys)
+#pragma unroll
+                for (int kk = 0; kk < NKV / 16; ++kk) {
+                    const uint64_t a_ds = smem_desc_sw128(sdS + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16);
+                    const uint64_t b_k = smem_desc_sw128(sK + kk * 2048, NKV * 128);
+                    mma_bf16_ss(tdQ, a_ds, b_k, idQ, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar_dq_full);
+            }
+            mma_commit(bar_final);
+            mbar_wait(bar_final, 0, abort_flag, 0x305);
+        }
+    } else {
+        const int r = threadIdx.x;
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        int t = 0, e = 0;
+        bool valid = ntiles > 0 && tile_row(R, T, 0, r, t, e);
+        gather_row(sQ, a.Q + (head_rows + (valid ? t : 0)) * kD, valid, r);
+        gather_row(sdO, a.dO + (head_rows + (valid ? t : 0)) * kD, valid, r);
+        cp_async_commit();
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        mbar_arrive(bar_qdo_full);
+        bool ok = true;
+        for (int it = 0; it < ntiles; ++it) {
+            const float lse2 = valid ? __ldg(a.lse + head_rows + t) * kLog2e : 0.f;
+            const float Dt = valid ? __ldg(a.Dvec + head_rows + t) : 0.f;
+            if (!mbar_wait(bar_sdp_full, it & 1, abort_flag, 0x306)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            for (int c0 = 0; c0 < NKV; c0 += 32) {
+                float sv[32], dp[32];
+                tmem_ld32(tS + lane_off + c0, sv);
+                tmem_ld32(tdP + lane_off + c0, dp);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int kv = kv0 + c0 + i;
+                    const bool keep = valid && kv <= t;
+                    const float p = keep ? fast_exp2(sv[i] * a.scale_log2 - lse2) : 0.f;
+                    sv[i] = p;
+                    dp[i] = p * (dp[i] - Dt);
+                }
+                store_row32_bf16(sP, kChunkBytes, r, c0, sv);
+                store_row32_bf16(sdS, kChunkBytes, r, c0, dp);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar_pds_full);
+            if (!mbar_wait(bar_dq_full, it & 1, abort_flag, 0x307)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            int t_next = 0, e_next = 0;
+            bool valid_next = false;
+            if (it + 1 < ntiles) {
+                valid_next = tile_row(R, T, it + 1, r, t_next, e_next);
+                const size_t src = head_rows + (valid_next ? t_next : 0);
+                gather_row(sQ, a.Q + src * kD, valid_next, r);
+                gather_row(sdO, a.dO + src * kD, valid_next, r);
+                cp_async_commit();
+            }
+            float *dq = a.dQacc + (head_rows + (valid ? t : 0)) * kD;
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+                float g[32];
+                tmem_ld32(tdQ + lane_off + c0, g);
+                if (valid) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        atomicAdd(reinterpret_cast<float4 *>(dq + c0) + q,
+                                  make_float4(g[4 * q] * a.scale, g[4 * q + 1] * a.scale, g[4 * q + 2] * a.scale,
+                                              g[4 * q + 3] * a.scale));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar_dq_empty);
+            if (it + 1 < ntiles) {
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                mbar_arrive(bar_qdo_full);
+                t = t_next;
+                e = e_next;
+                valid = valid_next;
+            }
+        }
+        cp_async_wait_all();
+        // Epilogue: thread r <-> head-dim row r of dV^T / dK^T; column c <-> key kv0 + c.
+        if (ok) {
+            for (int c0 = 0; c0 < NKV; c0 += 32) {
+                float gv[32], gk[32];
+                tmem_ld32(tdV + lane_off + c0, gv);
+                tmem_ld32(tdK + lane_off + c0, gk);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int kv = kv0 + c0 + i;
+                    if (kv < T) {
+                        const size_t off = (head_rows + kv) * kD + r;
+                        float vv = ntiles > 0 ? gv[i] : 0.f, kk = ntiles > 0 ? gk[i] * a.scale : 0.f;
+                        if (a.accumulate) {
+                            vv += __bfloat162float(a.dV[off]);
+                            kk += __bfloat162float(a.dK[off]);
+                        }
+                        a.dV[off] = __float2bfloat16_rn(vv);
+                        a.dK[off] = __float2bfloat16_rn(kk);
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace ssa

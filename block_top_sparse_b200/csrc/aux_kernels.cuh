@@ -1,0 +1,293 @@
+// aux_kernels.cuh -- bandwidth-bound helpers of the attention path:
+//   * inverse selection index (key block -> list of (query, slot) entries,
+//     ascending in query position), built deterministically in three passes;
+//   * merge of the block-major sparse forward's per-slot partial outputs;
+//   * backward pre/post-processing (D = rowsum(dO o O), dQ accumulator -> dQ);
+//   * bidirectional SmoothL1 alignment loss forward/backward (paper section 5);
+//   * dropped attention mass delta = 1 - exp(lse_s - lse_f) (section 4.2).
+#pragma once
+
+#include "device.cuh"
+#include "pool_select.cuh"
+
+namespace ssa {
+
+constexpr int kIdxChunk = 256;  // queries per counting chunk
+
+// Pass 1: cnt[bh][c][j] = number of entries of block j among queries of chunk c.
+__global__ void __launch_bounds__(256) index_count_kernel(const int32_t *__restrict__ idx, int *__restrict__ cnt,
+                                                          int T, int k, int nb, int nch) {
+    extern __shared__ int hcount[];
+    const int bh = blockIdx.y, c = blockIdx.x;
+    for (int j = threadIdx.x; j < nb; j += blockDim.x) hcount[j] = 0;
+    __syncthreads();
+    const int t0 = c * kIdxChunk;
+    const int n = min(kIdxChunk, T - t0) * k;
+    const int32_t *src = idx + (static_cast<size_t>(bh) * T + t0) * k;
+    for (int e = threadIdx.x; e < n; e += blockDim.x) {
+        const int j = __ldg(src + e);
+        if (j >= 0 && j < nb) atomicAdd(&hcount[j], 1);
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < nb; j += blockDim.x) cnt[(static_cast<size_t>(bh) * nch + c) * nb + j] = hcount[j];
+}
+
+// Pass 2 (one CTA per head): per-chunk write offsets (in place over cnt),
+// list start and length of every block within the head's entry region.
+__global__ void __launch_bounds__(1024) index_scan_kernel(int *__restrict__ cnt, int *__restrict__ lstart,
+                                                          int *__restrict__ llen, int nb, int nch) {
+    __shared__ int warp_tot[32];
+    __shared__ int carry;
+    const int bh = blockIdx.x;
+    int *base = cnt + static_cast<size_t>(bh) * nch * nb;
+    if (threadIdx.x == 0) carry = 0;
+    __syncthreads();
+    for (int j0 = 0; j0 < nb; j0 += blockDim.x) {
+        const int j = j0 + threadIdx.x;
+        int total = 0;
+        if (j < nb) {
+            for (int c = 0; c < nch; ++c) {
+                const int v = base[static_cast<size_t>(c) * nb + j];
+                base[static_cast<size_t>(c) * nb + j] = total;
+                total += v;
+            }
+        }
+        // exclusive scan of totals over j (block-wide)
+        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+        int incl = total;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) warp_tot[w] = incl;
+        __syncthreads();
+        if (w == 0) {
+            int x = (lane < static_cast<int>(blockDim.x >> 5)) ? warp_tot[lane] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += v;
+            }
+            warp_tot[lane] = x;  // inclusive over warps
+        }
+        __syncthreads();
+        const int start = carry + (w > 0 ? warp_tot[w - 1] : 0) + incl - total;
+        if (j < nb) {
+            lstart[bh * nb + j] = start;
+            llen[bh * nb + j] = total;
+            for (int c = 0; c < nch; ++c) base[static_cast<size_t>(c) * nb + j] += start;
+        }
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) carry = start + total;
+        __syncthreads();
+    }
+}
+
+// Pass 3: one warp per chunk writes entries t*k + slot at their final position,
+// in ascending query order (ranks within a 32-query step come from lane bitmasks).
+__global__ void __launch_bounds__(128) index_fill_kernel(const int32_t *__restrict__ idx,
+                                                         const int *__restrict__ off, int32_t *__restrict__ entries,
+                                                         int T, int k, int nb, int nch) {
+    extern __shared__ int sm_fill[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y, c = blockIdx.x * 4 + warp;
+    uint32_t *bits = reinterpret_cast<uint32_t *>(sm_fill) + warp * 2 * nb;
+    int *run = sm_fill + warp * 2 * nb + nb;
+    if (c < nch) {
+        for (int j = lane; j < nb; j += 32) {
+            bits[j] = 0u;
+            run[j] = off[(static_cast<size_t>(bh) * nch + c) * nb + j];
+        }
+    }
+    __syncwarp();
+    if (c >= nch) return;
+    int32_t *dst = entries + static_cast<size_t>(bh) * T * k;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const int t_end = min(T, (c + 1) * kIdxChunk);
+    for (int tb = c * kIdxChunk; tb < t_end; tb += 32) {
+        const int t = tb + lane;
+        const bool valid = t < t_end;
+        const int32_t *row = idx + (static_cast<size_t>(bh) * T + t) * k;
+        for (int i = 0; i < k; ++i) {
+            const int j = valid ? __ldg(row + i) : -1;
+            if (j >= 0 && j < nb) atomicOr(&bits[j], 1u << lane);
+        }
+        __syncwarp();
+        for (int i = 0; i < k; ++i) {
+            const int j = valid ? __ldg(row + i) : -1;
+            if (j >= 0 && j < nb) dst[run[j] + __popc(bits[j] & lt_mask)] = t * k + i;
+        }
+        __syncwarp();
+        for (int i = 0; i < k; ++i) {
+            const int j = valid ? __ldg(row + i) : -1;
+            if (j >= 0 && j < nb) {
+                const uint32_t b = bits[j];
+                if (b != 0u && lane == __ffs(b) - 1) {
+                    run[j] += __popc(b);
+                    bits[j] = 0u;
+                }
+            }
+        }
+        __syncwarp();
+    }
+}
+
+// Merge of the per-slot partials: one warp per query row, 4 columns per lane.
+//   lse = log sum_i exp(lse_i),  o = sum_i exp(lse_i - lse) o_i
+template <typename TO>
+__global__ void __launch_bounds__(256) sparse_merge_kernel(const int32_t *__restrict__ idx,
+                                                           const __nv_bfloat16 *__restrict__ Opart,
+                                                           const float *__restrict__ lsepart, TO *__restrict__ O,
+                                                           float *__restrict__ lse, size_t rows, int k) {
+    const size_t row = static_cast<size_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const int32_t *sel = idx + row * k;
+    float mx = -INFINITY;
+    for (int i = 0; i < k; ++i)
+        if (__ldg(sel + i) >= 0) mx = fmaxf(mx, __ldg(lsepart + row * k + i));
+    float wsum = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < k; ++i) {
+        if (__ldg(sel + i) < 0) continue;
+        const float w = __expf(__ldg(lsepart + row * k + i) - mx);
+        wsum += w;
+        const uint2 u = __ldg(reinterpret_cast<const uint2 *>(Opart + (row * k + i) * 128) + lane);
+        acc[0] += w * __uint_as_float(u.x << 16);
+        acc[1] += w * __uint_as_float(u.x & 0xFFFF0000u);
+        acc[2] += w * __uint_as_float(u.y << 16);
+        acc[3] += w * __uint_as_float(u.y & 0xFFFF0000u);
+    }
+    const float inv = 1.f / wsum;
+    TO *dst = O + row * 128 + lane * 4;
+    if constexpr (sizeof(TO) == 2) {
+        *reinterpret_cast<uint2 *>(dst) =
+            make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+    } else {
+        *reinterpret_cast<float4 *>(dst) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    }
+    if (lane == 0) lse[row] = mx + __logf(wsum);
+}
+
+// D[row] = sum_c dO[row,c] * O[row,c] (one warp per row) and zero the fp32 dQ accumulator row.
+template <typename T>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const T *__restrict__ dO, const T *__restrict__ O,
+                                                       float *__restrict__ Dvec, float *__restrict__ dQacc,
+                                                       size_t rows, int d) {
+    const size_t row = static_cast<size_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float acc = 0.f;
+    for (int c = lane; c < d; c += 32) {
+        acc += to_f32(dO[row * d + c]) * to_f32(O[row * d + c]);
+        dQacc[row * d + c] = 0.f;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) Dvec[row] = acc;
+}
+
+// out = (accumulate ? out : 0) + acc, rounded once to T.
+template <typename T>
+__global__ void __launch_bounds__(256) acc_to_out_kernel(const float *__restrict__ acc, T *__restrict__ out,
+                                                         size_t n, int accumulate) {
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        float v = acc[i];
+        if (accumulate) v += to_f32(out[i]);
+        if constexpr (sizeof(T) == 2)
+            out[i] = __float2bfloat16_rn(v);
+        else
+            out[i] = v;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Alignment loss (paper section 5).  huber_beta is symmetric, so both
+// directions share sum_i huber(Of_i - Os_i):
+//   loss = (w_sparsity + w_commit) * sum / n
+// Pass 1: fixed grid of kAlignBlocks CTAs, per-CTA partial sums (fp32);
+// pass 2: one warp adds the partials in fixed order (fp64) -> deterministic.
+// ---------------------------------------------------------------------------
+constexpr int kAlignBlocks = 1184;  // 8 x 148 SMs
+
+__device__ __forceinline__ float huber(float x, float beta) {
+    const float a = fabsf(x);
+    return a < beta ? 0.5f * x * x / beta : a - 0.5f * beta;
+}
+
+__device__ __forceinline__ float huber_slope(float x, float beta) {
+    if (fabsf(x) < beta) return x / beta;
+    return x > 0.f ? 1.f : -1.f;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) align_fwd_partial_kernel(const T *__restrict__ Of, const T *__restrict__ Os,
+                                                                float *__restrict__ partial, size_t n, float beta) {
+    constexpr int V = Vec16<T>::N;
+    __shared__ float red[8];
+    float acc = 0.f;
+    const size_t nv = n / V;
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nv;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        float a[V], b[V];
+        Vec16<T>::load(Of + i * V, a);
+        Vec16<T>::load(Os + i * V, b);
+#pragma unroll
+        for (int q = 0; q < V; ++q) acc += huber(a[q] - b[q], beta);
+    }
+    if (blockIdx.x == 0)
+        for (size_t i = nv * V + threadIdx.x; i < n; i += blockDim.x) acc += huber(to_f32(Of[i]) - to_f32(Os[i]), beta);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float s = 0.f;
+        for (int w = 0; w < 8; ++w) s += red[w];
+        partial[blockIdx.x] = s;
+    }
+}
+
+__global__ void align_fwd_final_kernel(const float *__restrict__ partial, int nparts, float *__restrict__ loss,
+                                       double scale) {
+    const int lane = threadIdx.x;
+    double s = 0.0;
+    for (int i = lane; i < nparts; i += 32) s += partial[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) *loss = static_cast<float>(s * scale);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) align_bwd_kernel(const T *__restrict__ Of, const T *__restrict__ Os,
+                                                        const float *__restrict__ dloss, T *__restrict__ dOf,
+                                                        T *__restrict__ dOs, size_t n, float beta, float w_s,
+                                                        float w_c, int accumulate) {
+    const float g = __ldg(dloss) / static_cast<float>(n);
+    const float cf = g * w_s, cs = g * w_c;
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const float x = to_f32(Of[i]) - to_f32(Os[i]);
+        const float h = huber_slope(x, beta);
+        float gf = cf * h, gs = -cs * h;  // huber' is odd: huber'(Os - Of) = -huber'(Of - Os)
+        if (accumulate & 1) gf += to_f32(dOf[i]);
+        if (accumulate & 2) gs += to_f32(dOs[i]);
+        if constexpr (sizeof(T) == 2) {
+            dOf[i] = __float2bfloat16_rn(gf);
+            dOs[i] = __float2bfloat16_rn(gs);
+        } else {
+            dOf[i] = gf;
+            dOs[i] = gs;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) dropped_mass_kernel(const float *__restrict__ ls, const float *__restrict__ lf,
+                                                           float *__restrict__ delta, size_t n) {
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x)
+        delta[i] = -expm1f(ls[i] - lf[i]);
+}
+
+}  // namespace ssa

@@ -1,0 +1,255 @@
+// pool_select.cuh -- block pooling and per-query causal top-k block selection.
+//
+// Paper section 3: keys are partitioned into contiguous blocks of s tokens,
+// each block is mean-pooled, every strictly preceding block is scored against
+// the query (r_j = q . Kbar_j) and the top blocks are kept.  Reading used here:
+// the query's own block is always kept and counted within k; ties go to the
+// lower block index; rows are ascending with -1 padding at the end.
+#pragma once
+
+#include "device.cuh"
+
+namespace ssa {
+
+// 16-byte vector load of dtype T converted to fp32.
+template <typename T>
+struct Vec16;
+
+template <>
+struct Vec16<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&f)[8]) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+};
+
+template <>
+struct Vec16<float> {
+    static constexpr int N = 4;
+    __device__ __forceinline__ static void load(const float *p, float (&f)[4]) {
+        const float4 u = __ldg(reinterpret_cast<const float4 *>(p));
+        f[0] = u.x;
+        f[1] = u.y;
+        f[2] = u.z;
+        f[3] = u.w;
+    }
+};
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) {
+    return x;
+}
+
+// ---------------------------------------------------------------------------
+// Pooling: one CTA (256 threads) per (head, block).  Thread (row group g,
+// column vector c) sums rows g, g+G, ... in order; the G partial sums are then
+// added in fixed order and divided by s.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ K, float *__restrict__ Kbar, int T_len, int d,
+                                                   int s, int nb) {
+    constexpr int V = Vec16<T>::N;
+    __shared__ float part[256 * V];
+    const int tpr = d / V;                  // threads per row
+    const int G = blockDim.x / tpr;         // rows in flight
+    const int g = threadIdx.x / tpr, cv = threadIdx.x % tpr;
+    const int bh = blockIdx.x / nb, j = blockIdx.x % nb;
+    const T *base = K + (static_cast<size_t>(bh) * T_len + static_cast<size_t>(j) * s) * d + cv * V;
+    float acc[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] = 0.f;
+#pragma unroll 4
+    for (int r = g; r < s; r += G) {
+        float f[V];
+        Vec16<T>::load(base + static_cast<size_t>(r) * d, f);
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] += f[i];
+    }
+#pragma unroll
+    for (int i = 0; i < V; ++i) part[g * d + cv * V + i] = acc[i];
+    __syncthreads();
+    for (int c = threadIdx.x; c < d; c += blockDim.x) {
+        float sum = 0.f;
+        for (int q = 0; q < G; ++q) sum += part[q * d + c];
+        Kbar[(static_cast<size_t>(bh) * nb + j) * d + c] = sum / static_cast<float>(s);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Selection.  One CTA (256 threads) per 32 consecutive queries of one head
+// (all in the same block, since s is a multiple of 32).
+//   phase 1: scores S[q][j] = q . Kbar_j for j < b(t), fp32 FMA in column order,
+//            4 queries x 4 blocks per thread, Kbar staged 128 blocks at a time;
+//   phase 2: one warp per query: radix select of the (k-1)-th largest score
+//            on order-preserving 32-bit keys, then an ascending ballot
+//            compaction that keeps equal scores in index order.
+// ---------------------------------------------------------------------------
+constexpr int kSelQ = 32;
+constexpr int kSelJ = 128;
+
+__host__ __device__ constexpr size_t select_smem_bytes(int d, int nb) {
+    return (static_cast<size_t>(kSelQ + kSelJ) * (d + 4) + static_cast<size_t>(kSelQ) * nb) * 4 + 8 * 256 * 4;
+}
+
+__device__ __forceinline__ uint32_t order_key(float x) {
+    uint32_t u = __float_as_uint(x);
+    if (u == 0x80000000u) u = 0u;  // -0 ranks as +0
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) select_kernel(const T *__restrict__ Q, const float *__restrict__ Kbar,
+                                                     int32_t *__restrict__ idx, int T_len, int d, int s, int k,
+                                                     int nb) {
+    extern __shared__ __align__(16) float sm[];
+    const int dp = d + 4;
+    float *sQ = sm;                       // [32][dp]
+    float *sK = sQ + kSelQ * dp;          // [128][dp]
+    float *sS = sK + kSelJ * dp;          // [32][nb]
+    int *hist = reinterpret_cast<int *>(sS + kSelQ * nb);  // [8][256]
+
+    const int bh = blockIdx.y, t0 = blockIdx.x * kSelQ;
+    const int bt = t0 / s;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    for (int e = tid; e < kSelQ * d; e += blockDim.x) {
+        const int qi = e / d, c = e % d;
+        sQ[qi * dp + c] = to_f32(Q[(static_cast<size_t>(bh) * T_len + t0 + qi) * d + c]);
+    }
+    const int qg = tid >> 5;  // queries 4*qg .. 4*qg+3
+    for (int jc = 0; jc < bt; jc += kSelJ) {
+        const int nj = min(kSelJ, bt - jc);
+        __syncthreads();
+        for (int e = tid; e < nj * (d / 4); e += blockDim.x) {
+            const int jj = e / (d / 4), c4 = e % (d / 4);
+            *reinterpret_cast<float4 *>(sK + jj * dp + c4 * 4) =
+                __ldg(reinterpret_cast<const float4 *>(Kbar + (static_cast<size_t>(bh) * nb + jc + jj) * d) + c4);
+        }
+        __syncthreads();
+        float acc[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+        for (int c = 0; c < d; c += 4) {
+            float4 qv[4], kv[4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) qv[a] = *reinterpret_cast<const float4 *>(sQ + (4 * qg + a) * dp + c);
+#pragma unroll
+            for (int b = 0; b < 4; ++b) kv[b] = *reinterpret_cast<const float4 *>(sK + (lane + 32 * b) * dp + c);
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    acc[a][b] = fmaf(qv[a].x, kv[b].x, acc[a][b]);
+                    acc[a][b] = fmaf(qv[a].y, kv[b].y, acc[a][b]);
+                    acc[a][b] = fmaf(qv[a].z, kv[b].z, acc[a][b]);
+                    acc[a][b] = fmaf(qv[a].w, kv[b].w, acc[a][b]);
+                }
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int jj = lane + 32 * b;
+                if (jj < nj) sS[(4 * qg + a) * nb + jc + jj] = acc[a][b];
+            }
+    }
+    __syncthreads();
+
+    // phase 2: warp w selects for queries 4w .. 4w+3
+    int *h = hist + warp * 256;
+    const int want = min(k - 1, bt);
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int qq = 0; qq < 4; ++qq) {
+        const int qi = 4 * warp + qq;
+        const float *row = sS + qi * nb;
+        int32_t *out = idx + (static_cast<size_t>(bh) * T_len + t0 + qi) * k;
+        uint32_t tau = 0u;
+        int need_eq = 0;  // how many scores equal to tau are taken
+        if (want > 0 && want < bt) {
+            uint32_t prefix = 0u, mask = 0u;
+            int rank = want;  // want-th largest (1-based)
+            for (int shift = 24; shift >= 0; shift -= 8) {
+                for (int b = lane; b < 256; b += 32) h[b] = 0;
+                __syncwarp();
+                for (int jj = lane; jj < bt; jj += 32) {
+                    const uint32_t key = order_key(row[jj]);
+                    if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1);
+                }
+                __syncwarp();
+                int c8[8], sum = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    c8[i] = h[255 - 8 * lane - i];
+                    sum += c8[i];
+                }
+                int incl = sum;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                const int excl = incl - sum;
+                const bool here = excl < rank && rank <= incl;
+                const uint32_t who = __ballot_sync(0xffffffffu, here);
+                const int src = __ffs(who) - 1;
+                int digit = 0, new_rank = 0;
+                if (here) {
+                    int cum = excl;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        if (cum < rank && rank <= cum + c8[i]) {
+                            digit = 255 - 8 * lane - i;
+                            new_rank = rank - cum;
+                        }
+                        cum += c8[i];
+                    }
+                }
+                digit = __shfl_sync(0xffffffffu, digit, src);
+                rank = __shfl_sync(0xffffffffu, new_rank, src);
+                prefix |= static_cast<uint32_t>(digit) << shift;
+                mask |= 0xFFu << shift;
+                __syncwarp();
+            }
+            tau = prefix;
+            need_eq = rank;
+        }
+        int taken = 0, eq_seen = 0;
+        for (int j0 = 0; want > 0 && j0 < bt; j0 += 32) {
+            const int jj = j0 + lane;
+            const bool in = jj < bt;
+            const uint32_t key = in ? order_key(row[jj]) : 0u;
+            bool sel;
+            uint32_t eqb = 0u;
+            if (want < bt) {
+                const bool gt = in && key > tau;
+                const bool eq = in && key == tau;
+                eqb = __ballot_sync(0xffffffffu, eq);
+                sel = gt || (eq && (eq_seen + __popc(eqb & lt_mask)) < need_eq);
+            } else {
+                sel = in;
+            }
+            const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+            const int pos = taken + __popc(sb & lt_mask);
+            if (sel && pos < want) out[pos] = jj;
+            taken += __popc(sb);
+            eq_seen += __popc(eqb);
+        }
+        for (int i = want + lane; i < k; i += 32) out[i] = (i == want) ? bt : -1;
+    }
+}
+
+}  // namespace ssa

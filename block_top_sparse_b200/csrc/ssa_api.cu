@@ -1,0 +1,505 @@
+// ssa_api.cu -- the C ABI of libssa (declared in include/ssa.h): argument
+// validation, workspace carving, TMA descriptor set-up and kernel launches.
+// All kernels are compiled into this one translation unit.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "ssa.h"
+
+#include "device.cuh"
+#include "pool_select.cuh"
+#include "aux_kernels.cuh"
+#include "attn_simt.cuh"
+#include "attn_tc.cuh"
+
+using namespace ssa;
+
+namespace {
+
+struct Shape {
+    int B, H, T, d, s, k, dtype;
+    float scale;
+    size_t BH, rows;  // rows = B*H*T
+    int nb;
+    size_t esz;       // element size in bytes
+    bool tc;          // tensor-core path (bf16, d == 128)
+};
+
+ssa_status_t check_dims(const ssa_dims_t *dims, Shape &S, bool need_k) {
+    if (!dims) return SSA_ERR_INVALID_ARG;
+    S.B = dims->B;
+    S.H = dims->H;
+    S.T = dims->T;
+    S.d = dims->d;
+    S.s = dims->s;
+    S.k = dims->k;
+    S.dtype = dims->dtype;
+    S.scale = dims->scale;
+    if (S.B < 1 || S.H < 1 || S.T < 1 || S.d < 1 || S.s < 1) return SSA_ERR_INVALID_ARG;
+    if (S.dtype != SSA_DT_BF16 && S.dtype != SSA_DT_FP32) return SSA_ERR_INVALID_ARG;
+    if (!(std::isfinite(S.scale) && S.scale > 0.f)) return SSA_ERR_INVALID_ARG;
+    if (S.d != 64 && S.d != 128) return SSA_ERR_UNSUPPORTED;
+    if (S.s != 64 && S.s != 128) return SSA_ERR_UNSUPPORTED;
+    if (S.T % S.s != 0) return SSA_ERR_UNSUPPORTED;
+    S.BH = static_cast<size_t>(S.B) * S.H;
+    S.rows = S.BH * S.T;
+    if (S.rows > 0x7FFFFFFFull) return SSA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+    S.nb = S.T / S.s;
+    if (need_k) {
+        if (S.k < 1 || S.k > S.nb) return SSA_ERR_INVALID_ARG;
+        if (static_cast<int64_t>(S.T) * S.k > 0x7FFFFFFFll) return SSA_ERR_UNSUPPORTED;
+    }
+    S.esz = S.dtype == SSA_DT_BF16 ? 2 : 4;
+    S.tc = S.dtype == SSA_DT_BF16 && S.d == 128;
+    return SSA_OK;
+}
+
+inline size_t align_up(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace layout of the sparse index.
+struct IndexWs {
+    int *cnt, *lstart, *llen;
+    int32_t *entries;
+    int nch;
+};
+
+size_t index_bytes(const Shape &S) {
+    const size_t nch = (S.T + kIdxChunk - 1) / kIdxChunk;
+    return align_up(S.BH * nch * S.nb * 4) + 2 * align_up(S.BH * S.nb * 4) + align_up(S.rows * S.k * 4);
+}
+
+uint8_t *carve_index(const Shape &S, uint8_t *p, IndexWs &W) {
+    W.nch = (S.T + kIdxChunk - 1) / kIdxChunk;
+    W.cnt = reinterpret_cast<int *>(p);
+    p += align_up(S.BH * W.nch * S.nb * 4);
+    W.lstart = reinterpret_cast<int *>(p);
+    p += align_up(S.BH * S.nb * 4);
+    W.llen = reinterpret_cast<int *>(p);
+    p += align_up(S.BH * S.nb * 4);
+    W.entries = reinterpret_cast<int32_t *>(p);
+    p += align_up(S.rows * S.k * 4);
+    return p;
+}
+
+size_t ws_bytes_for(const Shape &S, int op) {
+    switch (op) {
+        case SSA_OP_SPARSE_FWD:
+            if (!S.tc) return 0;
+            return index_bytes(S) + align_up(S.rows * S.k * 128 * 2) + align_up(S.rows * S.k * 4);
+        case SSA_OP_SPARSE_BWD:
+        case SSA_OP_FULL_BWD: {
+            size_t b = align_up(S.rows * 4) + align_up(S.rows * S.d * 4);  // D, dQacc
+            if (!S.tc) b += 2 * align_up(S.rows * S.d * 4);                // dKacc, dVacc
+            if (op == SSA_OP_SPARSE_BWD && S.tc) b += index_bytes(S);
+            return b;
+        }
+        case SSA_OP_FULL_FWD:
+            return 0;
+        case SSA_OP_ALIGN_FWD:
+            return align_up(kAlignBlocks * 4);
+        default:
+            return 0;
+    }
+}
+
+ssa_status_t check_ws(const Shape &S, int op, const void *ws, size_t ws_bytes) {
+    const size_t need = ws_bytes_for(S, op);
+    if (need == 0) return SSA_OK;
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u)) return SSA_ERR_WORKSPACE;
+    return SSA_OK;
+}
+
+ssa_status_t launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptors: 2D view [rows, 128] of a bf16 tensor, box 64 columns x box_rows.
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+bool make_tmap(CUtensorMap *m, const void *base, size_t rows, int box_rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t gdim[2] = {128, rows};
+    const cuuint64_t gstride[1] = {128 * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estride[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), gdim, gstride, box, estride,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename K>
+bool set_smem(K kernel, size_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) ==
+           cudaSuccess;
+}
+
+unsigned grid_for(size_t n, unsigned per_block) {
+    size_t g = (n + per_block - 1) / per_block;
+    if (g > 148u * 32u) g = 148u * 32u;
+    return static_cast<unsigned>(g ? g : 1);
+}
+
+// Inverse selection index: entries of block j of head bh (query order).
+ssa_status_t build_index(const Shape &S, const int32_t *idx, IndexWs &W, cudaStream_t st) {
+    const size_t hbytes = static_cast<size_t>(S.nb) * 4;
+    if (!set_smem(index_count_kernel, hbytes)) return SSA_ERR_CUDA;
+    index_count_kernel<<<dim3(W.nch, S.BH), 256, hbytes, st>>>(idx, W.cnt, S.T, S.k, S.nb, W.nch);
+    index_scan_kernel<<<S.BH, 1024, 0, st>>>(W.cnt, W.lstart, W.llen, S.nb, W.nch);
+    const size_t fbytes = static_cast<size_t>(S.nb) * 8 * 4;
+    if (!set_smem(index_fill_kernel, fbytes)) return SSA_ERR_CUDA;
+    index_fill_kernel<<<dim3((W.nch + 3) / 4, S.BH), 128, fbytes, st>>>(idx, W.cnt, W.entries, S.T, S.k, S.nb,
+                                                                          W.nch);
+    return launch_status();
+}
+
+template <typename T>
+void launch_simt_fwd(const Shape &S, const void *Q, const void *K, const void *V, const int32_t *idx, void *O,
+                     float *lse, cudaStream_t st) {
+    const unsigned g = static_cast<unsigned>((S.rows + 7) / 8);
+    if (S.d == 64)
+        simt_fwd_kernel<T, 2><<<g, 256, 0, st>>>((const T *)Q, (const T *)K, (const T *)V, idx, (T *)O, lse, S.rows,
+                                                 S.T, S.s, S.k, S.scale);
+    else
+        simt_fwd_kernel<T, 4><<<g, 256, 0, st>>>((const T *)Q, (const T *)K, (const T *)V, idx, (T *)O, lse, S.rows,
+                                                 S.T, S.s, S.k, S.scale);
+}
+
+template <typename T>
+ssa_status_t simt_bwd(const Shape &S, const void *Q, const void *K, const void *V, const void *O, const float *lse,
+                      const void *dO, const int32_t *idx, void *dQ, void *dK, void *dV, int accumulate, void *ws,
+                      cudaStream_t st) {
+    uint8_t *p = static_cast<uint8_t *>(ws);
+    float *Dvec = reinterpret_cast<float *>(p);
+    p += align_up(S.rows * 4);
+    float *dQacc = reinterpret_cast<float *>(p);
+    p += align_up(S.rows * S.d * 4);
+    float *dKacc = reinterpret_cast<float *>(p);
+    p += align_up(S.rows * S.d * 4);
+    float *dVacc = reinterpret_cast<float *>(p);
+    const size_t n = S.rows * S.d;
+    if (cudaMemsetAsync(dKacc, 0, n * 4, st) != cudaSuccess || cudaMemsetAsync(dVacc, 0, n * 4, st) != cudaSuccess)
+        return SSA_ERR_CUDA;
+    const unsigned g = static_cast<unsigned>((S.rows + 7) / 8);
+    bwd_prep_kernel<T><<<g, 256, 0, st>>>((const T *)dO, (const T *)O, Dvec, dQacc, S.rows, S.d);
+    if (S.d == 64)
+        simt_bwd_kernel<T, 2><<<g, 256, 0, st>>>((const T *)Q, (const T *)K, (const T *)V, (const T *)dO, idx, lse,
+                                                 Dvec, dQacc, dKacc, dVacc, S.rows, S.T, S.s, S.k, S.scale);
+    else
+        simt_bwd_kernel<T, 4><<<g, 256, 0, st>>>((const T *)Q, (const T *)K, (const T *)V, (const T *)dO, idx, lse,
+                                                 Dvec, dQacc, dKacc, dVacc, S.rows, S.T, S.s, S.k, S.scale);
+    const unsigned ge = grid_for(n, 256);
+    acc_to_out_kernel<T><<<ge, 256, 0, st>>>(dQacc, (T *)dQ, n, accumulate);
+    acc_to_out_kernel<T><<<ge, 256, 0, st>>>(dKacc, (T *)dK, n, accumulate);
+    acc_to_out_kernel<T><<<ge, 256, 0, st>>>(dVacc, (T *)dV, n, accumulate);
+    return launch_status();
+}
+
+// Tensor-core backward shared by both streams.
+ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V, const void *O, const float *lse,
+                    const void *dO, const int32_t *idx, void *dQ, void *dK, void *dV, int accumulate, void *ws,
+                    cudaStream_t st) {
+    uint8_t *p = static_cast<uint8_t *>(ws);
+    float *Dvec = reinterpret_cast<float *>(p);
+    p += align_up(S.rows * 4);
+    float *dQacc = reinterpret_cast<float *>(p);
+    p += align_up(S.rows * S.d * 4);
+    const bool sparse = idx != nullptr;
+    IndexWs W{};
+    if (sparse) {
+        carve_index(S, p, W);
+        const ssa_status_t e = build_index(S, idx, W, st);
+        if (e != SSA_OK) return e;
+    }
+    const unsigned g = static_cast<unsigned>((S.rows + 7) / 8);
+    bwd_prep_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16 *)dO, (const __nv_bfloat16 *)O, Dvec,
+                                                       dQacc, S.rows, S.d);
+    const int nkv = sparse ? S.s : 128;
+    CUtensorMap tmK, tmV;
+    if (!make_tmap(&tmK, K, S.rows, nkv) || !make_tmap(&tmV, V, S.rows, nkv)) return SSA_ERR_CUDA;
+    BwdArgs a{};
+    a.Q = (const __nv_bfloat16 *)Q;
+    a.dO = (const __nv_bfloat16 *)dO;
+    a.lse = lse;
+    a.Dvec = Dvec;
+    a.dQacc = dQacc;
+    a.dK = (__nv_bfloat16 *)dK;
+    a.dV = (__nv_bfloat16 *)dV;
+    a.entries = W.entries;
+    a.lstart = W.lstart;
+    a.llen = W.llen;
+    a.BH = static_cast<int>(S.BH);
+    a.T = S.T;
+    a.k = S.k;
+    a.nb = S.nb;
+    a.sparse = sparse ? 1 : 0;
+    a.accumulate = accumulate;
+    a.scale = S.scale;
+    a.scale_log2 = S.scale * kLog2e;
+    const unsigned units = static_cast<unsigned>(S.BH * (sparse ? S.nb : (S.T + 127) / 128));
+    if (nkv == 128) {
+        const size_t sm = BwdSmem<128>::kTotal + 1024;
+        if (!set_smem(attn_bwd_kernel<128>, sm)) return SSA_ERR_CUDA;
+        attn_bwd_kernel<128><<<units, 160, sm, st>>>(tmK, tmV, a);
+    } else {
+        const size_t sm = BwdSmem<64>::kTotal + 1024;
+        if (!set_smem(attn_bwd_kernel<64>, sm)) return SSA_ERR_CUDA;
+        attn_bwd_kernel<64><<<units, 160, sm, st>>>(tmK, tmV, a);
+    }
+    const size_t n = S.rows * S.d;
+    acc_to_out_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, st>>>(dQacc, (__nv_bfloat16 *)dQ, n, accumulate);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ssa_workspace_size(const ssa_dims_t *dims, int op) {
+    Shape S;
+    const bool need_k = op == SSA_OP_SPARSE_FWD || op == SSA_OP_SPARSE_BWD;
+    if (check_dims(dims, S, need_k) != SSA_OK) return 0;
+    return ws_bytes_for(S, op);
+}
+
+ssa_status_t ssa_block_pool(const ssa_dims_t *dims, const void *K, float *Kbar, ssa_stream_t stream) {
+    Shape S;
+    ssa_status_t e = check_dims(dims, S, false);
+    if (e != SSA_OK) return e;
+    if (!K || !Kbar) return SSA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const unsigned g = static_cast<unsigned>(S.BH * S.nb);
+    if (S.dtype == SSA_DT_BF16)
+        pool_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16 *)K, Kbar, S.T, S.d, S.s, S.nb);
+    else
+        pool_kernel<float><<<g, 256, 0, st>>>((const float *)K, Kbar, S.T, S.d, S.s, S.nb);
+    return launch_status();
+}
+
+ssa_status_t ssa_block_select(const ssa_dims_t *dims, const void *Q, const float *Kbar, int32_t *idx,
+                              unsigned flags, ssa_stream_t stream) {
+    Shape S;
+    ssa_status_t e = check_dims(dims, S, true);
+    if (e != SSA_OK) return e;
+    if (!Q || !Kbar || !idx) return SSA_ERR_INVALID_ARG;
+    if (!(flags & SSA_SEL_FORCE_CURRENT) || (flags & ~static_cast<unsigned>(SSA_SEL_FORCE_CURRENT)))
+        return SSA_ERR_UNSUPPORTED;
+    const size_t sm = select_smem_bytes(S.d, S.nb);
+    if (S.nb > 1024 || sm > 227 * 1024) return SSA_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid(S.T / kSelQ, S.BH);
+    if (S.dtype == SSA_DT_BF16) {
+        if (!set_smem(select_kernel<__nv_bfloat16>, sm)) return SSA_ERR_CUDA;
+        select_kernel<__nv_bfloat16><<<grid, 256, sm, st>>>((const __nv_bfloat16 *)Q, Kbar, idx, S.T, S.d, S.s,
+                                                            S.k, S.nb);
+    } else {
+        if (!set_smem(select_kernel<float>, sm)) return SSA_ERR_CUDA;
+        select_kernel<float><<<grid, 256, sm, st>>>((const float *)Q, Kbar, idx, S.T, S.d, S.s, S.k, S.nb);
+    }
+    return launch_status();
+}
+
+ssa_status_t ssa_sparse_attn_fwd(const ssa_dims_t *dims, const void *Q, const void *K, const void *V,
+                                 const int32_t *idx, void *O, float *lse, void *ws, size_t ws_bytes,
+                                 ssa_stream_t stream) {
+    Shape S;
+    ssa_status_t e = check_dims(dims, S, true);
+    if (e != SSA_OK) return e;
+    if (!Q || !K || !V || !idx || !O || !lse) return SSA_ERR_INVALID_ARG;
+    if ((e = check_ws(S, SSA_OP_SPARSE_FWD, ws, ws_bytes)) != SSA_OK) return e;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (!S.tc) {
+        if (S.dtype == SSA_DT_BF16)
+            launch_simt_fwd<__nv_bfloat16>(S, Q, K, V, idx, O, lse, st);
+        else
+            launch_simt_fwd<float>(S, Q, K, V, idx, O, lse, st);
+        return launch_status();
+    }
+    IndexWs W{};
+    uint8_t *p = carve_index(S, static_cast<uint8_t *>(ws), W);
+    __nv_bfloat16 *Opart = reinterpret_cast<__nv_bfloat16 *>(p);
+    p += align_up(S.rows * S.k * 128 * 2);
+    float *lsepart = reinterpret_cast<float *>(p);
+    if ((e = build_index(S, idx, W, st)) != SSA_OK) return e;
+    CUtensorMap tmK, tmV;
+    if (!make_tmap(&tmK, K, S.rows, S.s) || !make_tmap(&tmV, V, S.rows, S.s)) return SSA_ERR_CUDA;
+    const unsigned units = static_cast<unsigned>(S.BH * S.nb);
+    const float sl2 = S.scale * kLog2e;
+    if (S.s == 128) {
+        const size_t sm = SparseFwdSmem<128>::kTotal + 1024;
+        if (!set_smem(sparse_fwd_kernel<128>, sm)) return SSA_ERR_CUDA;
+        sparse_fwd_kernel<128><<<units, 160, sm, st>>>(tmK, tmV, (const __nv_bfloat16 *)Q, W.entries, W.lstart,
+                                                       W.llen, Opart, lsepart, static_cast<int>(S.BH), S.T, S.k,
+                                                       S.nb, sl2);
+    } else {
+        const size_t sm = SparseFwdSmem<64>::kTotal + 1024;
+        if (!set_smem(sparse_fwd_kernel<64>, sm)) return SSA_ERR_CUDA;
+        sparse_fwd_kernel<64><<<units, 160, sm, st>>>(tmK, tmV, (const __nv_bfloat16 *)Q, W.entries, W.lstart,
+                                                      W.llen, Opart, lsepart, static_cast<int>(S.BH), S.T, S.k,
+                                                      S.nb, sl2);
+    }
+    sparse_merge_kernel<__nv_bfloat16><<<static_cast<unsigned>((S.rows + 7) / 8), 256, 0, st>>>(
+        idx, Opart, lsepart, (__nv_bfloat16 *)O, lse, S.rows, S.k);
+    return launch_status();
+}
+
+ssa_status_t ssa_sparse_attn_bwd(const ssa_dims_t *dims, const void *Q, const void *K, const void *V,
+                                 const void *O, const float *lse, const void *dO, const int32_t *idx, void *dQ,
+                                 void *dK, void *dV, int accumulate, void *ws, size_t ws_bytes,
+                                 ssa_stream_t stream) {
+    Shape S;
+    ssa_status_t e = check_dims(dims, S, true);
+    if (e != SSA_OK) return e;
+    if (!Q || !K || !V || !O || !lse || !dO || !idx || !dQ || !dK || !dV) return SSA_ERR_INVALID_ARG;
+    if ((e = check_ws(S, SSA_OP_SPARSE_BWD, ws, ws_bytes)) != SSA_OK) return e;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (S.tc) return tc_bwd(S, Q, K, V, O, lse, dO, idx, dQ, dK, dV, accumulate, ws, st);
+    if (S.dtype == SSA_DT_BF16)
+        return simt_bwd<__nv_bfloat16>(S, Q, K, V, O, lse, dO, idx, dQ, dK, dV, accumulate, ws, st);
+    return simt_bwd<float>(S, Q, K, V, O, lse, dO, idx, dQ, dK, dV, accumulate, ws, st);
+}
+
+ssa_status_t ssa_full_attn_fwd(const ssa_dims_t *dims, const void *Q, const void *K, const void *V, void *O,
+                               float *lse, void *ws, size_t ws_bytes, ssa_stream_t stream) {
+    Shape S;
+    ssa_status_t e = check_dims(dims, S, false);
+    if (e != SSA_OK) return e;
+    if (!Q || !K || !V || !O || !lse) return SSA_ERR_INVALID_ARG;
+    (void)ws;
+    (void)ws_bytes;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (!S.tc) {
+        if (S.dtype == SSA_DT_BF16)
+            launch_simt_fwd<__nv_bfloat16>(S, Q, K, V, nullptr, O, lse, st);
+        else
+            launch_simt_fwd<float>(S, Q, K, V, nullptr, O, lse, st);
+        return launch_status();
+    }
+    CUtensorMap tmQ, tmK, tmV;
+    if (!make_tmap(&tmQ, Q, S.rows, 128) || !make_tmap(&tmK, K, S.rows, 128) || !make_tmap(&tmV, V, S.rows, 128))
+        return SSA_ERR_CUDA;
+    const size_t sm = FullFwdSmem::kTotal + 1024;
+    if (!set_smem(full_fwd_kernel, sm)) return SSA_ERR_CUDA;
+    const dim3 grid((S.T + 127) / 128, S.BH);
+    full_fwd_kernel<<<grid, 192, sm, st>>>(tmQ, tmK, tmV, (__nv_bfloat16 *)O, lse, S.T, S.scale * kLog2e);
+    return launch_status();
+}
+
+ssa_status_t ssa_full_attn_bwd(const ssa_dims_t *dims, const void *Q, const void *K, const void *V,
+                               const void *O, const float *lse, const void *dO, void *dQ, void *dK, void *dV,
+                               int accumulate, void *ws, size_t ws_bytes, ssa_stream_t stream) {
+    Shape S;
+    ssa_status_t e = check_dims(dims, S, false);
+    if (e != SSA_OK) return e;
+    if (!Q || !K || !V || !O || !lse || !dO || !dQ || !dK || !dV) return SSA_ERR_INVALID_ARG;
+    if ((e = check_ws(S, SSA_OP_FULL_BWD, ws, ws_bytes)) != SSA_OK) return e;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (S.tc) return tc_bwd(S, Q, K, V, O, lse, dO, nullptr, dQ, dK, dV, accumulate, ws, st);
+    if (S.dtype == SSA_DT_BF16)
+        return simt_bwd<__nv_bfloat16>(S, Q, K, V, O, lse, dO, nullptr, dQ, dK, dV, accumulate, ws, st);
+    return simt_bwd<float>(S, Q, K, V, O, lse, dO, nullptr, dQ, dK, dV, accumulate, ws, st);
+}
+
+ssa_status_t ssa_align_loss_fwd(const ssa_dims_t *dims, const void *Of, const void *Os, float beta,
+                                float w_sparsity, float w_commit, float *loss_dev, void *ws, size_t ws_bytes,
+                                ssa_stream_t stream) {
+    Shape S;
+    ssa_status_t e = check_dims(dims, S, false);
+    if (e != SSA_OK) return e;
+    if (!Of || !Os || !loss_dev) return SSA_ERR_INVALID_ARG;
+    if (!(beta > 0.f) || !std::isfinite(beta) || !std::isfinite(w_sparsity) || !std::isfinite(w_commit))
+        return SSA_ERR_INVALID_ARG;
+    if ((e = check_ws(S, SSA_OP_ALIGN_FWD, ws, ws_bytes)) != SSA_OK) return e;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    float *partial = static_cast<float *>(ws);
+    const size_t n = S.rows * S.d;
+    if (S.dtype == SSA_DT_BF16)
+        align_fwd_partial_kernel<__nv_bfloat16><<<kAlignBlocks, 256, 0, st>>>(
+            (const __nv_bfloat16 *)Of, (const __nv_bfloat16 *)Os, partial, n, beta);
+    else
+        align_fwd_partial_kernel<float><<<kAlignBlocks, 256, 0, st>>>((const float *)Of, (const float *)Os, partial,
+                                                                      n, beta);
+    align_fwd_final_kernel<<<1, 32, 0, st>>>(partial, kAlignBlocks, loss_dev,
+                                             (static_cast<double>(w_sparsity) + w_commit) / static_cast<double>(n));
+    return launch_status();
+}
+
+ssa_status_t ssa_align_loss_bwd(const ssa_dims_t *dims, const void *Of, const void *Os, float beta,
+                                float w_sparsity, float w_commit, const float *dloss_dev, void *dOf, void *dOs,
+                                int accumulate, ssa_stream_t stream) {
+    Shape S;
+    ssa_status_t e = check_dims(dims, S, false);
+    if (e != SSA_OK) return e;
+    if (!Of || !Os || !dloss_dev || !dOf || !dOs) return SSA_ERR_INVALID_ARG;
+    if (!(beta > 0.f) || !std::isfinite(beta) || !std::isfinite(w_sparsity) || !std::isfinite(w_commit))
+        return SSA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t n = S.rows * S.d;
+    if (S.dtype == SSA_DT_BF16)
+        align_bwd_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, st>>>(
+            (const __nv_bfloat16 *)Of, (const __nv_bfloat16 *)Os, dloss_dev, (__nv_bfloat16 *)dOf,
+            (__nv_bfloat16 *)dOs, n, beta, w_sparsity, w_commit, accumulate);
+    else
+        align_bwd_kernel<float><<<grid_for(n, 256), 256, 0, st>>>((const float *)Of, (const float *)Os, dloss_dev,
+                                                                  (float *)dOf, (float *)dOs, n, beta, w_sparsity,
+                                                                  w_commit, accumulate);
+    return launch_status();
+}
+
+ssa_status_t ssa_dropped_mass(const ssa_dims_t *dims, const float *lse_sparse, const float *lse_full, float *delta,
+                              ssa_stream_t stream) {
+    Shape S;
+    ssa_status_t e = check_dims(dims, S, false);
+    if (e != SSA_OK) return e;
+    if (!lse_sparse || !lse_full || !delta) return SSA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    dropped_mass_kernel<<<grid_for(S.rows, 256), 256, 0, st>>>(lse_sparse, lse_full, delta, S.rows);
+    return launch_status();
+}
+
+ssa_status_t ssa_get_device_error(ssa_stream_t stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return SSA_ERR_CUDA;
+    unsigned int w = 0;
+    if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)) != cudaSuccess) return SSA_ERR_CUDA;
+    if (w == 0) return SSA_OK;
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return SSA_ERR_CUDA;
+    return SSA_ERR_TIMEOUT;
+}
+
+const char *ssa_status_string(ssa_status_t s) {
+    switch (s) {
+        case SSA_OK: return "SSA_OK";
+        case SSA_ERR_INVALID_ARG: return "SSA_ERR_INVALID_ARG";
+        case SSA_ERR_UNSUPPORTED: return "SSA_ERR_UNSUPPORTED";
+        case SSA_ERR_WORKSPACE: return "SSA_ERR_WORKSPACE";
+        case SSA_ERR_CUDA: return "SSA_ERR_CUDA";
+        case SSA_ERR_TIMEOUT: return "SSA_ERR_TIMEOUT";
+    }
+    return "SSA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,210 @@
+/*
+ * ssa.h -- C ABI of libssa: the hot path of SSA block-sparse attention on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method: "SSA: Sparse Sparse Attention by Aligning Full and Sparse Attention
+ * Outputs in Feature Space" (arXiv 2511.20102).  Section 3 of the paper defines
+ * the sparse stream: keys are cut into contiguous blocks of s tokens, each
+ * block is mean-pooled, every preceding block is scored against each query,
+ * the top-k blocks are kept per query and attention runs over their k*s tokens.
+ * Full causal attention (section 3) runs beside it, and section 5 aligns the
+ * two outputs with a bidirectional SmoothL1 loss.
+ *
+ * Conventions shared by every call
+ *  - Tensors are DEVICE pointers allocated and owned by the caller; the library
+ *    never frees or retains them.  Q, K, V, O, dO, dQ, dK, dV, Of, Os, dOf, dOs
+ *    are contiguous [B, H, T, d] in the element type `dims->dtype` (bf16 or
+ *    fp32).  lse / delta are fp32 [B, H, T]; Kbar is fp32 [B, H, T/s, d]; idx is
+ *    int32 [B, H, T, k].
+ *  - Block j covers tokens [j*s, (j+1)*s); b(t) = floor(t/s); nb = T/s.
+ *  - Work is enqueued on `stream` and runs asynchronously.  Argument errors are
+ *    detected on the host before anything is enqueued and return
+ *    SSA_ERR_INVALID_ARG / SSA_ERR_UNSUPPORTED; a failed launch returns
+ *    SSA_ERR_CUDA.  A kernel that gives up on an internal wait (a hang guard,
+ *    about two seconds) records SSA_ERR_TIMEOUT, read by ssa_get_device_error().
+ *  - Supported: bf16 with d == 128 on the tensor-core path; fp32 (any op) and
+ *    bf16 with d == 64 on a CUDA-core path; s in {64, 128}; T % s == 0;
+ *    1 <= k <= nb; nb <= 1024 for ssa_block_select.
+ *  - Workspace: calls that take `ws` need at least ssa_workspace_size(dims, op)
+ *    bytes of device memory (16-byte aligned); its contents on entry are
+ *    ignored and on exit undefined.  The library allocates nothing.
+ */
+#ifndef SSA_H_
+#define SSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ABI-identical to cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *ssa_stream_t;
+
+typedef enum {
+    SSA_OK = 0,
+    SSA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, inconsistent dims */
+    SSA_ERR_UNSUPPORTED = 2, /* valid but outside the supported shapes listed above */
+    SSA_ERR_WORKSPACE = 3,   /* ws too small or misaligned */
+    SSA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+    SSA_ERR_TIMEOUT = 5      /* a kernel gave up on a wait (device error word) */
+} ssa_status_t;
+
+typedef enum { SSA_DT_BF16 = 0, SSA_DT_FP32 = 1 } ssa_dtype_t;
+
+/* Problem shape.  scale is the softmax temperature applied to q.k (1/sqrt(d) is
+ * the usual choice; the paper does not print it). */
+typedef struct {
+    int32_t B, H, T, d, s, k;
+    int32_t dtype; /* ssa_dtype_t */
+    float scale;
+} ssa_dims_t;
+
+/* Operations that need workspace (argument `op` of ssa_workspace_size). */
+enum {
+    SSA_OP_SPARSE_FWD = 0,
+    SSA_OP_SPARSE_BWD = 1,
+    SSA_OP_FULL_FWD = 2,
+    SSA_OP_FULL_BWD = 3,
+    SSA_OP_ALIGN_FWD = 4
+};
+
+/* ssa_block_select flags. */
+enum {
+    /* Always keep the query's own block b(t) (counted within k).  This is the
+     * only mode implemented; flags without this bit return SSA_ERR_UNSUPPORTED. */
+    SSA_SEL_FORCE_CURRENT = 1u
+};
+
+/* Bytes of workspace needed by `op` for these dims (0 when none, or when the
+ * dims are invalid). */
+size_t ssa_workspace_size(const ssa_dims_t *dims, int op);
+
+/*
+ * Block pooling (paper section 3: "scores preceding blocks using mean-pooled
+ * keys").  Kbar[b,h,j,:] = (1/s) * sum_{t in block j} K[b,h,t,:], fp32
+ * accumulation, unweighted.
+ *   K    in   [B,H,T,d] dtype
+ *   Kbar out  [B,H,T/s,d] fp32
+ */
+ssa_status_t ssa_block_pool(const ssa_dims_t *dims, const void *K, float *Kbar, ssa_stream_t stream);
+
+/*
+ * Per-query causal top-k block selection (paper section 3: score preceding
+ * blocks with the pooled keys, keep the top-k; receptive field k*s).
+ * Row t of idx holds the query's own block b(t) plus the k-1 highest-scoring
+ * strictly preceding blocks, score r_j = q_t . Kbar_j evaluated in fp32; equal
+ * scores go to the lower block index.  Entries are ascending; when fewer than
+ * k-1 blocks precede, the row is padded with -1 at the end.  The softmax scale
+ * does not affect the ranking.
+ *   Q    in   [B,H,T,d] dtype
+ *   Kbar in   [B,H,T/s,d] fp32 (from ssa_block_pool)
+ *   idx  out  [B,H,T,k] int32
+ *   flags     SSA_SEL_FORCE_CURRENT
+ */
+ssa_status_t ssa_block_select(const ssa_dims_t *dims, const void *Q, const float *Kbar, int32_t *idx,
+                              unsigned flags, ssa_stream_t stream);
+
+/*
+ * Sparse attention forward (paper section 3: the selected blocks' tokens form
+ * the reduced key and value matrices).  For every query t,
+ *   o_t = softmax_{u in S(t)}(scale * q_t . k_u) v_u,
+ * S(t) = tokens of the blocks in idx[t] with position <= t (causal inside the
+ * query's own block); lse[t] = log sum_{u in S(t)} exp(scale * q_t . k_u).
+ *   idx  in   [B,H,T,k] int32, rows as produced by ssa_block_select (ascending,
+ *             distinct, -1 padding at the end, containing b(t))
+ *   O    out  [B,H,T,d] dtype;  lse out [B,H,T] fp32
+ *   ws        >= ssa_workspace_size(dims, SSA_OP_SPARSE_FWD) bytes
+ */
+ssa_status_t ssa_sparse_attn_fwd(const ssa_dims_t *dims, const void *Q, const void *K, const void *V,
+                                 const int32_t *idx, void *O, float *lse, void *ws, size_t ws_bytes,
+                                 ssa_stream_t stream);
+
+/*
+ * Sparse attention backward (paper section 4.2: keys outside S(t) take no part
+ * in the normalisation and receive no gradient; no gradient flows through the
+ * selection or the pooling).  With P the sparse softmax weights and
+ * D_t = dO_t . o_t:
+ *   dQ_t = scale sum_{u in S(t)} P_tu (dO_t.v_u - D_t) k_u
+ *   dK_u = scale sum_{t: u in S(t)} P_tu (dO_t.v_u - D_t) q_t
+ *   dV_u = sum_{t: u in S(t)} P_tu dO_t
+ *   O, lse     in   outputs of ssa_sparse_attn_fwd for the same Q, K, V, idx
+ *   dO         in   [B,H,T,d] dtype
+ *   dQ, dK, dV out  [B,H,T,d] dtype; accumulate != 0 adds to their current
+ *                   contents (sum formed in fp32, then rounded once)
+ *   ws              >= ssa_workspace_size(dims, SSA_OP_SPARSE_BWD) bytes
+ */
+ssa_status_t ssa_sparse_attn_bwd(const ssa_dims_t *dims, const void *Q, const void *K, const void *V,
+                                 const void *O, const float *lse, const void *dO, const int32_t *idx, void *dQ,
+                                 void *dK, void *dV, int accumulate, void *ws, size_t ws_bytes,
+                                 ssa_stream_t stream);
+
+/*
+ * Full causal attention forward (paper section 3: full attention uses all
+ * preceding tokens): S(t) = {0..t}; outputs as for ssa_sparse_attn_fwd.
+ *   ws  >= ssa_workspace_size(dims, SSA_OP_FULL_FWD) bytes (0 today; may be NULL)
+ */
+ssa_status_t ssa_full_attn_fwd(const ssa_dims_t *dims, const void *Q, const void *K, const void *V, void *O,
+                               float *lse, void *ws, size_t ws_bytes, ssa_stream_t stream);
+
+/*
+ * Full causal attention backward: the formulas of ssa_sparse_attn_bwd with
+ * S(t) = {0..t}.  Same argument meaning and accumulate rule.
+ */
+ssa_status_t ssa_full_attn_bwd(const ssa_dims_t *dims, const void *Q, const void *K, const void *V,
+                               const void *O, const float *lse, const void *dO, void *dQ, void *dK, void *dV,
+                               int accumulate, void *ws, size_t ws_bytes, ssa_stream_t stream);
+
+/*
+ * Bidirectional output alignment, forward (paper section 5: full-attention
+ * outputs are trained toward the sparse ones, a commitment term keeps the
+ * sparse outputs near the full ones, SmoothL1 for both, weighted by alpha).
+ *   loss = w_sparsity * mean huber_beta(Of - sg(Os)) + w_commit * mean huber_beta(Os - sg(Of))
+ *   huber_beta(x) = 0.5 x^2 / beta for |x| < beta, |x| - 0.5 beta otherwise;
+ *   the mean runs over all B*H*T*d elements.
+ *   Of, Os   in   [B,H,T,d] dtype (full / sparse attention outputs)
+ *   beta     > 0
+ *   loss_dev out  one fp32 on the device
+ *   ws            >= ssa_workspace_size(dims, SSA_OP_ALIGN_FWD) bytes
+ */
+ssa_status_t ssa_align_loss_fwd(const ssa_dims_t *dims, const void *Of, const void *Os, float beta,
+                                float w_sparsity, float w_commit, float *loss_dev, void *ws, size_t ws_bytes,
+                                ssa_stream_t stream);
+
+/*
+ * Alignment backward with the stop-gradients of section 5:
+ *   dOf = g * w_sparsity * huber_beta'(Of - Os) / n
+ *   dOs = g * w_commit   * huber_beta'(Os - Of) / n
+ * g = *dloss_dev (device fp32 scalar), n = B*H*T*d.  accumulate is a bit set:
+ * SSA_ACC_OF adds the result into dOf, SSA_ACC_OS into dOs (sum in fp32, one
+ * rounding); a clear bit overwrites.  This lets the main stream's upstream
+ * gradient, preloaded into its buffer, receive the alignment gradient in place.
+ */
+enum { SSA_ACC_OF = 1u, SSA_ACC_OS = 2u };
+ssa_status_t ssa_align_loss_bwd(const ssa_dims_t *dims, const void *Of, const void *Os, float beta,
+                                float w_sparsity, float w_commit, const float *dloss_dev, void *dOf, void *dOs,
+                                int accumulate, ssa_stream_t stream);
+
+/*
+ * Dropped attention mass (paper section 4.2 and Appendix B: the approximation
+ * error is linear in the full-attention mass outside S(t)):
+ *   delta[t] = 1 - exp(lse_sparse[t] - lse_full[t])
+ *   lse_sparse, lse_full in [B,H,T] fp32;  delta out [B,H,T] fp32
+ */
+ssa_status_t ssa_dropped_mass(const ssa_dims_t *dims, const float *lse_sparse, const float *lse_full, float *delta,
+                              ssa_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word:
+ * SSA_OK, or SSA_ERR_TIMEOUT when a kernel gave up on a wait since the last
+ * call; SSA_ERR_CUDA when the synchronisation itself failed. */
+ssa_status_t ssa_get_device_error(ssa_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char *ssa_status_string(ssa_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSA_H_ */

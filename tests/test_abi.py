@@ -1,0 +1,139 @@
+"""Host-side checks of the C ABI: the library builds for sm_100a, loads, exports
+every entry point include/ssa.h declares, and validates arguments on the host
+(no kernel is launched: every call here fails validation before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_top_sparse_b200 import _lib as L
+from block_top_sparse_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "ssa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssa_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    assert names == sorted(L.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = os.popen("nm -D --defined-only %s" % L.LIB_PATH).read()
+    for name in declared_functions():
+        assert re.search(r"\bT %s\b" % name, out), name
+
+
+def test_no_torch_in_boundary():
+    src = open(os.path.join(ROOT, "include", "ssa.h")).read()
+    assert "torch" not in src.lower() and "at::" not in src
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert L.status_string(code).startswith("SSA_")
+    assert L.status_string(99) == "SSA_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(lib):
+    d = L.make_dims(1, 32, 32768, 128, 128, 16)
+    # sparse forward: index (counts, starts, lengths, entries) + bf16 partials + partial lse
+    sf = L.ssa_workspace_size(d, L.SSA_OP_SPARSE_FWD)
+    assert sf >= 32 * 32768 * 16 * (128 * 2 + 4 + 4)
+    fb = L.ssa_workspace_size(d, L.SSA_OP_FULL_BWD)
+    assert fb >= 32 * 32768 * (128 * 4 + 4)
+    assert L.ssa_workspace_size(d, L.SSA_OP_SPARSE_BWD) > fb
+    assert L.ssa_workspace_size(d, L.SSA_OP_FULL_FWD) == 0
+    assert L.ssa_workspace_size(d, L.SSA_OP_ALIGN_FWD) > 0
+    # invalid dims -> 0
+    assert L.ssa_workspace_size(L.make_dims(1, 1, 100, 128, 64, 1), L.SSA_OP_FULL_BWD) == 0
+    # fp32 backward keeps three fp32 accumulators
+    d32 = L.make_dims(1, 2, 1024, 64, 64, 4, dtype="fp32")
+    assert L.ssa_workspace_size(d32, L.SSA_OP_FULL_BWD) >= 3 * 2 * 1024 * 64 * 4
+
+
+def _call(fn, dims, *args):
+    return getattr(L.load(), fn)(ctypes.byref(dims) if dims is not None else None, *args)
+
+
+BAD_DIMS = [
+    (dict(B=0), L.SSA_ERR_INVALID_ARG),
+    (dict(T=-64), L.SSA_ERR_INVALID_ARG),
+    (dict(d=96), L.SSA_ERR_UNSUPPORTED),
+    (dict(s=32), L.SSA_ERR_UNSUPPORTED),
+    (dict(T=1000), L.SSA_ERR_UNSUPPORTED),      # T % s != 0
+    (dict(k=0), L.SSA_ERR_INVALID_ARG),
+    (dict(k=17), L.SSA_ERR_INVALID_ARG),        # k > nb
+    (dict(dtype=7), L.SSA_ERR_INVALID_ARG),
+    (dict(scale=0.0), L.SSA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), L.SSA_ERR_INVALID_ARG),
+]
+
+
+@pytest.mark.parametrize("over,code", BAD_DIMS)
+def test_dims_validation(lib, over, code):
+    base = dict(B=1, H=2, T=1024, d=128, s=64, k=4, dtype=0, scale=0.088)
+    base.update(over)
+    d = L.Dims(base["B"], base["H"], base["T"], base["d"], base["s"], base["k"], base["dtype"], base["scale"])
+    p = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    st = _call("ssa_sparse_attn_fwd", d, p, p, p, p, p, p, p, 1 << 40, None)
+    assert st == code
+
+
+def test_null_pointers_and_workspace(lib):
+    d = L.make_dims(1, 2, 1024, 128, 64, 4)
+    p = ctypes.c_void_p(16)
+    assert _call("ssa_block_pool", None, p, p, None) == L.SSA_ERR_INVALID_ARG
+    assert _call("ssa_block_pool", d, None, p, None) == L.SSA_ERR_INVALID_ARG
+    assert _call("ssa_block_select", d, p, p, None, 1, None) == L.SSA_ERR_INVALID_ARG
+    assert _call("ssa_block_select", d, p, p, p, 0, None) == L.SSA_ERR_UNSUPPORTED
+    assert _call("ssa_block_select", d, p, p, p, 3, None) == L.SSA_ERR_UNSUPPORTED
+    big = L.make_dims(1, 1, 2048 * 64, 128, 64, 4)     # nb = 2048 > 1024
+    assert _call("ssa_block_select", big, p, p, p, 1, None) == L.SSA_ERR_UNSUPPORTED
+    # short / missing / misaligned workspace
+    need = L.ssa_workspace_size(d, L.SSA_OP_SPARSE_FWD)
+    assert _call("ssa_sparse_attn_fwd", d, p, p, p, p, p, p, None, need, None) == L.SSA_ERR_WORKSPACE
+    assert _call("ssa_sparse_attn_fwd", d, p, p, p, p, p, p, p, need - 1, None) == L.SSA_ERR_WORKSPACE
+    assert _call("ssa_sparse_attn_fwd", d, p, p, p, p, p, p, ctypes.c_void_p(24), need, None) == L.SSA_ERR_WORKSPACE
+    need_b = L.ssa_workspace_size(d, L.SSA_OP_FULL_BWD)
+    assert _call("ssa_full_attn_bwd", d, p, p, p, p, p, p, p, p, p, 0, p, need_b - 16, None) == L.SSA_ERR_WORKSPACE
+    assert _call("ssa_align_loss_fwd", d, p, p, ctypes.c_float(0.0), ctypes.c_float(1), ctypes.c_float(1), p, p,
+                 1 << 20, None) == L.SSA_ERR_INVALID_ARG
+    assert _call("ssa_align_loss_bwd", d, p, p, ctypes.c_float(1.0), ctypes.c_float(1), ctypes.c_float(1), None, p,
+                 p, 0, None) == L.SSA_ERR_INVALID_ARG
+    assert _call("ssa_dropped_mass", d, p, None, p, None) == L.SSA_ERR_INVALID_ARG
+
+
+def test_binding_raises_on_error(lib):
+    d = L.make_dims(1, 2, 1024, 128, 64, 4)
+    with pytest.raises(L.SSAError) as e:
+        L.ssa_block_pool(d, None, None, stream=0)
+    assert e.value.status == L.SSA_ERR_INVALID_ARG
+
+
+def test_build_flags_target_sm100a():
+    flags = B.nvcc_flags()
+    assert "arch=compute_100a,code=sm_100a" in flags and "-lineinfo" in flags
+
+
+def test_product_does_not_import_oracle():
+    pkg = os.path.join(ROOT, "block_top_sparse_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt and "ssa_oracle" not in txt, f
