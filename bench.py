@@ -323,6 +323,55 @@ def ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def single_op(args):
+    """One library call at a chosen size, timed with CUDA events (for profiling runs)."""
+    import torch
+    from block_top_sparse_b200 import _lib as L
+    from block_top_sparse_b200 import build, inputs, ops
+
+    build.build()
+    wl = inputs.WORKLOADS[args.workload]
+    g = inputs.generate(wl, H=args.H or wl.H, T=args.T or wl.T, with_dO=True)
+    w = g["wl"]
+    k = args.k or w.k[0]
+    dims = L.make_dims(w.B, w.H, w.T, w.d, w.s, k, dtype=w.dtype)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dev = {key: torch.from_numpy(g[key].view(np.int16) if w.dtype == "bf16" else g[key]).view(dt).cuda()
+           for key in ("Q", "K", "V", "dO")}
+    st = ops.SSAStep(dims)
+    st.forward(dev["Q"], dev["K"], dev["V"])
+    st.dOf.copy_(dev["dO"])
+    st.dOs.copy_(dev["dO"])
+    Q, K, V = dev["Q"], dev["K"], dev["V"]
+    calls = {
+        "pool": lambda: L.ssa_block_pool(dims, K, st.Kbar),
+        "select": lambda: L.ssa_block_select(dims, Q, st.Kbar, st.idx),
+        "full_fwd": lambda: L.ssa_full_attn_fwd(dims, Q, K, V, st.Of, st.lse_f, st.ws[L.SSA_OP_FULL_FWD]),
+        "sparse_fwd": lambda: L.ssa_sparse_attn_fwd(dims, Q, K, V, st.idx, st.Os, st.lse_s,
+                                                    st.ws[L.SSA_OP_SPARSE_FWD]),
+        "full_bwd": lambda: L.ssa_full_attn_bwd(dims, Q, K, V, st.Of, st.lse_f, st.dOf, st.dQ, st.dK, st.dV, 0,
+                                                st.ws[L.SSA_OP_FULL_BWD]),
+        "sparse_bwd": lambda: L.ssa_sparse_attn_bwd(dims, Q, K, V, st.Os, st.lse_s, st.dOs, st.idx, st.dQ, st.dK,
+                                                    st.dV, 0, st.ws[L.SSA_OP_SPARSE_BWD]),
+    }
+    fn = calls[args.op]
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    sf, sb, ff, fb = flops(w.B, w.H, w.T, w.d, w.s, k)
+    fl = {"full_fwd": ff, "full_bwd": fb, "sparse_fwd": sf, "sparse_bwd": sb}.get(args.op)
+    print(json.dumps({"op": args.op, "workload": w.name, "B": w.B, "H": w.H, "T": w.T, "k": k, "ms": ms,
+                      "tflops": fl / (ms / 1e3) / 1e12 if fl else None,
+                      "device_error": L.ssa_get_device_error()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -331,7 +380,17 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=4096, help="prefix length of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default=None,
+                    choices=["pool", "select", "full_fwd", "sparse_fwd", "full_bwd", "sparse_bwd"],
+                    help="time one library call instead of the whole step (profiling)")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--T", type=int, default=0)
+    ap.add_argument("--H", type=int, default=0)
+    ap.add_argument("--k", type=int, default=0)
     args = ap.parse_args()
+    if args.op:
+        single_op(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
