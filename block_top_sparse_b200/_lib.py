@@ -20,12 +20,13 @@ SSA_DT_BF16, SSA_DT_FP32 = 0, 1
 SSA_OP_SPARSE_FWD, SSA_OP_SPARSE_BWD, SSA_OP_FULL_FWD, SSA_OP_FULL_BWD, SSA_OP_ALIGN_FWD = range(5)
 SSA_SEL_FORCE_CURRENT = 1
 SSA_ACC_OF, SSA_ACC_OS = 1, 2
+SSA_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 # Every entry point include/ssa.h declares.
 EXPORTS = (
     "ssa_workspace_size", "ssa_block_pool", "ssa_block_select", "ssa_sparse_attn_fwd", "ssa_sparse_attn_bwd",
     "ssa_full_attn_fwd", "ssa_full_attn_bwd", "ssa_align_loss_fwd", "ssa_align_loss_bwd", "ssa_dropped_mass",
-    "ssa_get_device_error", "ssa_status_string",
+    "ssa_get_device_error", "ssa_status_string", "ssa_full_attn_bwd_noalloc",
 )
 
 
@@ -70,6 +71,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "ssa_sparse_attn_bwd": (I, [C, P, P, P, P, P, P, P, P, P, P, I, P, S, P]),
         "ssa_full_attn_fwd": (I, [C, P, P, P, P, P, P, S, P]),
         "ssa_full_attn_bwd": (I, [C, P, P, P, P, P, P, P, P, P, I, P, S, P]),
+        "ssa_full_attn_bwd_noalloc": (I, [C, P, P, P, P, P, P, P, P, P, I, P]),
         "ssa_align_loss_fwd": (I, [C, P, P, F, F, F, P, P, S, P]),
         "ssa_align_loss_bwd": (I, [C, P, P, F, F, F, P, P, P, I, P]),
         "ssa_dropped_mass": (I, [C, P, P, P, P]),
@@ -150,6 +152,13 @@ def ssa_full_attn_bwd(dims, Q, K, V, O, lse, dO, dQ, dK, dV, accumulate=0, ws=No
     _check("ssa_full_attn_bwd",
            load().ssa_full_attn_bwd(ctypes.byref(dims), _p(Q), _p(K), _p(V), _p(O), _p(lse), _p(dO), _p(dQ),
                                     _p(dK), _p(dV), int(accumulate), _p(ws), _nbytes(ws), _stream(stream)))
+
+
+def ssa_full_attn_bwd_noalloc(dims, Q, K, V, O, lse, dO, dQ, dK, dV, accumulate=0, stream=None):
+    """Full attention backward with library-held scratch (no workspace, no allocation)."""
+    _check("ssa_full_attn_bwd_noalloc",
+           load().ssa_full_attn_bwd_noalloc(ctypes.byref(dims), _p(Q), _p(K), _p(V), _p(O), _p(lse), _p(dO),
+                                            _p(dQ), _p(dK), _p(dV), int(accumulate), _stream(stream)))
 
 
 def ssa_align_loss_fwd(dims, Of, Os, beta, w_sparsity, w_commit, loss, ws=None, stream=None):

@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "ssa.h"
 
@@ -477,6 +478,51 @@ ssa_status_t ssa_dropped_mass(const ssa_dims_t *dims, const float *lse_sparse, c
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     dropped_mass_kernel<<<grid_for(S.rows, 256), 256, 0, st>>>(lse_sparse, lse_full, delta, S.rows);
     return launch_status();
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free full attention backward: scratch in a static device array.
+// In host code the array's name is only a stand-in; its device address comes
+// from cudaGetSymbolAddress, looked up once per device with that device current.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SSA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+void *g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mutex;
+
+ssa_status_t noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SSA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SSA_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+ssa_status_t ssa_full_attn_bwd_noalloc(const ssa_dims_t *dims, const void *Q, const void *K, const void *V,
+                                       const void *O, const float *lse, const void *dO, void *dQ, void *dK,
+                                       void *dV, int accumulate, ssa_stream_t stream) {
+    Shape S;
+    ssa_status_t e = check_dims(dims, S, false);
+    if (e != SSA_OK) return e;
+    if (!Q || !K || !V || !O || !lse || !dO || !dQ || !dK || !dV) return SSA_ERR_INVALID_ARG;
+    const size_t need = ws_bytes_for(S, SSA_OP_FULL_BWD);
+    if (need > SSA_NOALLOC_SCRATCH_BYTES) return SSA_ERR_WORKSPACE;
+    void *ws = nullptr;
+    if ((e = noalloc_scratch(&ws)) != SSA_OK) return e;
+    return ssa_full_attn_bwd(dims, Q, K, V, O, lse, dO, dQ, dK, dV, accumulate, ws, SSA_NOALLOC_SCRATCH_BYTES,
+                             stream);
 }
 
 ssa_status_t ssa_get_device_error(ssa_stream_t stream) {

@@ -195,6 +195,33 @@ ssa_status_t ssa_align_loss_bwd(const ssa_dims_t *dims, const void *Of, const vo
 ssa_status_t ssa_dropped_mass(const ssa_dims_t *dims, const float *lse_sparse, const float *lse_full, float *delta,
                               ssa_stream_t stream);
 
+/*
+ * Full causal attention backward that allocates nothing and takes no workspace.
+ * The paper has no counterpart: this entry point exists for callers that cannot
+ * allocate device memory at the point of the call -- for example code running
+ * inside a host that owns every allocation through its own pool and forbids
+ * others, or a real-time path that must not call cudaMalloc (which may
+ * synchronise the device).  Same arguments and results as ssa_full_attn_bwd
+ * without ws / ws_bytes.
+ *  - Scratch: a file-scope device array of SSA_NOALLOC_SCRATCH_BYTES (32 MiB)
+ *    inside libssa, present on every GPU that loads the library until the
+ *    process exits.  The call needs ssa_workspace_size(dims, SSA_OP_FULL_BWD)
+ *    bytes of it (bf16, d = 128: 516 bytes per query row, so at most 65,027
+ *    rows B*H*T); larger problems return SSA_ERR_WORKSPACE before anything is
+ *    enqueued.
+ *  - The first call on a device looks up the array's device address with that
+ *    device current; make this first call before any stream capture begins.
+ *  - Every call shares the one array and leaves its contents behind; the parts
+ *    that must start at zero are cleared by the call itself on `stream`.  Calls
+ *    that overlap on the GPU (other streams, other host threads) race on the
+ *    scratch: serialise them.
+ *  - No cudaMalloc, cudaFree or allocating library routine is called.
+ */
+#define SSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+ssa_status_t ssa_full_attn_bwd_noalloc(const ssa_dims_t *dims, const void *Q, const void *K, const void *V,
+                                       const void *O, const float *lse, const void *dO, void *dQ, void *dK,
+                                       void *dV, int accumulate, ssa_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word:
  * SSA_OK, or SSA_ERR_TIMEOUT when a kernel gave up on a wait since the last
  * call; SSA_ERR_CUDA when the synchronisation itself failed. */
