@@ -9,11 +9,7 @@
 //                     holds j (gathered by row), and writes a normalised
 //                     partial output + log-sum-exp per (query, slot); a merge
 //                     kernel combines the k partials of each query.
-//  attn_bwd_kernel    backward for both streams, key-block-outer: one CTA per
-//                     key tile (full) or key block (sparse) keeps K_j, V_j and
-//                     the transposed dK_j, dV_j accumulators resident and loops
-//                     over the query rows that attend to it; dQ is accumulated
-//                     with fp32 vector atomics.
+//  (the backward kernel shared by both streams is in attn_bwd.cuh)
 //
 // Shared-memory operand tiles are "chunks" of R rows x 64 bf16 (128 B rows,
 // 128-byte swizzle), see smem_desc_sw128().  Warps 0..3 (128 threads) own one
@@ -490,250 +486,6 @@ __global__ void __launch_bounds__(160, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, 256);
-}
-
-// ---------------------------------------------------------------------------
-// Backward for full (NKV = 128, contiguous query tiles) and sparse (gathered
-// query rows of key block j) attention.
-// grid: full   -> (nkt * BH) units, u -> key tile n = u / BH, head bh = u % BH
-//       sparse -> (nb * BH) units,  u -> block j = u / BH,   head bh = u % BH
-// block = 160.  Per query tile:
-//   S = Q K^T, dP = dO V^T                       (thread r <-> query row r)
-//   P = exp(scale S - lse), dS = P (dP - D)      -> shared memory, bf16
-//   dV^T += dO^T P, dK^T += Q^T dS               (tensor memory, M = head dim)
-//   dQ = dS K  -> fp32 atomics into dQacc (scaled)
-// smem: Q 32 KB | dO 32 KB | K, V NKV*256 each | P, dS (NKV/64)*16 KB each
-// tmem: S / dQ at 0, dP at 128, dV^T at 256, dK^T at 384 (512 allocated).
-// ---------------------------------------------------------------------------
-template <int NKV>
-struct BwdSmem {
-    static constexpr int kQ = 0;
-    static constexpr int kdO = kQ + 2 * kChunkBytes;
-    static constexpr int kK = kdO + 2 * kChunkBytes;
-    static constexpr int kV = kK + 2 * NKV * 128;
-    static constexpr int kP = kV + 2 * NKV * 128;
-    static constexpr int kdS = kP + (NKV / 64) * kChunkBytes;
-    static constexpr int kBar = kdS + (NKV / 64) * kChunkBytes;
-    static constexpr int kTotal = kBar + 256;
-};
-
-struct BwdArgs {
-    const __nv_bfloat16 *Q, *dO;
-    const float *lse, *Dvec;
-    float *dQacc;
-    __nv_bfloat16 *dK, *dV;
-    const float *dK_in_f32;  // unused (reserved)
-    const int32_t *entries, *lstart, *llen;  // sparse only
-    int BH, T, k, nb, sparse, accumulate;
-    float scale, scale_log2;
-};
-
-template <int NKV>
-__global__ void __launch_bounds__(160, 1)
-    attn_bwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                    const BwdArgs a) {
-    using L = BwdSmem<NKV>;
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
-    uint64_t *bar_kv = bars + 0, *bar_qdo_full = bars + 1, *bar_sdp_full = bars + 2, *bar_pds_full = bars + 3;
-    uint64_t *bar_dq_full = bars + 4, *bar_dq_empty = bars + 5, *bar_final = bars + 6;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 9);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int T = a.T;
-    const int kb = blockIdx.x / a.BH, bh = blockIdx.x % a.BH;
-    const int kv0 = kb * NKV;
-    const size_t head_rows = static_cast<size_t>(bh) * T;
-    Rows R;
-    int ntiles;
-    if (a.sparse) {
-        R.list = a.entries + head_rows * a.k + a.lstart[bh * a.nb + kb];
-        R.len = a.llen[bh * a.nb + kb];
-        R.first = 0;
-        ntiles = (R.len + kTileQ - 1) / kTileQ;
-    } else {
-        R.list = nullptr;
-        R.first = kv0;  // causal: query tiles from the key tile onward
-        R.len = T - kv0;
-        ntiles = (R.len + kTileQ - 1) / kTileQ;
-    }
-    R.k = a.k;
-
-    const uint32_t sQ = smem_u32(smem + L::kQ), sdO = smem_u32(smem + L::kdO), sK = smem_u32(smem + L::kK),
-                   sV = smem_u32(smem + L::kV), sP = smem_u32(smem + L::kP), sdS = smem_u32(smem + L::kdS);
-
-    if (threadIdx.x == 0) {
-        mbar_init(bar_kv, 1);
-        mbar_init(bar_qdo_full, 128);
-        mbar_init(bar_sdp_full, 1);
-        mbar_init(bar_pds_full, 128);
-        mbar_init(bar_dq_full, 1);
-        mbar_init(bar_dq_empty, 128);
-        mbar_init(bar_final, 1);
-        *abort_flag = 0;
-        fence_barrier_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(tmem_slot, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384, tdQ = tmem;
-
-    if (warp == 4) {
-        if (lane == 0) {
-            const int krow = static_cast<int>(head_rows) + kv0;
-            mbar_arrive_expect_tx(bar_kv, 4 * NKV * 128);
-            tma_load_2d(&tmK, bar_kv, smem + L::kK, 0, krow);
-            tma_load_2d(&tmK, bar_kv, smem + L::kK + NKV * 128, 64, krow);
-            tma_load_2d(&tmV, bar_kv, smem + L::kV, 0, krow);
-            tma_load_2d(&tmV, bar_kv, smem + L::kV + NKV * 128, 64, krow);
-            const uint32_t idS = idesc_bf16(128, NKV, false, false);   // S, dP
-            const uint32_t idT = idesc_bf16(128, NKV, true, true);     // dV^T, dK^T
-            const uint32_t idQ = idesc_bf16(128, 128, false, true);    // dQ
-            bool ok = mbar_wait(bar_kv, 0, abort_flag, 0x301);
-            for (int it = 0; ok && it < ntiles; ++it) {
-                if (!mbar_wait(bar_qdo_full, it & 1, abort_flag, 0x302)) break;
-                if (it > 0 && !mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x303)) break;
-                tc_fence_after();
-                mma_k128_kmajor(tS, sQ, sK, NKV * 128, idS);
-                mma_k128_kmajor(tdP, sdO, sV, NKV * 128, idS);
-                mma_commit(bar_sdp_full);
-                if (!mbar_wait(bar_pds_full, it & 1, abort_flag, 0x304)) break;
-                tc_fence_after();
-                // dV^T[d x kv] += dO^T P ; dK^T[d x kv] += Q^T dS   (K = 128 query rows)
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t a_do = smem_desc_sw128(sdO + kk * 2048, kChunkBytes);
-                    const uint64_t b_p = smem_desc_sw128(sP + kk * 2048, kChunkBytes);
-                    mma_bf16_ss(tdV, a_do, b_p, idT, (it > 0 || kk > 0) ? 1u : 0u);
-                }
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t a_q = smem_desc_sw128(sQ + kk * 2048, kChunkBytes);
-                    const uint64_t b_ds = smem_desc_sw128(sdS + kk * 2048, kChunkBytes);
-                    mma_bf16_ss(tdK, a_q, b_ds, idT, (it > 0 || kk > 0) ? 1u : 0u);
-                }
-                // dQ[q x d] = dS K   (K = NKV keys)
-#pragma unroll
-                for (int kk = 0; kk < NKV / 16; ++kk) {
-                    const uint64_t a_ds = smem_desc_sw128(sdS + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16);
-                    const uint64_t b_k = smem_desc_sw128(sK + kk * 2048, NKV * 128);
-                    mma_bf16_ss(tdQ, a_ds, b_k, idQ, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(bar_dq_full);
-            }
-            mma_commit(bar_final);
-            mbar_wait(bar_final, 0, abort_flag, 0x305);
-        }
-    } else {
-        const int r = threadIdx.x;
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        int t = 0, e = 0;
-        bool valid = ntiles > 0 && tile_row(R, T, 0, r, t, e);
-        gather_row(sQ, a.Q + (head_rows + (valid ? t : 0)) * kD, valid, r);
-        gather_row(sdO, a.dO + (head_rows + (valid ? t : 0)) * kD, valid, r);
-        cp_async_commit();
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        mbar_arrive(bar_qdo_full);
-        bool ok = true;
-        for (int it = 0; it < ntiles; ++it) {
-            const float lse2 = valid ? __ldg(a.lse + head_rows + t) * kLog2e : 0.f;
-            const float Dt = valid ? __ldg(a.Dvec + head_rows + t) : 0.f;
-            if (!mbar_wait(bar_sdp_full, it & 1, abort_flag, 0x306)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            for (int c0 = 0; c0 < NKV; c0 += 32) {
-                float sv[32], dp[32];
-                tmem_ld32(tS + lane_off + c0, sv);
-                tmem_ld32(tdP + lane_off + c0, dp);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int kv = kv0 + c0 + i;
-                    const bool keep = valid && kv <= t;
-                    const float p = keep ? fast_exp2(sv[i] * a.scale_log2 - lse2) : 0.f;
-                    sv[i] = p;
-                    dp[i] = p * (dp[i] - Dt);
-                }
-                store_row32_bf16(sP, kChunkBytes, r, c0, sv);
-                store_row32_bf16(sdS, kChunkBytes, r, c0, dp);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(bar_pds_full);
-            if (!mbar_wait(bar_dq_full, it & 1, abort_flag, 0x307)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            int t_next = 0, e_next = 0;
-            bool valid_next = false;
-            if (it + 1 < ntiles) {
-                valid_next = tile_row(R, T, it + 1, r, t_next, e_next);
-                const size_t src = head_rows + (valid_next ? t_next : 0);
-                gather_row(sQ, a.Q + src * kD, valid_next, r);
-                gather_row(sdO, a.dO + src * kD, valid_next, r);
-                cp_async_commit();
-            }
-            float *dq = a.dQacc + (head_rows + (valid ? t : 0)) * kD;
-            for (int c0 = 0; c0 < 128; c0 += 32) {
-                float g[32];
-                tmem_ld32(tdQ + lane_off + c0, g);
-                if (valid) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        atomicAdd(reinterpret_cast<float4 *>(dq + c0) + q,
-                                  make_float4(g[4 * q] * a.scale, g[4 * q + 1] * a.scale, g[4 * q + 2] * a.scale,
-                                              g[4 * q + 3] * a.scale));
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(bar_dq_empty);
-            if (it + 1 < ntiles) {
-                cp_async_wait_all();
-                fence_proxy_async_smem();
-                mbar_arrive(bar_qdo_full);
-                t = t_next;
-                e = e_next;
-                valid = valid_next;
-            }
-        }
-        cp_async_wait_all();
-        // Epilogue: thread r <-> head-dim row r of dV^T / dK^T; column c <-> key kv0 + c.
-        if (ok) {
-            for (int c0 = 0; c0 < NKV; c0 += 32) {
-                float gv[32], gk[32];
-                tmem_ld32(tdV + lane_off + c0, gv);
-                tmem_ld32(tdK + lane_off + c0, gk);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int kv = kv0 + c0 + i;
-                    if (kv < T) {
-                        const size_t off = (head_rows + kv) * kD + r;
-                        float vv = ntiles > 0 ? gv[i] : 0.f, kk = ntiles > 0 ? gk[i] * a.scale : 0.f;
-                        if (a.accumulate) {
-                            vv += __bfloat162float(a.dV[off]);
-                            kk += __bfloat162float(a.dK[off]);
-                        }
-                        a.dV[off] = __float2bfloat16_rn(vv);
-                        a.dK[off] = __float2bfloat16_rn(kk);
-                    }
-                }
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace ssa

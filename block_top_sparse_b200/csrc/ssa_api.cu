@@ -17,6 +17,7 @@
 #include "aux_kernels.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
+#include "attn_bwd.cuh"
 
 using namespace ssa;
 
@@ -238,8 +239,10 @@ ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V,
     bwd_prep_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16 *)dO, (const __nv_bfloat16 *)O, Dvec,
                                                        dQacc, S.rows, S.d);
     const int nkv = sparse ? S.s : 128;
-    CUtensorMap tmK, tmV;
-    if (!make_tmap(&tmK, K, S.rows, nkv) || !make_tmap(&tmV, V, S.rows, nkv)) return SSA_ERR_CUDA;
+    CUtensorMap tmK, tmV, tmQ, tmdO;
+    if (!make_tmap(&tmK, K, S.rows, nkv) || !make_tmap(&tmV, V, S.rows, nkv) || !make_tmap(&tmQ, Q, S.rows, 128) ||
+        !make_tmap(&tmdO, dO, S.rows, 128))
+        return SSA_ERR_CUDA;
     BwdArgs a{};
     a.Q = (const __nv_bfloat16 *)Q;
     a.dO = (const __nv_bfloat16 *)dO;
@@ -263,11 +266,11 @@ ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V,
     if (nkv == 128) {
         const size_t sm = BwdSmem<128>::kTotal + 1024;
         if (!set_smem(attn_bwd_kernel<128>, sm)) return SSA_ERR_CUDA;
-        attn_bwd_kernel<128><<<units, 160, sm, st>>>(tmK, tmV, a);
+        attn_bwd_kernel<128><<<units, kBwdThreads, sm, st>>>(tmK, tmV, tmQ, tmdO, a);
     } else {
         const size_t sm = BwdSmem<64>::kTotal + 1024;
         if (!set_smem(attn_bwd_kernel<64>, sm)) return SSA_ERR_CUDA;
-        attn_bwd_kernel<64><<<units, 160, sm, st>>>(tmK, tmV, a);
+        attn_bwd_kernel<64><<<units, kBwdThreads, sm, st>>>(tmK, tmV, tmQ, tmdO, a);
     }
     const size_t n = S.rows * S.d;
     acc_to_out_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, st>>>(dQacc, (__nv_bfloat16 *)dQ, n, accumulate);
