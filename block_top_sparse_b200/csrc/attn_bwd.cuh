@@ -71,7 +71,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T;
-    const int kb = blockIdx.x / a.BH, bh = blockIdx.x % a.BH;
+    // Head-major unit order, heaviest key block of each head first: the query
+    // rows and the dQ accumulator of the head being worked on stay in L2.
+    const int units_per_head = a.sparse ? a.nb : (a.T + NKV - 1) / NKV;
+    const int bh = blockIdx.x / units_per_head, kb = blockIdx.x % units_per_head;
     const int kv0 = kb * NKV;
     const size_t head_rows = static_cast<size_t>(bh) * T;
     const bool sparse = a.sparse != 0;
@@ -198,20 +201,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 break;
             }
             tc_fence_after();
+            // all tensor-memory loads of this row half in flight at once, one wait
+            uint32_t sraw[HALF / 32][32], draw[HALF / 32][32];
 #pragma unroll
-            for (int c0 = h * HALF; c0 < (h + 1) * HALF; c0 += 32) {
+            for (int c = 0; c < HALF / 32; ++c) {
+                tmem_ld32_async(tS + lane_off + h * HALF + 32 * c, sraw[c]);
+                tmem_ld32_async(tdP + lane_off + h * HALF + 32 * c, draw[c]);
+            }
+            tmem_ld_wait();
+            // key kv0 + col is attended when col <= lim (causal inside the diagonal block)
+            const int lim = valid ? t - kv0 - h * HALF : -1;
+#pragma unroll
+            for (int c = 0; c < HALF / 32; ++c) {
                 float sv[32], dp[32];
-                tmem_ld32(tS + lane_off + c0, sv);
-                tmem_ld32(tdP + lane_off + c0, dp);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const bool keep = valid && (kv0 + c0 + i <= t);
-                    const float p = keep ? fast_exp2(sv[i] * a.scale_log2 - lse2) : 0.f;
+                    const float p = (32 * c + i <= lim)
+                                        ? fast_exp2(fmaf(__uint_as_float(sraw[c][i]), a.scale_log2, -lse2))
+                                        : 0.f;
                     sv[i] = p;
-                    dp[i] = p * (dp[i] - Dt);
+                    dp[i] = p * (__uint_as_float(draw[c][i]) - Dt);
                 }
-                store_row32_bf16(sP, kChunkBytes, r, c0, sv);
-                store_row32_bf16(sdS, kChunkBytes, r, c0, dp);
+                store_row32_bf16(sP, kChunkBytes, r, h * HALF + 32 * c, sv);
+                store_row32_bf16(sdS, kChunkBytes, r, h * HALF + 32 * c, dp);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -235,21 +247,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 break;
             }
             tc_fence_after();
-            float g0[32], g1[32];
-            tmem_ld32(tdQ + lane_off + h * 64, g0);
-            tmem_ld32(tdQ + lane_off + h * 64 + 32, g1);
+            uint32_t g[2][32];
+            tmem_ld32_async(tdQ + lane_off + h * 64, g[0]);
+            tmem_ld32_async(tdQ + lane_off + h * 64 + 32, g[1]);
+            tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(bar_dq_empty);
             if (valid) {
                 float4 *dq = reinterpret_cast<float4 *>(a.dQacc + (head_rows + t) * kD + h * 64);
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    atomicAdd(dq + q, make_float4(g0[4 * q] * a.scale, g0[4 * q + 1] * a.scale,
-                                                  g0[4 * q + 2] * a.scale, g0[4 * q + 3] * a.scale));
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    atomicAdd(dq + 8 + q, make_float4(g1[4 * q] * a.scale, g1[4 * q + 1] * a.scale,
-                                                      g1[4 * q + 2] * a.scale, g1[4 * q + 3] * a.scale));
+                for (int q = 0; q < 16; ++q) {
+                    const uint32_t *x = g[q >> 3] + 4 * (q & 7);
+                    atomicAdd(dq + q, make_float4(__uint_as_float(x[0]) * a.scale, __uint_as_float(x[1]) * a.scale,
+                                                  __uint_as_float(x[2]) * a.scale, __uint_as_float(x[3]) * a.scale));
+                }
             }
             if (sparse && more) {
                 cp_async_wait_all();
@@ -265,9 +276,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (ok) {
 #pragma unroll
             for (int c0 = h * HALF; c0 < (h + 1) * HALF; c0 += 32) {
+                uint32_t rv[32], rk[32];
+                tmem_ld32_async(tdV + lane_off + c0, rv);
+                tmem_ld32_async(tdK + lane_off + c0, rk);
+                tmem_ld_wait();
                 float gv[32], gk[32];
-                tmem_ld32(tdV + lane_off + c0, gv);
-                tmem_ld32(tdK + lane_off + c0, gk);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    gv[i] = __uint_as_float(rv[i]);
+                    gk[i] = __uint_as_float(rk[i]);
+                }
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int kv = kv0 + c0 + i;

@@ -223,19 +223,19 @@ __global__ void __launch_bounds__(192, 1)
             }
             tc_fence_after();
             const uint32_t tS = tmem + sb * 128 + lane_off;
-            const bool diag = (n == m);
-            // pass 1: row maximum (log2 domain)
-            float mx = -INFINITY;
-            for (int c0 = 0; c0 < 128; c0 += 32) {
-                float v[32];
-                tmem_ld32(tS + c0, v);
+            // the whole S row in registers: four loads in flight, one wait
+            uint32_t sr[4][32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int kv = n * kTileQ + c0 + i;
-                    const float x = (diag && kv > t) ? -INFINITY : v[i] * scale_log2;
-                    mx = fmaxf(mx, x);
-                }
-            }
+            for (int c = 0; c < 4; ++c) tmem_ld32_async(tS + 32 * c, sr[c]);
+            tmem_ld_wait();
+            // key n*128 + col is attended when col <= lim (causal on the diagonal tile)
+            const int lim = (n == m) ? t - n * kTileQ : 127;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    mx = fmaxf(mx, (32 * c + i <= lim) ? __uint_as_float(sr[c][i]) * scale_log2 : -INFINITY);
             float alpha = 1.f;
             if (n == 0) {
                 m_used = mx;
@@ -261,18 +261,18 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             l *= alpha;
-            // pass 2: probabilities -> P (bf16) in shared memory
-            for (int c0 = 0; c0 < 128; c0 += 32) {
+            // probabilities -> P (bf16) in shared memory
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
                 float v[32];
-                tmem_ld32(tS + c0, v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int kv = n * kTileQ + c0 + i;
-                    const float p = (diag && kv > t) ? 0.f : fast_exp2(v[i] * scale_log2 - m_used);
+                    const float p =
+                        (32 * c + i <= lim) ? fast_exp2(fmaf(__uint_as_float(sr[c][i]), scale_log2, -m_used)) : 0.f;
                     l += p;
                     v[i] = p;
                 }
-                store_row32_bf16(sP, kChunkBytes, r, c0, v);
+                store_row32_bf16(sP, kChunkBytes, r, 32 * c, v);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -416,29 +416,31 @@ __global__ void __launch_bounds__(160, 1)
         for (int it = 0; it < ntiles; ++it) {
             if (!mbar_wait(bar_s_full, it & 1, abort_flag, 0x206)) break;
             tc_fence_after();
-            float mx = -INFINITY;
-            for (int c0 = 0; c0 < NKV; c0 += 32) {
-                float v[32];
-                tmem_ld32(tS + lane_off + c0, v);
+            uint32_t sr[NKV / 32][32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const bool keep = valid && (kv0 + c0 + i <= t);
-                    mx = fmaxf(mx, keep ? v[i] * scale_log2 : -INFINITY);
-                }
-            }
+            for (int c = 0; c < NKV / 32; ++c) tmem_ld32_async(tS + lane_off + 32 * c, sr[c]);
+            tmem_ld_wait();
+            // key kv0 + col is attended when col <= lim (causal inside the query's own block)
+            const int lim = valid ? t - kv0 : -1;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < NKV / 32; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    mx = fmaxf(mx, (32 * c + i <= lim) ? __uint_as_float(sr[c][i]) * scale_log2 : -INFINITY);
             const float mref = (mx == -INFINITY) ? 0.f : mx;
             float l = 0.f;
-            for (int c0 = 0; c0 < NKV; c0 += 32) {
+#pragma unroll
+            for (int c = 0; c < NKV / 32; ++c) {
                 float v[32];
-                tmem_ld32(tS + lane_off + c0, v);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const bool keep = valid && (kv0 + c0 + i <= t);
-                    const float p = keep ? fast_exp2(v[i] * scale_log2 - mref) : 0.f;
+                    const float p =
+                        (32 * c + i <= lim) ? fast_exp2(fmaf(__uint_as_float(sr[c][i]), scale_log2, -mref)) : 0.f;
                     l += p;
                     v[i] = p;
                 }
-                store_row32_bf16(sP, kChunkBytes, r, c0, v);
+                store_row32_bf16(sP, kChunkBytes, r, 32 * c, v);
             }
             fence_proxy_async_smem();
             tc_fence_before();
