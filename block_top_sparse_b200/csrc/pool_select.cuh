@@ -89,18 +89,22 @@ __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ K, floa
 
 // ---------------------------------------------------------------------------
 // Selection.  One CTA (256 threads) per 32 consecutive queries of one head
-// (all in the same block, since s is a multiple of 32).
-//   phase 1: scores S[q][j] = q . Kbar_j for j < b(t), fp32 FMA in column order,
-//            4 queries x 4 blocks per thread, Kbar staged 128 blocks at a time;
-//   phase 2: one warp per query: radix select of the (k-1)-th largest score
-//            on order-preserving 32-bit keys, then an ascending ballot
-//            compaction that keeps equal scores in index order.
+// (all in the same block, since s is a multiple of 32); warp w owns queries
+// 4w .. 4w+3 from scoring to output.
+//   scores: r[q][j] = q . Kbar_j for j < b(t), fp32 FMA in column order; Kbar
+//           staged 64 blocks at a time; lane l of warp w scores blocks l and
+//           l + 32 of the chunk for the warp's 4 queries;
+//   top-(k-1): the (k-1)-th largest order-preserving 32-bit key is built bit by
+//           bit from the most significant end (count of keys >= candidate by
+//           warp reduction); keys above it are kept, keys equal to it are kept
+//           in ascending block order until k-1 are chosen; a ballot compaction
+//           writes the chosen blocks in ascending order, then b(t), then -1.
 // ---------------------------------------------------------------------------
 constexpr int kSelQ = 32;
-constexpr int kSelJ = 128;
+constexpr int kSelJ = 64;
 
 __host__ __device__ constexpr size_t select_smem_bytes(int d, int nb) {
-    return (static_cast<size_t>(kSelQ + kSelJ) * (d + 4) + static_cast<size_t>(kSelQ) * nb) * 4 + 8 * 256 * 4;
+    return (static_cast<size_t>(kSelQ + kSelJ) * (d + 4) + static_cast<size_t>(kSelQ) * nb) * 4;
 }
 
 __device__ __forceinline__ uint32_t order_key(float x) {
@@ -109,16 +113,66 @@ __device__ __forceinline__ uint32_t order_key(float x) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-template <typename T>
+// Top-(want) of row[0..n) for one warp; KPL keys per lane (n <= 32*KPL).
+template <int KPL>
+__device__ __forceinline__ void select_row(const float *row, int n, int want, int bt, int k, int32_t *out, int lane) {
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    uint32_t key[KPL];
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+        const int j = 32 * i + lane;
+        key[i] = j < n ? order_key(row[j]) : 0u;  // 0 is below every real key
+    }
+    uint32_t tau = 0u;
+    int need_eq = 0;
+    if (want > 0 && want < n) {
+#pragma unroll 1
+        for (int b = 31; b >= 0; --b) {
+            const uint32_t cand = tau | (1u << b);
+            unsigned c = 0;
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) c += key[i] >= cand ? 1u : 0u;
+            if (__reduce_add_sync(0xffffffffu, c) >= static_cast<unsigned>(want)) tau = cand;
+        }
+        unsigned gt = 0;
+#pragma unroll
+        for (int i = 0; i < KPL; ++i) gt += key[i] > tau ? 1u : 0u;
+        need_eq = want - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+    }
+    int taken = 0, eq_seen = 0;
+    if (want > 0) {
+#pragma unroll
+        for (int i = 0; i < KPL; ++i) {
+            if (32 * i >= n) break;
+            const bool in = 32 * i + lane < n;
+            bool sel;
+            uint32_t eqb = 0u;
+            if (want < n) {
+                const bool eq = in && key[i] == tau;
+                eqb = __ballot_sync(0xffffffffu, eq);
+                sel = (in && key[i] > tau) || (eq && (eq_seen + __popc(eqb & lt_mask)) < need_eq);
+            } else {
+                sel = in;
+            }
+            const uint32_t sb = __ballot_sync(0xffffffffu, sel);
+            const int pos = taken + __popc(sb & lt_mask);
+            if (sel && pos < want) out[pos] = 32 * i + lane;
+            taken += __popc(sb);
+            eq_seen += __popc(eqb);
+        }
+    }
+    for (int i = want + lane; i < k; i += 32) out[i] = (i == want) ? bt : -1;
+}
+
+template <typename T, int KPL>
 __global__ void __launch_bounds__(256) select_kernel(const T *__restrict__ Q, const float *__restrict__ Kbar,
                                                      int32_t *__restrict__ idx, int T_len, int d, int s, int k,
                                                      int nb) {
     extern __shared__ __align__(16) float sm[];
     const int dp = d + 4;
     float *sQ = sm;                       // [32][dp]
-    float *sK = sQ + kSelQ * dp;          // [128][dp]
+    float *sK = sQ + kSelQ * dp;          // [64][dp]
     float *sS = sK + kSelJ * dp;          // [32][nb]
-    int *hist = reinterpret_cast<int *>(sS + kSelQ * nb);  // [8][256]
 
     const int bh = blockIdx.y, t0 = blockIdx.x * kSelQ;
     const int bt = t0 / s;
@@ -128,7 +182,6 @@ __global__ void __launch_bounds__(256) select_kernel(const T *__restrict__ Q, co
         const int qi = e / d, c = e % d;
         sQ[qi * dp + c] = to_f32(Q[(static_cast<size_t>(bh) * T_len + t0 + qi) * d + c]);
     }
-    const int qg = tid >> 5;  // queries 4*qg .. 4*qg+3
     for (int jc = 0; jc < bt; jc += kSelJ) {
         const int nj = min(kSelJ, bt - jc);
         __syncthreads();
@@ -138,21 +191,20 @@ __global__ void __launch_bounds__(256) select_kernel(const T *__restrict__ Q, co
                 __ldg(reinterpret_cast<const float4 *>(Kbar + (static_cast<size_t>(bh) * nb + jc + jj) * d) + c4);
         }
         __syncthreads();
-        float acc[4][4];
+        float acc[4][2];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+        for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = 0.f;
+#pragma unroll 4
         for (int c = 0; c < d; c += 4) {
-            float4 qv[4], kv[4];
+            float4 qv[4], kv[2];
 #pragma unroll
-            for (int a = 0; a < 4; ++a) qv[a] = *reinterpret_cast<const float4 *>(sQ + (4 * qg + a) * dp + c);
+            for (int a = 0; a < 4; ++a) qv[a] = *reinterpret_cast<const float4 *>(sQ + (4 * warp + a) * dp + c);
 #pragma unroll
-            for (int b = 0; b < 4; ++b) kv[b] = *reinterpret_cast<const float4 *>(sK + (lane + 32 * b) * dp + c);
+            for (int b = 0; b < 2; ++b) kv[b] = *reinterpret_cast<const float4 *>(sK + (lane + 32 * b) * dp + c);
 #pragma unroll
             for (int a = 0; a < 4; ++a)
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
+                for (int b = 0; b < 2; ++b) {
                     acc[a][b] = fmaf(qv[a].x, kv[b].x, acc[a][b]);
                     acc[a][b] = fmaf(qv[a].y, kv[b].y, acc[a][b]);
                     acc[a][b] = fmaf(qv[a].z, kv[b].z, acc[a][b]);
@@ -162,93 +214,16 @@ __global__ void __launch_bounds__(256) select_kernel(const T *__restrict__ Q, co
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
+            for (int b = 0; b < 2; ++b) {
                 const int jj = lane + 32 * b;
-                if (jj < nj) sS[(4 * qg + a) * nb + jc + jj] = acc[a][b];
+                if (jj < nj) sS[(4 * warp + a) * nb + jc + jj] = acc[a][b];
             }
     }
-    __syncthreads();
-
-    // phase 2: warp w selects for queries 4w .. 4w+3
-    int *h = hist + warp * 256;
+    __syncwarp();
     const int want = min(k - 1, bt);
-    const uint32_t lt_mask = (1u << lane) - 1u;
     for (int qq = 0; qq < 4; ++qq) {
         const int qi = 4 * warp + qq;
-        const float *row = sS + qi * nb;
-        int32_t *out = idx + (static_cast<size_t>(bh) * T_len + t0 + qi) * k;
-        uint32_t tau = 0u;
-        int need_eq = 0;  // how many scores equal to tau are taken
-        if (want > 0 && want < bt) {
-            uint32_t prefix = 0u, mask = 0u;
-            int rank = want;  // want-th largest (1-based)
-            for (int shift = 24; shift >= 0; shift -= 8) {
-                for (int b = lane; b < 256; b += 32) h[b] = 0;
-                __syncwarp();
-                for (int jj = lane; jj < bt; jj += 32) {
-                    const uint32_t key = order_key(row[jj]);
-                    if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1);
-                }
-                __syncwarp();
-                int c8[8], sum = 0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    c8[i] = h[255 - 8 * lane - i];
-                    sum += c8[i];
-                }
-                int incl = sum;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += v;
-                }
-                const int excl = incl - sum;
-                const bool here = excl < rank && rank <= incl;
-                const uint32_t who = __ballot_sync(0xffffffffu, here);
-                const int src = __ffs(who) - 1;
-                int digit = 0, new_rank = 0;
-                if (here) {
-                    int cum = excl;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        if (cum < rank && rank <= cum + c8[i]) {
-                            digit = 255 - 8 * lane - i;
-                            new_rank = rank - cum;
-                        }
-                        cum += c8[i];
-                    }
-                }
-                digit = __shfl_sync(0xffffffffu, digit, src);
-                rank = __shfl_sync(0xffffffffu, new_rank, src);
-                prefix |= static_cast<uint32_t>(digit) << shift;
-                mask |= 0xFFu << shift;
-                __syncwarp();
-            }
-            tau = prefix;
-            need_eq = rank;
-        }
-        int taken = 0, eq_seen = 0;
-        for (int j0 = 0; want > 0 && j0 < bt; j0 += 32) {
-            const int jj = j0 + lane;
-            const bool in = jj < bt;
-            const uint32_t key = in ? order_key(row[jj]) : 0u;
-            bool sel;
-            uint32_t eqb = 0u;
-            if (want < bt) {
-                const bool gt = in && key > tau;
-                const bool eq = in && key == tau;
-                eqb = __ballot_sync(0xffffffffu, eq);
-                sel = gt || (eq && (eq_seen + __popc(eqb & lt_mask)) < need_eq);
-            } else {
-                sel = in;
-            }
-            const uint32_t sb = __ballot_sync(0xffffffffu, sel);
-            const int pos = taken + __popc(sb & lt_mask);
-            if (sel && pos < want) out[pos] = jj;
-            taken += __popc(sb);
-            eq_seen += __popc(eqb);
-        }
-        for (int i = want + lane; i < k; i += 32) out[i] = (i == want) ? bt : -1;
+        select_row<KPL>(sS + qi * nb, bt, want, bt, k, idx + (static_cast<size_t>(bh) * T_len + t0 + qi) * k, lane);
     }
 }
 

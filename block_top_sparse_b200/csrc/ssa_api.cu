@@ -164,6 +164,13 @@ unsigned grid_for(size_t n, unsigned per_block) {
     return static_cast<unsigned>(g ? g : 1);
 }
 
+template <typename T, int KPL>
+ssa_status_t launch_select(const Shape &S, const void *Q, const float *Kbar, int32_t *idx, size_t sm, cudaStream_t st) {
+    if (!set_smem(select_kernel<T, KPL>, sm)) return SSA_ERR_CUDA;
+    select_kernel<T, KPL><<<dim3(S.T / kSelQ, S.BH), 256, sm, st>>>((const T *)Q, Kbar, idx, S.T, S.d, S.s, S.k, S.nb);
+    return SSA_OK;
+}
+
 // Inverse selection index: entries of block j of head bh (query order).
 ssa_status_t build_index(const Shape &S, const int32_t *idx, IndexWs &W, cudaStream_t st) {
     const size_t hbytes = static_cast<size_t>(S.nb) * 4;
@@ -313,15 +320,22 @@ ssa_status_t ssa_block_select(const ssa_dims_t *dims, const void *Q, const float
     const size_t sm = select_smem_bytes(S.d, S.nb);
     if (S.nb > 1024 || sm > 227 * 1024) return SSA_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const dim3 grid(S.T / kSelQ, S.BH);
     if (S.dtype == SSA_DT_BF16) {
-        if (!set_smem(select_kernel<__nv_bfloat16>, sm)) return SSA_ERR_CUDA;
-        select_kernel<__nv_bfloat16><<<grid, 256, sm, st>>>((const __nv_bfloat16 *)Q, Kbar, idx, S.T, S.d, S.s,
-                                                            S.k, S.nb);
+        if (S.nb <= 256)
+            e = launch_select<__nv_bfloat16, 8>(S, Q, Kbar, idx, sm, st);
+        else if (S.nb <= 512)
+            e = launch_select<__nv_bfloat16, 16>(S, Q, Kbar, idx, sm, st);
+        else
+            e = launch_select<__nv_bfloat16, 32>(S, Q, Kbar, idx, sm, st);
     } else {
-        if (!set_smem(select_kernel<float>, sm)) return SSA_ERR_CUDA;
-        select_kernel<float><<<grid, 256, sm, st>>>((const float *)Q, Kbar, idx, S.T, S.d, S.s, S.k, S.nb);
+        if (S.nb <= 256)
+            e = launch_select<float, 8>(S, Q, Kbar, idx, sm, st);
+        else if (S.nb <= 512)
+            e = launch_select<float, 16>(S, Q, Kbar, idx, sm, st);
+        else
+            e = launch_select<float, 32>(S, Q, Kbar, idx, sm, st);
     }
+    if (e != SSA_OK) return e;
     return launch_status();
 }
 
