@@ -58,6 +58,20 @@ __device__ __forceinline__ void gather_row(uint32_t tile, const __nv_bfloat16 *s
     }
 }
 
+// One warp gathers the 128 rows of a query tile (4 rows per lane) into a
+// 2-chunk swizzled tile; rows past the list are zero-filled.  The caller then
+// signals completion with cp_async_mbar_arrive_noinc().
+__device__ __forceinline__ void warp_gather_tile(uint32_t tile, const __nv_bfloat16 *base, const Rows &R, int T,
+                                                 int it, size_t head_rows, int lane) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int r = lane + 32 * q;
+        int t = 0, e = 0;
+        const bool valid = tile_row(R, T, it, r, t, e);
+        gather_row(tile, base + (head_rows + (valid ? t : 0)) * kD, valid, r);
+    }
+}
+
 // Write 32 fp32 values as bf16 into row r, columns [c0, c0+32) of a swizzled
 // multi-chunk tile (chunk = 64 columns, chunk stride `cstride` bytes).
 __device__ __forceinline__ void store_row32_bf16(uint32_t tile, uint32_t cstride, int r, int c0, const float (&v)[32]) {
@@ -194,13 +208,13 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 if (!mbar_wait(bar_p_full, n & 1, abort_flag, 0x105)) break;
                 tc_fence_after();
-                // O += P V : A = P [128 q x 128 kv] K-major, B = V [kv rows x d] MN-major.
+                // O += P V : A = P from tensor memory (bf16 pairs written over S), B = V [kv rows x d] MN-major.
                 const uint32_t vb = sV + st * 2 * kChunkBytes;
+                const uint32_t tP = tmem + st * 128;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t da = smem_desc_sw128(sP + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16);
                     const uint64_t db = smem_desc_sw128(vb + kk * 2048, kChunkBytes);
-                    mma_bf16_ss(tO, da, db, idO, (n > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16_ts(tO, tP + kk * 8, db, idO, (n > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(bar_o_full);
                 mma_commit(bar_kv_empty + st);
@@ -261,20 +275,24 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             l *= alpha;
-            // probabilities -> P (bf16) in shared memory
+            // probabilities -> P (bf16 pairs) in tensor memory, over the first 64 columns of S
+            uint32_t pw[2][32];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                float v[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float p =
+                for (int i = 0; i < 32; i += 2) {
+                    const float p0 =
                         (32 * c + i <= lim) ? fast_exp2(fmaf(__uint_as_float(sr[c][i]), scale_log2, -m_used)) : 0.f;
-                    l += p;
-                    v[i] = p;
+                    const float p1 = (32 * c + i + 1 <= lim)
+                                         ? fast_exp2(fmaf(__uint_as_float(sr[c][i + 1]), scale_log2, -m_used))
+                                         : 0.f;
+                    l += p0 + p1;
+                    pw[c >> 1][16 * (c & 1) + (i >> 1)] = pack_bf16x2(p0, p1);
                 }
-                store_row32_bf16(sP, kChunkBytes, r, 32 * c, v);
             }
-            fence_proxy_async_smem();
+            tmem_st32_u(tS, pw[0]);
+            tmem_st32_u(tS + 32, pw[1]);
+            tmem_st_wait();
             tc_fence_before();
             mbar_arrive(bar_p_full);
         }
@@ -306,25 +324,34 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Sparse forward, block-major.
-// grid = (B*H*nb): unit u -> block j = u / BH, head bh = u % BH.  block = 160.
-// For every tile of the block's query list: S = Q_g K_j^T, masked softmax over
-// the block's NKV keys, O = P V_j, partial (o / l, lse) stored per entry.
-// smem: Q 32 KB | K NKV*256 | V NKV*256 | P (NKV/64)*16 KB | barriers
-// tmem: S at 0, O at 128 (256 allocated).
+// Sparse forward, block-major, two warpgroups in ping-pong.
+// grid = (B*H*nb): unit u -> head bh = u / nb, block j = u % nb (head-major, so
+// the head's query rows stay in L2).  block = 320 threads:
+//   warpgroup g (warps 4g .. 4g+3) owns the query tiles it = g, g+2, ... of the
+//   block's list: masked softmax over the block's NKV keys, normalised partial
+//   (o / l, lse) per (query, slot);
+//   warp 9 gathers each tile's query rows (cp.async, completion on an mbarrier);
+//   warp 8 loads K_j, V_j (TMA) and issues the MMAs in the order
+//   S(it), PV(it-1), S(it+1), PV(it), ... so that one warpgroup's softmax
+//   overlaps the other's MMAs and epilogue.
+// smem: Q[2] 32 KB each | K, V NKV*256 each | P[2] (NKV/64)*16 KB each | barriers
+// tmem: S[2] at 0 / 128, O[2] at 256 / 384 (512 allocated).
 // ---------------------------------------------------------------------------
 template <int NKV>
 struct SparseFwdSmem {
-    static constexpr int kQ = 0;
-    static constexpr int kK = kQ + 2 * kChunkBytes;
+    static constexpr int kQ = 0;                          // [2]
+    static constexpr int kK = kQ + 2 * 2 * kChunkBytes;
     static constexpr int kV = kK + 2 * NKV * 128;
-    static constexpr int kP = kV + 2 * NKV * 128;
-    static constexpr int kBar = kP + (NKV / 64) * kChunkBytes;
+    static constexpr int kP = kV + 2 * NKV * 128;         // [2]
+    static constexpr int kPStage = (NKV / 64) * kChunkBytes;
+    static constexpr int kBar = kP + 2 * kPStage;
     static constexpr int kTotal = kBar + 256;
 };
 
+constexpr int kSparseFwdThreads = 320;
+
 template <int NKV>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(kSparseFwdThreads, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __nv_bfloat16 *__restrict__ Q, const int32_t *__restrict__ entries,
                       const int32_t *__restrict__ lstart, const int32_t *__restrict__ llen,
@@ -334,13 +361,18 @@ __global__ void __launch_bounds__(160, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
-    uint64_t *bar_kv = bars + 0, *bar_q_full = bars + 1, *bar_s_full = bars + 2, *bar_p_full = bars + 3;
-    uint64_t *bar_o_full = bars + 4, *bar_o_empty = bars + 5, *bar_final = bars + 6;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 8);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 9);
+    uint64_t *bar_kv = bars + 0;
+    uint64_t *bar_q_full = bars + 1;   // [2]
+    uint64_t *bar_s_full = bars + 3;   // [2]
+    uint64_t *bar_p_full = bars + 5;   // [2]
+    uint64_t *bar_o_full = bars + 7;   // [2]
+    uint64_t *bar_o_empty = bars + 9;  // [2]
+    uint64_t *bar_final = bars + 11;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 15);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int j = blockIdx.x / BH, bh = blockIdx.x % BH;
+    const int bh = blockIdx.x / nb, j = blockIdx.x % nb;
     const int kv0 = j * NKV;
     const size_t head_rows = static_cast<size_t>(bh) * T;
     Rows R;
@@ -350,31 +382,40 @@ __global__ void __launch_bounds__(160, 1)
     R.k = k;
     const int ntiles = (R.len + kTileQ - 1) / kTileQ;
 
-    const uint32_t sQ = smem_u32(smem + L::kQ), sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV),
-                   sP = smem_u32(smem + L::kP);
-
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
-        mbar_init(bar_q_full, 128);
-        mbar_init(bar_s_full, 1);
-        mbar_init(bar_p_full, 128);
-        mbar_init(bar_o_full, 1);
-        mbar_init(bar_o_empty, 128);
+        for (int g = 0; g < 2; ++g) {
+            mbar_init(bar_q_full + g, 32);  // one cp.async arrival per lane of the gather warp
+            mbar_init(bar_s_full + g, 1);
+            mbar_init(bar_p_full + g, 128);
+            mbar_init(bar_o_full + g, 1);
+            mbar_init(bar_o_empty + g, 128);
+        }
         mbar_init(bar_final, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tO = tmem + 128;
+    const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
 
-    if (warp == 4) {
+    if (warp == 9) {
+        // ---------------- gather warp: query rows of tile it into Q[it & 1] ----------------
+        for (int it = 0; it < ntiles; ++it) {
+            const int g = it & 1;
+            // Q[g] is free once the S MMA of tile it-2 has completed
+            if (it >= 2 && !mbar_wait(bar_s_full + g, ((it - 2) >> 1) & 1, abort_flag, 0x208)) break;
+            warp_gather_tile(smem_u32(smem + L::kQ + g * 2 * kChunkBytes), Q, R, T, it, head_rows, lane);
+            cp_async_mbar_arrive_noinc(bar_q_full + g);
+        }
+        cp_async_wait_all();
+    } else if (warp == 8) {
         if (lane == 0) {
             mbar_arrive_expect_tx(bar_kv, 4 * NKV * 128);
             tma_load_2d(&tmK, bar_kv, smem + L::kK, 0, static_cast<int>(head_rows) + kv0);
@@ -384,110 +425,103 @@ __global__ void __launch_bounds__(160, 1)
             const uint32_t idS = idesc_bf16(128, NKV, false, false);
             const uint32_t idO = idesc_bf16(128, 128, false, true);
             bool ok = mbar_wait(bar_kv, 0, abort_flag, 0x201);
-            for (int it = 0; ok && it < ntiles; ++it) {
-                if (!mbar_wait(bar_q_full, it & 1, abort_flag, 0x202)) break;
-                if (it > 0 && !mbar_wait(bar_o_empty, (it - 1) & 1, abort_flag, 0x203)) break;
-                tc_fence_after();
-                mma_k128_kmajor(tS, sQ, sK, NKV * 128, idS);
-                mma_commit(bar_s_full);
-                if (!mbar_wait(bar_p_full, it & 1, abort_flag, 0x204)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < NKV / 16; ++kk) {
-                    const uint64_t da = smem_desc_sw128(sP + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16);
-                    const uint64_t db = smem_desc_sw128(sV + kk * 2048, NKV * 128);
-                    mma_bf16_ss(tO, da, db, idO, kk > 0 ? 1u : 0u);
+            for (int it = 0; ok && it <= ntiles; ++it) {
+                if (it < ntiles) {
+                    const int g = it & 1, i = it >> 1;
+                    if (!mbar_wait(bar_q_full + g, i & 1, abort_flag, 0x202)) break;
+                    if (i > 0 && !mbar_wait(bar_o_empty + g, (i - 1) & 1, abort_flag, 0x203)) break;
+                    fence_proxy_async_smem();  // cp.async-written rows -> tensor-core reads
+                    tc_fence_after();
+                    mma_k128_kmajor(tmem + 128 * g, smem_u32(smem + L::kQ + g * 2 * kChunkBytes), sK, NKV * 128,
+                                    idS);
+                    mma_commit(bar_s_full + g);
                 }
-                mma_commit(bar_o_full);
+                if (it >= 1) {
+                    const int g = (it - 1) & 1, i = (it - 1) >> 1;
+                    if (!mbar_wait(bar_p_full + g, i & 1, abort_flag, 0x204)) break;
+                    tc_fence_after();
+                    const uint32_t sP = smem_u32(smem + L::kP + g * L::kPStage);
+#pragma unroll
+                    for (int kk = 0; kk < NKV / 16; ++kk)
+                        mma_bf16_ss(tmem + 256 + 128 * g,
+                                    smem_desc_sw128(sP + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16),
+                                    smem_desc_sw128(sV + kk * 2048, NKV * 128), idO, kk > 0 ? 1u : 0u);
+                    mma_commit(bar_o_full + g);
+                }
             }
             mma_commit(bar_final);
             mbar_wait(bar_final, 0, abort_flag, 0x205);
         }
     } else {
-        const int r = threadIdx.x;
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        int t = 0, e = 0;
-        bool valid = ntiles > 0 && tile_row(R, T, 0, r, t, e);
-        gather_row(sQ, Q + (head_rows + (valid ? t : 0)) * kD, valid, r);
-        cp_async_commit();
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        mbar_arrive(bar_q_full);
-        for (int it = 0; it < ntiles; ++it) {
-            if (!mbar_wait(bar_s_full, it & 1, abort_flag, 0x206)) break;
+        const int g = warp >> 2;                  // warpgroup: tiles g, g+2, ...
+        const int r = ((warp & 3) << 5) | lane;   // tile row
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t sP = smem_u32(smem + L::kP + g * L::kPStage);
+        const uint32_t tS = tmem + 128 * g + lane_off, tO = tmem + 256 + 128 * g + lane_off;
+        for (int it = g; it < ntiles; it += 2) {
+            const int i = it >> 1;
+            int t = 0, e = 0;
+            const bool valid = tile_row(R, T, it, r, t, e);  // load overlaps the wait below
+            if (!mbar_wait(bar_s_full + g, i & 1, abort_flag, 0x206)) break;
             tc_fence_after();
             uint32_t sr[NKV / 32][32];
 #pragma unroll
-            for (int c = 0; c < NKV / 32; ++c) tmem_ld32_async(tS + lane_off + 32 * c, sr[c]);
+            for (int c = 0; c < NKV / 32; ++c) tmem_ld32_async(tS + 32 * c, sr[c]);
             tmem_ld_wait();
             // key kv0 + col is attended when col <= lim (causal inside the query's own block)
             const int lim = valid ? t - kv0 : -1;
-            float mx = -INFINITY;
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int c = 0; c < NKV / 32; ++c)
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    mx = fmaxf(mx, (32 * c + i <= lim) ? __uint_as_float(sr[c][i]) * scale_log2 : -INFINITY);
+                for (int i2 = 0; i2 < 32; ++i2)
+                    mx4[i2 & 3] = fmaxf(mx4[i2 & 3], (32 * c + i2 <= lim) ? __uint_as_float(sr[c][i2]) : -INFINITY);
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
             const float mref = (mx == -INFINITY) ? 0.f : mx;
-            float l = 0.f;
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < NKV / 32; ++c) {
                 float v[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i2 = 0; i2 < 32; ++i2) {
                     const float p =
-                        (32 * c + i <= lim) ? fast_exp2(fmaf(__uint_as_float(sr[c][i]), scale_log2, -mref)) : 0.f;
-                    l += p;
-                    v[i] = p;
+                        (32 * c + i2 <= lim) ? fast_exp2(fmaf(__uint_as_float(sr[c][i2]), scale_log2, -mref)) : 0.f;
+                    l4[i2 & 3] += p;
+                    v[i2] = p;
                 }
                 store_row32_bf16(sP, kChunkBytes, r, 32 * c, v);
             }
+            const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(bar_p_full);
-            if (!mbar_wait(bar_o_full, it & 1, abort_flag, 0x207)) break;
+            mbar_arrive(bar_p_full + g);
+            if (!mbar_wait(bar_o_full + g, i & 1, abort_flag, 0x207)) break;
             tc_fence_after();
-            // prefetch the next tile's query rows (S of this tile is complete)
-            int t_next = 0, e_next = 0;
-            bool valid_next = false;
-            if (it + 1 < ntiles) {
-                valid_next = tile_row(R, T, it + 1, r, t_next, e_next);
-                gather_row(sQ, Q + (head_rows + (valid_next ? t_next : 0)) * kD, valid_next, r);
-                cp_async_commit();
-            }
-            const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-            __nv_bfloat16 *dst = Opart + (head_rows * k + (valid ? e : 0)) * kD;
-            for (int c0 = 0; c0 < 128; c0 += 32) {
-                float o[32];
-                tmem_ld32(tO + lane_off + c0, o);
-                if (valid) {
-                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + c0);
+            uint32_t orow[4][32];
 #pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        d4[g] = make_uint4(pack_bf16x2(o[8 * g] * inv_l, o[8 * g + 1] * inv_l),
-                                           pack_bf16x2(o[8 * g + 2] * inv_l, o[8 * g + 3] * inv_l),
-                                           pack_bf16x2(o[8 * g + 4] * inv_l, o[8 * g + 5] * inv_l),
-                                           pack_bf16x2(o[8 * g + 6] * inv_l, o[8 * g + 7] * inv_l));
-                }
-            }
-            if (valid) lsepart[head_rows * k + e] = (l > 0.f) ? (mref + __log2f(l)) * kLn2 : -INFINITY;
+            for (int c = 0; c < 4; ++c) tmem_ld32_async(tO + 32 * c, orow[c]);
+            tmem_ld_wait();
             tc_fence_before();
-            mbar_arrive(bar_o_empty);
-            if (it + 1 < ntiles) {
-                cp_async_wait_all();
-                fence_proxy_async_smem();
-                mbar_arrive(bar_q_full);
-                t = t_next;
-                e = e_next;
-                valid = valid_next;
+            mbar_arrive(bar_o_empty + g);
+            if (valid) {
+                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+                uint4 *d4 = reinterpret_cast<uint4 *>(Opart + (head_rows * k + e) * kD);
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const uint32_t *x = orow[q >> 2] + 8 * (q & 3);
+                    d4[q] = make_uint4(pack_bf16x2(__uint_as_float(x[0]) * inv_l, __uint_as_float(x[1]) * inv_l),
+                                       pack_bf16x2(__uint_as_float(x[2]) * inv_l, __uint_as_float(x[3]) * inv_l),
+                                       pack_bf16x2(__uint_as_float(x[4]) * inv_l, __uint_as_float(x[5]) * inv_l),
+                                       pack_bf16x2(__uint_as_float(x[6]) * inv_l, __uint_as_float(x[7]) * inv_l));
+                }
+                lsepart[head_rows * k + e] = (l > 0.f) ? (mref + __log2f(l)) * kLn2 : -INFINITY;
             }
         }
-        cp_async_wait_all();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, 256);
+    if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace ssa

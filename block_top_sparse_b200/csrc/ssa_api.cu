@@ -368,13 +368,13 @@ ssa_status_t ssa_sparse_attn_fwd(const ssa_dims_t *dims, const void *Q, const vo
     if (S.s == 128) {
         const size_t sm = SparseFwdSmem<128>::kTotal + 1024;
         if (!set_smem(sparse_fwd_kernel<128>, sm)) return SSA_ERR_CUDA;
-        sparse_fwd_kernel<128><<<units, 160, sm, st>>>(tmK, tmV, (const __nv_bfloat16 *)Q, W.entries, W.lstart,
+        sparse_fwd_kernel<128><<<units, kSparseFwdThreads, sm, st>>>(tmK, tmV, (const __nv_bfloat16 *)Q, W.entries, W.lstart,
                                                        W.llen, Opart, lsepart, static_cast<int>(S.BH), S.T, S.k,
                                                        S.nb, sl2);
     } else {
         const size_t sm = SparseFwdSmem<64>::kTotal + 1024;
         if (!set_smem(sparse_fwd_kernel<64>, sm)) return SSA_ERR_CUDA;
-        sparse_fwd_kernel<64><<<units, 160, sm, st>>>(tmK, tmV, (const __nv_bfloat16 *)Q, W.entries, W.lstart,
+        sparse_fwd_kernel<64><<<units, kSparseFwdThreads, sm, st>>>(tmK, tmV, (const __nv_bfloat16 *)Q, W.entries, W.lstart,
                                                       W.llen, Opart, lsepart, static_cast<int>(S.BH), S.T, S.k,
                                                       S.nb, sl2);
     }
