@@ -61,11 +61,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const BwdArgs a) {
     using L = BwdSmem<NKV>;
     constexpr int HALF = NKV / 2;  // S / dP columns per warpgroup
+    // 128-key units stage the dQ tile (64 KB) through the P / dS buffers and add it
+    // with coalesced row reductions; 64-key units (buffers of 32 KB) add per row.
+    constexpr bool kCoalescedFlush = NKV == 128;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
     uint64_t *bar_kv = bars + 0, *bar_qdo_full = bars + 1, *bar_sdp_full = bars + 2, *bar_pds_full = bars + 3;
     uint64_t *bar_qdo_free = bars + 4, *bar_dq_full = bars + 5, *bar_dq_empty = bars + 6, *bar_final = bars + 7;
+    uint64_t *bar_staged = bars + 8, *bar_flushed = bars + 9;  // dQ staging in the P / dS buffers
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 11);
 
@@ -103,6 +107,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(bar_dq_full, 1);
         mbar_init(bar_dq_empty, 256);
         mbar_init(bar_final, 1);
+        mbar_init(bar_staged, 256);
+        mbar_init(bar_flushed, 256);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -201,6 +207,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 break;
             }
             tc_fence_after();
+            // the previous tile's dQ flush staged through P / dS: wait until it has read them
+            if (kCoalescedFlush && it > 0 && !mbar_wait(bar_flushed, (it - 1) & 1, abort_flag, 0x309)) {
+                ok = false;
+                break;
+            }
             // all tensor-memory loads of this row half in flight at once, one wait
             uint32_t sraw[HALF / 32][32], draw[HALF / 32][32];
 #pragma unroll
@@ -253,7 +264,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(bar_dq_empty);
-            if (valid) {
+            if constexpr (kCoalescedFlush) {
+                // Stage the tile's dQ rows (fp32, 512 B per row, 16-byte units XOR-swizzled by
+                // row) in the P / dS buffers, free once every MMA of this tile has completed;
+                // then each warp adds 16 whole rows with coalesced float4 reductions.
+                auto stage_addr = [&](int row, int unit) -> uint32_t {
+                    const uint32_t base = row < 64 ? sP + row * 512 : sdS + (row - 64) * 512;
+                    return base + (((unit ^ row) & 31) << 4);
+                };
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const uint32_t *x = g[q >> 3] + 4 * (q & 7);
+                    st_shared_v4(stage_addr(r, 16 * h + q), __float_as_uint(__uint_as_float(x[0]) * a.scale),
+                                 __float_as_uint(__uint_as_float(x[1]) * a.scale),
+                                 __float_as_uint(__uint_as_float(x[2]) * a.scale),
+                                 __float_as_uint(__uint_as_float(x[3]) * a.scale));
+                }
+                mbar_arrive(bar_staged);
+                if (!mbar_wait(bar_staged, it & 1, abort_flag, 0x30a)) {
+                    ok = false;
+                    break;
+                }
+                const int t_mine = valid ? t : -1;
+#pragma unroll 4
+                for (int i = 0; i < 16; ++i) {
+                    const int row = 32 * (warp & 3) + 16 * h + i;
+                    const int t_dst = __shfl_sync(0xffffffffu, t_mine, 16 * h + i);
+                    if (t_dst >= 0) {
+                        float4 v;
+                        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                                     : "r"(stage_addr(row, lane)));
+                        atomicAdd(reinterpret_cast<float4 *>(a.dQacc + (head_rows + t_dst) * kD) + lane, v);
+                    }
+                }
+                mbar_arrive(bar_flushed);
+            } else if (valid) {
                 float4 *dq = reinterpret_cast<float4 *>(a.dQacc + (head_rows + t) * kD + h * 64);
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {

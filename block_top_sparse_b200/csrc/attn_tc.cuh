@@ -28,11 +28,16 @@ constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16
 struct Rows {
     // Row source of a query tile: contiguous (full attention) or gathered from
     // the inverse selection index (sparse attention).
-    const int32_t *list;  // entries t*k + slot, or nullptr for contiguous rows
+    const int32_t *list;  // entries (t << 8) | slot, or nullptr for contiguous rows
     int len;              // number of rows in the list / valid rows overall
     int first;            // contiguous: first query position
     int k;
 };
+
+// Row of the [.., T, k] per-(query, slot) arrays addressed by an index entry.
+__device__ __forceinline__ size_t entry_row(int entry, int k) {
+    return static_cast<size_t>(entry >> 8) * k + (entry & 255);
+}
 
 // Query position and global selection entry of tile row r of tile `it`.
 __device__ __forceinline__ bool tile_row(const Rows &R, int T, int it, int r, int &t, int &entry) {
@@ -40,7 +45,7 @@ __device__ __forceinline__ bool tile_row(const Rows &R, int T, int it, int r, in
         const int li = it * kTileQ + r;
         if (li >= R.len) return false;
         entry = __ldg(R.list + li);
-        t = entry / R.k;
+        t = entry >> 8;
         return true;
     }
     t = R.first + it * kTileQ + r;
@@ -505,7 +510,7 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
             mbar_arrive(bar_o_empty + g);
             if (valid) {
                 const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-                uint4 *d4 = reinterpret_cast<uint4 *>(Opart + (head_rows * k + e) * kD);
+                uint4 *d4 = reinterpret_cast<uint4 *>(Opart + (head_rows * k + entry_row(e, k)) * kD);
 #pragma unroll
                 for (int q = 0; q < 16; ++q) {
                     const uint32_t *x = orow[q >> 2] + 8 * (q & 3);
@@ -514,7 +519,7 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
                                        pack_bf16x2(__uint_as_float(x[4]) * inv_l, __uint_as_float(x[5]) * inv_l),
                                        pack_bf16x2(__uint_as_float(x[6]) * inv_l, __uint_as_float(x[7]) * inv_l));
                 }
-                lsepart[head_rows * k + e] = (l > 0.f) ? (mref + __log2f(l)) * kLn2 : -INFINITY;
+                lsepart[head_rows * k + entry_row(e, k)] = (l > 0.f) ? (mref + __log2f(l)) * kLn2 : -INFINITY;
             }
         }
     }

@@ -84,8 +84,9 @@ __global__ void __launch_bounds__(1024) index_scan_kernel(int *__restrict__ cnt,
     }
 }
 
-// Pass 3: one warp per chunk writes entries t*k + slot at their final position,
-// in ascending query order (ranks within a 32-query step come from lane bitmasks).
+// Pass 3: one warp per chunk writes entries (t << 8) | slot at their final
+// position, in ascending query order (ranks within a 32-query step come from
+// lane bitmasks).  k <= 256 and T < 2^23 keep the encoding in an int32.
 __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t *__restrict__ idx,
                                                          const int *__restrict__ off, int32_t *__restrict__ entries,
                                                          int T, int k, int nb, int nch) {
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t *__restri
         __syncwarp();
         for (int i = 0; i < k; ++i) {
             const int j = valid ? __ldg(row + i) : -1;
-            if (j >= 0 && j < nb) dst[run[j] + __popc(bits[j] & lt_mask)] = t * k + i;
+            if (j >= 0 && j < nb) dst[run[j] + __popc(bits[j] & lt_mask)] = (t << 8) | i;
         }
         __syncwarp();
         for (int i = 0; i < k; ++i) {

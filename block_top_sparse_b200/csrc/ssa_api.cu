@@ -58,6 +58,8 @@ ssa_status_t check_dims(const ssa_dims_t *dims, Shape &S, bool need_k) {
     }
     S.esz = S.dtype == SSA_DT_BF16 ? 2 : 4;
     S.tc = S.dtype == SSA_DT_BF16 && S.d == 128;
+    // the sparse index packs (t << 8) | slot into an int32
+    if (need_k && S.tc && (S.k > 256 || S.T >= (1 << 23))) return SSA_ERR_UNSUPPORTED;
     return SSA_OK;
 }
 
