@@ -107,21 +107,32 @@ __device__ __forceinline__ void mma_k128_kmajor(uint32_t d_tmem, uint32_t a, uin
 }
 
 // ---------------------------------------------------------------------------
-// Full causal attention forward.
-// grid = (ceil(T/128), B*H); block = 192 threads.
-// smem: Q 32 KB | K[2] 64 KB | V[2] 64 KB | P 32 KB | barriers
-// tmem: S[2] at columns 0 / 128, O at 256 (512 allocated).
+// Full causal attention forward, two query tiles per CTA in ping-pong.
+// grid = (ceil(T/256), B*H), heaviest query blocks first; block = 384 threads.
+//   warpgroup x in {0, 1} owns query tile x (rows 256*qb + 128*x + row): online
+//   softmax over the key tiles 0..diag(x) with lazy rescaling of O (only when the
+//   running maximum grows by more than 2^8), P written as bf16 pairs over S in
+//   tensor memory;
+//   warp 8 issues S_a(0), S_b(0), then per key tile n:
+//     PV_a(n), S_a(n+1), PV_b(n), S_b(n+1)
+//   so that one warpgroup's softmax overlaps the other's MMAs;
+//   warp 9 streams K/V tiles by TMA through a 2-stage ring; warps 10-11 idle.
+// smem: Q_a, Q_b 64 KB | K/V 2 stages x 64 KB | barriers
+// tmem: S_a 0, S_b 128, O_a 256, O_b 384 (512 allocated).
 // ---------------------------------------------------------------------------
 struct FullFwdSmem {
-    static constexpr int kQ = 0;
-    static constexpr int kK = kQ + 2 * kChunkBytes;
-    static constexpr int kV = kK + 2 * 2 * kChunkBytes;
-    static constexpr int kP = kV + 2 * 2 * kChunkBytes;
-    static constexpr int kBar = kP + 2 * kChunkBytes;
+    static constexpr int kQ = 0;                              // [2 tiles] x 32 KB
+    static constexpr int kK = kQ + 2 * 2 * kChunkBytes;       // [2 stages] x 32 KB
+    static constexpr int kV = kK + 2 * 2 * kChunkBytes;       // [2 stages] x 32 KB
+    static constexpr int kBar = kV + 2 * 2 * kChunkBytes;
     static constexpr int kTotal = kBar + 256;
 };
 
-__global__ void __launch_bounds__(192, 1)
+// 384 threads launched with 168 registers each (64,512); softmax warpgroups grow
+// to 224 and the MMA / producer warpgroup shrinks to 56: 2*128*224 + 128*56 = 64,512.
+constexpr int kFullFwdThreads = 384;
+
+__global__ void __launch_bounds__(kFullFwdThreads, 1)
     full_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ O, float *__restrict__ lse,
                     int T, float scale_log2) {
@@ -131,24 +142,21 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t *bar_q = bars + 0;
     uint64_t *bar_kv_full = bars + 1;   // [2]
     uint64_t *bar_kv_empty = bars + 3;  // [2]
-    uint64_t *bar_s_full = bars + 5;    // [2]
-    uint64_t *bar_p_full = bars + 7;
-    uint64_t *bar_o_full = bars + 8;
-    uint64_t *bar_final = bars + 9;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 12);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 13);
+    uint64_t *bar_s_full = bars + 5;    // [2 tiles]
+    uint64_t *bar_p_full = bars + 7;    // [2 tiles]
+    uint64_t *bar_o_full = bars + 9;    // [2 tiles]
+    uint64_t *bar_final = bars + 11;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 13);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 14);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nq = (T + kTileQ - 1) / kTileQ;
-    const int m = nq - 1 - blockIdx.x;  // heaviest tiles first
+    const int nqb = (T + 255) / 256;
+    const int qb = nqb - 1 - blockIdx.x;  // heaviest query blocks first
     const int bh = blockIdx.y;
-    const int row0 = bh * T;            // first tensor-map row of this head
-    const int nkv = m + 1;              // causal key tiles 0..m
-
-    const uint32_t sQ = smem_u32(smem + FullFwdSmem::kQ);
-    const uint32_t sK = smem_u32(smem + FullFwdSmem::kK);
-    const uint32_t sV = smem_u32(smem + FullFwdSmem::kV);
-    const uint32_t sP = smem_u32(smem + FullFwdSmem::kP);
+    const int row0 = bh * T;              // first tensor-map row of this head
+    const int q0 = qb * 256;              // first query of tile a; tile b starts at q0 + 128
+    // key tiles 0 .. diag: tile a ends at key tile 2qb, tile b at 2qb+1
+    const int nkv_a = 2 * qb + 1, nkv_b = 2 * qb + 2;
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
@@ -156,9 +164,9 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(bar_kv_full + i, 1);
             mbar_init(bar_kv_empty + i, 1);
             mbar_init(bar_s_full + i, 1);
+            mbar_init(bar_p_full + i, 128);
+            mbar_init(bar_o_full + i, 1);
         }
-        mbar_init(bar_p_full, 128);
-        mbar_init(bar_o_full, 1);
         mbar_init(bar_final, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -171,15 +179,18 @@ __global__ void __launch_bounds__(192, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS0 = tmem, tO = tmem + 256;
 
-    if (warp == 5) {
+    if (warp >= 8) regs_shrink<56>();
+    if (warp == 9) {
         // ---------------- TMA producer ----------------
         if (lane == 0) {
-            mbar_arrive_expect_tx(bar_q, 2 * kChunkBytes);
-            tma_load_2d(&tmQ, bar_q, smem + FullFwdSmem::kQ, 0, row0 + m * kTileQ);
-            tma_load_2d(&tmQ, bar_q, smem + FullFwdSmem::kQ + kChunkBytes, 64, row0 + m * kTileQ);
-            for (int n = 0; n < nkv; ++n) {
+            mbar_arrive_expect_tx(bar_q, 4 * kChunkBytes);
+            for (int x = 0; x < 2; ++x) {
+                uint8_t *q = smem + FullFwdSmem::kQ + x * 2 * kChunkBytes;
+                tma_load_2d(&tmQ, bar_q, q, 0, row0 + q0 + 128 * x);
+                tma_load_2d(&tmQ, bar_q, q + kChunkBytes, 64, row0 + q0 + 128 * x);
+            }
+            for (int n = 0; n < nkv_b; ++n) {
                 const int st = n & 1;
                 if (n >= 2 && !mbar_wait(bar_kv_empty + st, ((n >> 1) - 1) & 1, abort_flag, 0x101)) break;
                 mbar_arrive_expect_tx(bar_kv_full + st, 4 * kChunkBytes);
@@ -191,70 +202,94 @@ __global__ void __launch_bounds__(192, 1)
                 tma_load_2d(&tmV, bar_kv_full + st, v + kChunkBytes, 64, row0 + n * kTileQ);
             }
         }
-    } else if (warp == 4) {
+    } else if (warp == 8) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             const uint32_t idS = idesc_bf16(128, 128, false, false);
             const uint32_t idO = idesc_bf16(128, 128, false, true);
+            const uint32_t sQ = smem_u32(smem + FullFwdSmem::kQ);
+            const uint32_t sK = smem_u32(smem + FullFwdSmem::kK), sV = smem_u32(smem + FullFwdSmem::kV);
+            auto issue_S = [&](int x, int n) {
+                mma_k128_kmajor(tmem + 128 * x, sQ + x * 2 * kChunkBytes, sK + (n & 1) * 2 * kChunkBytes, kChunkBytes,
+                                idS);
+                mma_commit(bar_s_full + x);
+            };
+            auto issue_PV = [&](int x, int n) {
+                // O_x += P_x V_n : A = P from tensor memory (bf16 pairs over S_x), B = V [kv rows x d] MN-major
+                const uint32_t vb = sV + (n & 1) * 2 * kChunkBytes;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ts(tmem + 256 + 128 * x, tmem + 128 * x + kk * 8, smem_desc_sw128(vb + kk * 2048, kChunkBytes),
+                                idO, (n > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar_o_full + x);
+            };
             bool ok = mbar_wait(bar_q, 0, abort_flag, 0x102) && mbar_wait(bar_kv_full, 0, abort_flag, 0x103);
             if (ok) {
                 tc_fence_after();
-                mma_k128_kmajor(tS0, sQ, sK, kChunkBytes, idS);
-                mma_commit(bar_s_full);
+                issue_S(0, 0);
+                issue_S(1, 0);
             }
-            for (int n = 0; ok && n < nkv; ++n) {
-                const int st = n & 1;
-                if (n + 1 < nkv) {
-                    const int s1 = (n + 1) & 1;
-                    if (!mbar_wait(bar_kv_full + s1, ((n + 1) >> 1) & 1, abort_flag, 0x104)) break;
+            for (int n = 0; ok && n < nkv_b; ++n) {
+                bool next_ready = false;
+                auto wait_next = [&]() {
+                    if (!next_ready) {
+                        next_ready = true;
+                        if (!mbar_wait(bar_kv_full + ((n + 1) & 1), ((n + 1) >> 1) & 1, abort_flag, 0x104)) return false;
+                        tc_fence_after();
+                    }
+                    return true;
+                };
+                if (n < nkv_a) {
+                    if (!mbar_wait(bar_p_full + 0, n & 1, abort_flag, 0x105)) break;
                     tc_fence_after();
-                    mma_k128_kmajor(tmem + s1 * 128, sQ, sK + s1 * 2 * kChunkBytes, kChunkBytes, idS);
-                    mma_commit(bar_s_full + s1);
+                    issue_PV(0, n);
+                    if (n + 1 < nkv_a) {
+                        if (!wait_next()) break;
+                        issue_S(0, n + 1);
+                    }
                 }
-                if (!mbar_wait(bar_p_full, n & 1, abort_flag, 0x105)) break;
+                if (!mbar_wait(bar_p_full + 1, n & 1, abort_flag, 0x106)) break;
                 tc_fence_after();
-                // O += P V : A = P from tensor memory (bf16 pairs written over S), B = V [kv rows x d] MN-major.
-                const uint32_t vb = sV + st * 2 * kChunkBytes;
-                const uint32_t tP = tmem + st * 128;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t db = smem_desc_sw128(vb + kk * 2048, kChunkBytes);
-                    mma_bf16_ts(tO, tP + kk * 8, db, idO, (n > 0 || kk > 0) ? 1u : 0u);
+                issue_PV(1, n);
+                if (n + 1 < nkv_b) {
+                    if (!wait_next()) break;
+                    issue_S(1, n + 1);
                 }
-                mma_commit(bar_o_full);
-                mma_commit(bar_kv_empty + st);
+                mma_commit(bar_kv_empty + (n & 1));  // every MMA reading stage n&1 has been issued
             }
             mma_commit(bar_final);
-            mbar_wait(bar_final, 0, abort_flag, 0x106);
+            mbar_wait(bar_final, 0, abort_flag, 0x107);
         }
-    } else {
-        // ---------------- softmax warps (thread r <-> query row r) ----------------
-        const int r = threadIdx.x;
-        const int t = m * kTileQ + r;
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    } else if (warp < 8) {
+        // ---------------- softmax warpgroup x (thread <-> query row) ----------------
+        regs_grow<224>();
+        const int x = warp >> 2;
+        const int r = ((warp & 3) << 5) | lane;
+        const int t = q0 + 128 * x + r;
+        const int nkv = x == 0 ? nkv_a : nkv_b;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + 128 * x + lane_off, tO = tmem + 256 + 128 * x + lane_off;
         float m_used = -INFINITY, l = 0.f;
         bool ok = true;
         for (int n = 0; n < nkv; ++n) {
-            const int sb = n & 1;
-            if (!mbar_wait(bar_s_full + sb, (n >> 1) & 1, abort_flag, 0x107)) {
+            if (!mbar_wait(bar_s_full + x, n & 1, abort_flag, 0x108)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t tS = tmem + sb * 128 + lane_off;
-            // the whole S row in registers: four loads in flight, one wait
             uint32_t sr[4][32];
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_ld32_async(tS + 32 * c, sr[c]);
             tmem_ld_wait();
             // key n*128 + col is attended when col <= lim (causal on the diagonal tile)
-            const int lim = (n == m) ? t - n * kTileQ : 127;
-            float mx = -INFINITY;
+            const int lim = (n == nkv - 1) ? t - n * kTileQ : 127;
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int c = 0; c < 4; ++c)
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    mx = fmaxf(mx, (32 * c + i <= lim) ? __uint_as_float(sr[c][i]) * scale_log2 : -INFINITY);
+                    mx4[i & 3] = fmaxf(mx4[i & 3], (32 * c + i <= lim) ? __uint_as_float(sr[c][i]) : -INFINITY);
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
             float alpha = 1.f;
             if (n == 0) {
                 m_used = mx;
@@ -262,28 +297,28 @@ __global__ void __launch_bounds__(192, 1)
                 alpha = fast_exp2(m_used - mx);
                 m_used = mx;
             }
-            if (n > 0) {
-                // PV of the previous tile must be done before P is overwritten / O rescaled.
-                if (!mbar_wait(bar_o_full, (n - 1) & 1, abort_flag, 0x108)) {
+            if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                // the previous PV of this tile must be complete before O is rescaled
+                if (!mbar_wait(bar_o_full + x, (n - 1) & 1, abort_flag, 0x109)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
-                    for (int c0 = 0; c0 < 128; c0 += 32) {
-                        float o[32];
-                        tmem_ld32(tO + lane_off + c0, o);
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    float o[32];
+                    tmem_ld32(tO + c0, o);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                        tmem_st32(tO + lane_off + c0, o);
-                    }
+                    for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                    tmem_st32(tO + c0, o);
                 }
             }
             l *= alpha;
             // probabilities -> P (bf16 pairs) in tensor memory, over the first 64 columns of S
-            uint32_t pw[2][32];
+            // (chunk c of S lands in packed columns 16c .. 16c+15; every S value is already in registers)
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
+                uint32_t pw[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
                     const float p0 =
@@ -291,35 +326,39 @@ __global__ void __launch_bounds__(192, 1)
                     const float p1 = (32 * c + i + 1 <= lim)
                                          ? fast_exp2(fmaf(__uint_as_float(sr[c][i + 1]), scale_log2, -m_used))
                                          : 0.f;
-                    l += p0 + p1;
-                    pw[c >> 1][16 * (c & 1) + (i >> 1)] = pack_bf16x2(p0, p1);
+                    l4[(i >> 1) & 3] += p0 + p1;
+                    pw[i >> 1] = pack_bf16x2(p0, p1);
                 }
+                tmem_st16_u(tS + 16 * c, pw);
             }
-            tmem_st32_u(tS, pw[0]);
-            tmem_st32_u(tS + 32, pw[1]);
+            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(bar_p_full);
+            mbar_arrive(bar_p_full + x);
         }
-        if (ok && mbar_wait(bar_o_full, (nkv - 1) & 1, abort_flag, 0x109)) {
+        if (ok && mbar_wait(bar_o_full + x, (nkv - 1) & 1, abort_flag, 0x10a)) {
             tc_fence_after();
             const float inv_l = 1.f / l;
-            const bool valid = t < T;
-            __nv_bfloat16 *dst = O + (static_cast<size_t>(row0) + (valid ? t : 0)) * kD;
-            for (int c0 = 0; c0 < 128; c0 += 32) {
-                float o[32];
-                tmem_ld32(tO + lane_off + c0, o);  // warp-collective: outside the per-row branch
-                if (valid) {
-                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + c0);
+            uint4 *d4 = reinterpret_cast<uint4 *>(O + (static_cast<size_t>(row0) + (t < T ? t : 0)) * kD);
 #pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        d4[g] = make_uint4(pack_bf16x2(o[8 * g] * inv_l, o[8 * g + 1] * inv_l),
-                                           pack_bf16x2(o[8 * g + 2] * inv_l, o[8 * g + 3] * inv_l),
-                                           pack_bf16x2(o[8 * g + 4] * inv_l, o[8 * g + 5] * inv_l),
-                                           pack_bf16x2(o[8 * g + 6] * inv_l, o[8 * g + 7] * inv_l));
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t orow[2][32];
+                tmem_ld32_async(tO + 64 * hh, orow[0]);  // warp-collective: outside the row branch
+                tmem_ld32_async(tO + 64 * hh + 32, orow[1]);
+                tmem_ld_wait();
+                if (t < T) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint32_t *xo = orow[q >> 2] + 8 * (q & 3);
+                        d4[8 * hh + q] =
+                            make_uint4(pack_bf16x2(__uint_as_float(xo[0]) * inv_l, __uint_as_float(xo[1]) * inv_l),
+                                       pack_bf16x2(__uint_as_float(xo[2]) * inv_l, __uint_as_float(xo[3]) * inv_l),
+                                       pack_bf16x2(__uint_as_float(xo[4]) * inv_l, __uint_as_float(xo[5]) * inv_l),
+                                       pack_bf16x2(__uint_as_float(xo[6]) * inv_l, __uint_as_float(xo[7]) * inv_l));
+                    }
                 }
             }
-            if (valid) lse[static_cast<size_t>(row0) + t] = (m_used + __log2f(l)) * kLn2;
+            if (t < T) lse[static_cast<size_t>(row0) + t] = (m_used + __log2f(l)) * kLn2;
         }
     }
     tc_fence_before();
