@@ -370,7 +370,7 @@ __global__ void __launch_bounds__(kFullFwdThreads, 1)
 // ---------------------------------------------------------------------------
 // Sparse forward, block-major, two warpgroups in ping-pong.
 // grid = (B*H*nb): unit u -> head bh = u / nb, block j = u % nb (head-major, so
-// the head's query rows stay in L2).  block = 320 threads:
+// the head's query rows stay in L2).  block = 384 threads:
 //   warpgroup g (warps 4g .. 4g+3) owns the query tiles it = g, g+2, ... of the
 //   block's list: masked softmax over the block's NKV keys, normalised partial
 //   (o / l, lse) per (query, slot);
@@ -392,7 +392,9 @@ struct SparseFwdSmem {
     static constexpr int kTotal = kBar + 256;
 };
 
-constexpr int kSparseFwdThreads = 320;
+// 384 threads launched with 168 registers each; softmax warpgroups grow to 208,
+// warps 8-11 (MMA, gather, two idle) shrink to 88: 2*128*208 + 128*88 = 64,512.
+constexpr int kSparseFwdThreads = 384;
 
 template <int NKV>
 __global__ void __launch_bounds__(kSparseFwdThreads, 1)
@@ -449,6 +451,7 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
 
+    if (warp >= 8) regs_shrink<88>();
     if (warp == 9) {
         // ---------------- gather warp: query rows of tile it into Q[it & 1] ----------------
         for (int it = 0; it < ntiles; ++it) {
@@ -496,7 +499,8 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
             mma_commit(bar_final);
             mbar_wait(bar_final, 0, abort_flag, 0x205);
         }
-    } else {
+    } else if (warp < 8) {
+        regs_grow<208>();
         const int g = warp >> 2;                  // warpgroup: tiles g, g+2, ...
         const int r = ((warp & 3) << 5) | lane;   // tile row
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
