@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool sparse = a.sparse != 0;
     Rows R;
     if (sparse) {
-        R.list = a.entries + head_rows * a.k + a.lstart[bh * a.nb + kb];
+        R.list = a.entries + static_cast<size_t>(bh) * list_stride(T, a.k, a.nb) + a.lstart[bh * a.nb + kb];
         R.len = a.llen[bh * a.nb + kb];
         R.first = 0;
     } else {

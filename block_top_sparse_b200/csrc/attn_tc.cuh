@@ -370,39 +370,74 @@ __global__ void __launch_bounds__(kFullFwdThreads, 1)
 // ---------------------------------------------------------------------------
 // Sparse forward, block-major, two warpgroups in ping-pong.
 // grid = (B*H*nb): unit u -> head bh = u / nb, block j = u % nb (head-major, so
-// the head's query rows stay in L2).  block = 384 threads:
+// the head's query rows stay in L2).  block = 512 threads:
 //   warpgroup g (warps 4g .. 4g+3) owns the query tiles it = g, g+2, ... of the
-//   block's list: masked softmax over the block's NKV keys, normalised partial
-//   (o / l, lse) per (query, slot);
-//   warp 9 gathers each tile's query rows (cp.async, completion on an mbarrier);
-//   warp 8 loads K_j, V_j (TMA) and issues the MMAs in the order
+//   block's list: masked softmax over the block's NKV keys, P written back over
+//   S in tensor memory as bf16 pairs, then the normalised partial output o / l
+//   and the partial log-sum-exp of every (query, slot) at the entry's position
+//   in the block's list (each warp stages its 32 rows in shared memory and
+//   writes them with two TMA tile stores: a tile's rows are contiguous);
+//   warps 8-11 and 13-15 gather each tile's query rows with cp.async, a
+//   half-warp per 256-byte row (a gather's cost is set by the number of warp
+//   instructions in flight, so seven warps share it; completion on an mbarrier);
+//   warp 12 loads K_j, V_j (TMA) and issues the MMAs in the order
 //   S(it), PV(it-1), S(it+1), PV(it), ... so that one warpgroup's softmax
 //   overlaps the other's MMAs and epilogue.
-// smem: Q[2] 32 KB each | K, V NKV*256 each | P[2] (NKV/64)*16 KB each | barriers
-// tmem: S[2] at 0 / 128, O[2] at 256 / 384 (512 allocated).
+// smem: Q[2] 32 KB each | K, V NKV*256 each | O staging[2] 32 KB each | barriers
+// tmem: S/P[2] at 0 / 128, O[2] at 256 / 384 (512 allocated).
 // ---------------------------------------------------------------------------
 template <int NKV>
 struct SparseFwdSmem {
     static constexpr int kQ = 0;                          // [2]
     static constexpr int kK = kQ + 2 * 2 * kChunkBytes;
     static constexpr int kV = kK + 2 * NKV * 128;
-    static constexpr int kP = kV + 2 * NKV * 128;         // [2]
-    static constexpr int kPStage = (NKV / 64) * kChunkBytes;
-    static constexpr int kBar = kP + 2 * kPStage;
+    static constexpr int kO = kV + 2 * NKV * 128;         // [2] 2 chunks x 128 rows x 128 B, swizzled
+    static constexpr int kOStage = 2 * kChunkBytes;
+    static constexpr int kBar = kO + 2 * kOStage;
     static constexpr int kTotal = kBar + 256;
 };
 
-// 384 threads launched with 168 registers each; softmax warpgroups grow to 208,
-// warps 8-11 (MMA, gather, two idle) shrink to 88: 2*128*208 + 128*88 = 64,512.
-constexpr int kSparseFwdThreads = 384;
+// 512 threads launched with 128 registers each; the softmax warpgroups grow to
+// 192 and the gather / MMA warpgroups shrink to 64: 2*128*192 + 2*128*64 = 65,536.
+constexpr int kSparseFwdThreads = 512;
+constexpr int kSparseFwdGatherWarps = 7;
+
+// Gather warp gw (of kSparseFwdGatherWarps) copies the row pairs p = gw, gw + 7, ...
+// of a 128-row query tile: half-warp h takes row 2p + h, lane l & 15 its 16-byte
+// unit, into the 2-chunk 128-byte-swizzled tile.  Rows past the list are zero-filled.
+constexpr int kGatherPairs = (64 + kSparseFwdGatherWarps - 1) / kSparseFwdGatherWarps;
+
+__device__ __forceinline__ void gather_rows_load(const Rows &R, int it, int gw, int lane, int (&t)[kGatherPairs]) {
+#pragma unroll
+    for (int q = 0; q < kGatherPairs; ++q) {
+        const int p = gw + kSparseFwdGatherWarps * q;
+        const int li = it * kTileQ + 2 * p + (lane >> 4);
+        t[q] = (p < 64 && li < R.len) ? (__ldg(R.list + li) >> 8) : -1;
+    }
+}
+
+__device__ __forceinline__ void gather_rows_issue(uint32_t tile, const __nv_bfloat16 *base, size_t head_rows, int gw,
+                                                  int lane, const int (&t)[kGatherPairs]) {
+    const int u = lane & 15;
+#pragma unroll
+    for (int q = 0; q < kGatherPairs; ++q) {
+        const int p = gw + kSparseFwdGatherWarps * q;
+        if (p < 64) {
+            const int r = 2 * p + (lane >> 4);
+            const uint32_t dst = tile + (u >> 3) * kChunkBytes + r * 128 + ((((u & 7) ^ (r & 7)) & 7) << 4);
+            const bool valid = t[q] >= 0;
+            cp_async_16(dst, base + (head_rows + (valid ? t[q] : 0)) * kD + u * 8, valid ? 16u : 0u);
+        }
+    }
+}
 
 template <int NKV>
 __global__ void __launch_bounds__(kSparseFwdThreads, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                      const __nv_bfloat16 *__restrict__ Q, const int32_t *__restrict__ entries,
-                      const int32_t *__restrict__ lstart, const int32_t *__restrict__ llen,
-                      __nv_bfloat16 *__restrict__ Opart, float *__restrict__ lsepart, int BH, int T, int k,
-                      int nb, float scale_log2) {
+                      const __grid_constant__ CUtensorMap tmO, const __nv_bfloat16 *__restrict__ Q,
+                      const int32_t *__restrict__ entries, const int32_t *__restrict__ lstart,
+                      const int32_t *__restrict__ llen, float *__restrict__ lsepart, int BH, int T, int k, int nb,
+                      float scale_log2) {
     using L = SparseFwdSmem<NKV>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -412,7 +447,6 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
     uint64_t *bar_s_full = bars + 3;   // [2]
     uint64_t *bar_p_full = bars + 5;   // [2]
     uint64_t *bar_o_full = bars + 7;   // [2]
-    uint64_t *bar_o_empty = bars + 9;  // [2]
     uint64_t *bar_final = bars + 11;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 15);
@@ -421,8 +455,10 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
     const int bh = blockIdx.x / nb, j = blockIdx.x % nb;
     const int kv0 = j * NKV;
     const size_t head_rows = static_cast<size_t>(bh) * T;
+    // this block's list (and partial-output rows) start at list position obase
+    const size_t obase = static_cast<size_t>(bh) * list_stride(T, k, nb) + lstart[bh * nb + j];
     Rows R;
-    R.list = entries + head_rows * k + lstart[bh * nb + j];
+    R.list = entries + obase;
     R.len = llen[bh * nb + j];
     R.first = 0;
     R.k = k;
@@ -431,11 +467,10 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
         for (int g = 0; g < 2; ++g) {
-            mbar_init(bar_q_full + g, 32);  // one cp.async arrival per lane of the gather warp
+            mbar_init(bar_q_full + g, 32 * kSparseFwdGatherWarps);  // one cp.async arrival per gather lane
             mbar_init(bar_s_full + g, 1);
             mbar_init(bar_p_full + g, 128);
             mbar_init(bar_o_full + g, 1);
-            mbar_init(bar_o_empty + g, 128);
         }
         mbar_init(bar_final, 1);
         *abort_flag = 0;
@@ -451,18 +486,27 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
 
-    if (warp >= 8) regs_shrink<88>();
-    if (warp == 9) {
-        // ---------------- gather warp: query rows of tile it into Q[it & 1] ----------------
+    if (warp >= 8) regs_shrink<64>();
+    if (warp >= 8 && warp != 12) {
+        // ---------------- gather warps: query rows of tile it into Q[it & 1] ----------------
+        const int gw = warp < 12 ? warp - 8 : warp - 9;
+        int tn[kGatherPairs];
+        gather_rows_load(R, 0, gw, lane, tn);
         for (int it = 0; it < ntiles; ++it) {
             const int g = it & 1;
-            // Q[g] is free once the S MMA of tile it-2 has completed
-            if (it >= 2 && !mbar_wait(bar_s_full + g, ((it - 2) >> 1) & 1, abort_flag, 0x208)) break;
-            warp_gather_tile(smem_u32(smem + L::kQ + g * 2 * kChunkBytes), Q, R, T, it, head_rows, lane);
+            int tc[kGatherPairs];
+#pragma unroll
+            for (int q = 0; q < kGatherPairs; ++q) tc[q] = tn[q];
+            if (it + 1 < ntiles) gather_rows_load(R, it + 1, gw, lane, tn);  // one tile ahead
+            // Q[g] is free once the S MMA of tile it-2 has completed (one lane waits for the warp)
+            bool ok = true;
+            if (lane == 0 && it >= 2) ok = mbar_wait(bar_s_full + g, ((it - 2) >> 1) & 1, abort_flag, 0x208);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            gather_rows_issue(smem_u32(smem + L::kQ + g * 2 * kChunkBytes), Q, head_rows, gw, lane, tc);
             cp_async_mbar_arrive_noinc(bar_q_full + g);
         }
         cp_async_wait_all();
-    } else if (warp == 8) {
+    } else if (warp == 12) {
         if (lane == 0) {
             mbar_arrive_expect_tx(bar_kv, 4 * NKV * 128);
             tma_load_2d(&tmK, bar_kv, smem + L::kK, 0, static_cast<int>(head_rows) + kv0);
@@ -472,12 +516,12 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
             const uint32_t idS = idesc_bf16(128, NKV, false, false);
             const uint32_t idO = idesc_bf16(128, 128, false, true);
             bool ok = mbar_wait(bar_kv, 0, abort_flag, 0x201);
+            // S(it) overwrites the P of tile it-2 in the same tensor-memory columns; the PV MMA
+            // reading it was issued earlier and tensor-core operations run in issue order.
             for (int it = 0; ok && it <= ntiles; ++it) {
                 if (it < ntiles) {
                     const int g = it & 1, i = it >> 1;
                     if (!mbar_wait(bar_q_full + g, i & 1, abort_flag, 0x202)) break;
-                    if (i > 0 && !mbar_wait(bar_o_empty + g, (i - 1) & 1, abort_flag, 0x203)) break;
-                    fence_proxy_async_smem();  // cp.async-written rows -> tensor-core reads
                     tc_fence_after();
                     mma_k128_kmajor(tmem + 128 * g, smem_u32(smem + L::kQ + g * 2 * kChunkBytes), sK, NKV * 128,
                                     idS);
@@ -487,11 +531,10 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
                     const int g = (it - 1) & 1, i = (it - 1) >> 1;
                     if (!mbar_wait(bar_p_full + g, i & 1, abort_flag, 0x204)) break;
                     tc_fence_after();
-                    const uint32_t sP = smem_u32(smem + L::kP + g * L::kPStage);
+                    // O_g = P_g V : A = P from tensor memory (bf16 pairs over S_g), B = V [NKV x d] MN-major
 #pragma unroll
                     for (int kk = 0; kk < NKV / 16; ++kk)
-                        mma_bf16_ss(tmem + 256 + 128 * g,
-                                    smem_desc_sw128(sP + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16),
+                        mma_bf16_ts(tmem + 256 + 128 * g, tmem + 128 * g + kk * 8,
                                     smem_desc_sw128(sV + kk * 2048, NKV * 128), idO, kk > 0 ? 1u : 0u);
                     mma_commit(bar_o_full + g);
                 }
@@ -500,71 +543,99 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
             mbar_wait(bar_final, 0, abort_flag, 0x205);
         }
     } else if (warp < 8) {
-        regs_grow<208>();
+        regs_grow<192>();
         const int g = warp >> 2;                  // warpgroup: tiles g, g+2, ...
         const int r = ((warp & 3) << 5) | lane;   // tile row
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t sP = smem_u32(smem + L::kP + g * L::kPStage);
+        const uint32_t sO = smem_u32(smem + L::kO + g * L::kOStage);  // this warpgroup's staging tile
         const uint32_t tS = tmem + 128 * g + lane_off, tO = tmem + 256 + 128 * g + lane_off;
         for (int it = g; it < ntiles; it += 2) {
             const int i = it >> 1;
-            int t = 0, e = 0;
-            const bool valid = tile_row(R, T, it, r, t, e);  // load overlaps the wait below
+            const bool valid = it * kTileQ + r < R.len;
+            const int lim = valid ? (__ldg(R.list + it * kTileQ + r) >> 8) - kv0 : -1;  // overlaps the wait
             if (!mbar_wait(bar_s_full + g, i & 1, abort_flag, 0x206)) break;
             tc_fence_after();
             uint32_t sr[NKV / 32][32];
 #pragma unroll
             for (int c = 0; c < NKV / 32; ++c) tmem_ld32_async(tS + 32 * c, sr[c]);
             tmem_ld_wait();
-            // key kv0 + col is attended when col <= lim (causal inside the query's own block)
-            const int lim = valid ? t - kv0 : -1;
+            // key kv0 + col is attended when col <= lim (causal inside the query's own block);
+            // masked scores become -inf, and only warps holding such a row pay for the mask
+            if (!__all_sync(0xffffffffu, lim >= NKV - 1)) {
+#pragma unroll
+                for (int c = 0; c < NKV / 32; ++c)
+#pragma unroll
+                    for (int i2 = 0; i2 < 32; ++i2)
+                        if (32 * c + i2 > lim) sr[c][i2] = 0xff800000u;
+            }
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int c = 0; c < NKV / 32; ++c)
 #pragma unroll
-                for (int i2 = 0; i2 < 32; ++i2)
-                    mx4[i2 & 3] = fmaxf(mx4[i2 & 3], (32 * c + i2 <= lim) ? __uint_as_float(sr[c][i2]) : -INFINITY);
+                for (int i2 = 0; i2 < 32; ++i2) mx4[i2 & 3] = fmaxf(mx4[i2 & 3], __uint_as_float(sr[c][i2]));
             const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
             const float mref = (mx == -INFINITY) ? 0.f : mx;
-            float l4[4] = {0.f, 0.f, 0.f, 0.f};
+            // p = 2^(s * scale_log2 - mref) in packed pairs; P (bf16 pairs) goes to tensor memory over
+            // the first NKV/2 columns of S
+            const uint64_t sl2 = f2_pack(scale_log2, scale_log2), nm = f2_pack(-mref, -mref);
+            uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
             for (int c = 0; c < NKV / 32; ++c) {
-                float v[32];
+                uint32_t pw[16];
 #pragma unroll
-                for (int i2 = 0; i2 < 32; ++i2) {
-                    const float p =
-                        (32 * c + i2 <= lim) ? fast_exp2(fmaf(__uint_as_float(sr[c][i2]), scale_log2, -mref)) : 0.f;
-                    l4[i2 & 3] += p;
-                    v[i2] = p;
+                for (int i2 = 0; i2 < 32; i2 += 2) {
+                    float x0, x1;
+                    f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c][i2]), __uint_as_float(sr[c][i2 + 1])), sl2, nm), x0,
+                              x1);
+                    const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                    l2[(i2 >> 1) & 1] = fadd2(l2[(i2 >> 1) & 1], f2_pack(p0, p1));
+                    pw[i2 >> 1] = pack_bf16x2(p0, p1);
                 }
-                store_row32_bf16(sP, kChunkBytes, r, 32 * c, v);
+                tmem_st16_u(tS + 16 * c, pw);
             }
-            const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            fence_proxy_async_smem();
+            tmem_st_wait();
             tc_fence_before();
             mbar_arrive(bar_p_full + g);
+            float la, lb, lc, ld;
+            f2_unpack(l2[0], la, lb);
+            f2_unpack(l2[1], lc, ld);
+            const float l = (la + lb) + (lc + ld);
+            const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+            const size_t orow = obase + static_cast<size_t>(it) * kTileQ + r;  // list position of this row
+            if (valid) lsepart[orow] = (l > 0.f) ? (mref + __log2f(l)) * kLn2 : -INFINITY;
+            // the TMA stores of tile it-2 must have read this warp's staging rows
+            if (lane == 0) bulk_wait_read();
+            __syncwarp();
             if (!mbar_wait(bar_o_full + g, i & 1, abort_flag, 0x207)) break;
             tc_fence_after();
-            uint32_t orow[4][32];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32_async(tO + 32 * c, orow[c]);
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive(bar_o_empty + g);
-            if (valid) {
-                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-                uint4 *d4 = reinterpret_cast<uint4 *>(Opart + (head_rows * k + entry_row(e, k)) * kD);
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t ov[2][32];
+                tmem_ld32_async(tO + 64 * hh, ov[0]);
+                tmem_ld32_async(tO + 64 * hh + 32, ov[1]);
+                tmem_ld_wait();
+                // row r of column chunk hh, 128-byte swizzle (conflict-free 16-byte stores)
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const uint32_t *x = orow[q >> 2] + 8 * (q & 3);
-                    d4[q] = make_uint4(pack_bf16x2(__uint_as_float(x[0]) * inv_l, __uint_as_float(x[1]) * inv_l),
-                                       pack_bf16x2(__uint_as_float(x[2]) * inv_l, __uint_as_float(x[3]) * inv_l),
-                                       pack_bf16x2(__uint_as_float(x[4]) * inv_l, __uint_as_float(x[5]) * inv_l),
-                                       pack_bf16x2(__uint_as_float(x[6]) * inv_l, __uint_as_float(x[7]) * inv_l));
+                for (int u = 0; u < 8; ++u) {
+                    const uint32_t *xo = ov[u >> 2] + 8 * (u & 3);
+                    st_shared_v4(sO + hh * kChunkBytes + r * 128 + (((u ^ (r & 7)) & 7) << 4),
+                                 pack_bf16x2(__uint_as_float(xo[0]) * inv_l, __uint_as_float(xo[1]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(xo[2]) * inv_l, __uint_as_float(xo[3]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(xo[4]) * inv_l, __uint_as_float(xo[5]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(xo[6]) * inv_l, __uint_as_float(xo[7]) * inv_l));
                 }
-                lsepart[head_rows * k + entry_row(e, k)] = (l > 0.f) ? (mref + __log2f(l)) * kLn2 : -INFINITY;
+            }
+            fence_proxy_async_smem();  // generic-proxy staging writes -> TMA reads
+            __syncwarp();
+            if (lane == 0) {
+                // rows 32w .. 32w+31 of the tile: the padded list region keeps them inside this block's rows
+                const int row0 = static_cast<int>(obase + static_cast<size_t>(it) * kTileQ + (r - lane));
+                tma_store_2d(&tmO, sO + (r - lane) * 128, 0, row0);
+                tma_store_2d(&tmO, sO + kChunkBytes + (r - lane) * 128, 64, row0);
+                bulk_commit();
             }
         }
+        if (lane == 0) bulk_wait();
     }
     tc_fence_before();
     __syncthreads();

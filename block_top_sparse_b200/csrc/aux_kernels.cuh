@@ -52,9 +52,11 @@ __global__ void __launch_bounds__(1024) index_scan_kernel(int *__restrict__ cnt,
                 total += v;
             }
         }
-        // exclusive scan of totals over j (block-wide)
+        // exclusive scan over j of the totals rounded up to whole 128-entry tiles
+        // (every block's list region starts on a tile boundary)
+        const int padded = (total + kListPad - 1) / kListPad * kListPad;
         const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-        int incl = total;
+        int incl = padded;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -72,14 +74,14 @@ __global__ void __launch_bounds__(1024) index_scan_kernel(int *__restrict__ cnt,
             warp_tot[lane] = x;  // inclusive over warps
         }
         __syncthreads();
-        const int start = carry + (w > 0 ? warp_tot[w - 1] : 0) + incl - total;
+        const int start = carry + (w > 0 ? warp_tot[w - 1] : 0) + incl - padded;
         if (j < nb) {
             lstart[bh * nb + j] = start;
             llen[bh * nb + j] = total;
             for (int c = 0; c < nch; ++c) base[static_cast<size_t>(c) * nb + j] += start;
         }
         __syncthreads();
-        if (threadIdx.x == blockDim.x - 1) carry = start + total;
+        if (threadIdx.x == blockDim.x - 1) carry = start + padded;
         __syncthreads();
     }
 }
@@ -89,7 +91,7 @@ __global__ void __launch_bounds__(1024) index_scan_kernel(int *__restrict__ cnt,
 // lane bitmasks).  k <= 256 and T < 2^23 keep the encoding in an int32.
 __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t *__restrict__ idx,
                                                          const int *__restrict__ off, int32_t *__restrict__ entries,
-                                                         int T, int k, int nb, int nch) {
+                                                         int32_t *__restrict__ pos, int T, int k, int nb, int nch) {
     extern __shared__ int sm_fill[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.y, c = blockIdx.x * 4 + warp;
@@ -103,7 +105,7 @@ __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t *__restri
     }
     __syncwarp();
     if (c >= nch) return;
-    int32_t *dst = entries + static_cast<size_t>(bh) * T * k;
+    int32_t *dst = entries + static_cast<size_t>(bh) * list_stride(T, k, nb);
     const uint32_t lt_mask = (1u << lane) - 1u;
     const int t_end = min(T, (c + 1) * kIdxChunk);
     for (int tb = c * kIdxChunk; tb < t_end; tb += 32) {
@@ -117,7 +119,9 @@ __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t *__restri
         __syncwarp();
         for (int i = 0; i < k; ++i) {
             const int j = valid ? __ldg(row + i) : -1;
-            if (j >= 0 && j < nb) dst[run[j] + __popc(bits[j] & lt_mask)] = (t << 8) | i;
+            const int at = (j >= 0 && j < nb) ? run[j] + __popc(bits[j] & lt_mask) : -1;
+            if (at >= 0) dst[at] = (t << 8) | i;
+            if (pos && valid) pos[(static_cast<size_t>(bh) * T + t) * k + i] = at;
         }
         __syncwarp();
         for (int i = 0; i < k; ++i) {
@@ -136,29 +140,55 @@ __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t *__restri
 
 // Merge of the per-slot partials: one warp per query row, 4 columns per lane.
 //   lse = log sum_i exp(lse_i),  o = sum_i exp(lse_i - lse) o_i
+// The partial of (query, slot i) sits at list position pos[query * k + i] of its
+// head's region (-1: slot not attended).  Lane i holds slot i's position and
+// weight (32 slots at a time), so the slots' row loads are all in flight at once.
 template <typename TO>
-__global__ void __launch_bounds__(256) sparse_merge_kernel(const int32_t *__restrict__ idx,
+__global__ void __launch_bounds__(256) sparse_merge_kernel(const int32_t *__restrict__ pos,
                                                            const __nv_bfloat16 *__restrict__ Opart,
                                                            const float *__restrict__ lsepart, TO *__restrict__ O,
-                                                           float *__restrict__ lse, size_t rows, int k) {
+                                                           float *__restrict__ lse, size_t rows, int T, int k,
+                                                           int nb) {
     const size_t row = static_cast<size_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
-    const int32_t *sel = idx + row * k;
+    const size_t region = (row / T) * list_stride(T, k, nb);
+    const int32_t *ps = pos + row * k;
     float mx = -INFINITY;
-    for (int i = 0; i < k; ++i)
-        if (__ldg(sel + i) >= 0) mx = fmaxf(mx, __ldg(lsepart + row * k + i));
-    float wsum = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int i = 0; i < k; ++i) {
-        if (__ldg(sel + i) < 0) continue;
-        const float w = __expf(__ldg(lsepart + row * k + i) - mx);
-        wsum += w;
-        const uint2 u = __ldg(reinterpret_cast<const uint2 *>(Opart + (row * k + i) * 128) + lane);
-        acc[0] += w * __uint_as_float(u.x << 16);
-        acc[1] += w * __uint_as_float(u.x & 0xFFFF0000u);
-        acc[2] += w * __uint_as_float(u.y << 16);
-        acc[3] += w * __uint_as_float(u.y & 0xFFFF0000u);
+    for (int i0 = 0; i0 < k; i0 += 32) {
+        const int p = (i0 + lane < k) ? __ldg(ps + i0 + lane) : -1;
+        if (p >= 0) mx = fmaxf(mx, __ldg(lsepart + region + p));
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float wsum = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i0 = 0; i0 < k; i0 += 32) {
+        const int p = (i0 + lane < k) ? __ldg(ps + i0 + lane) : -1;
+        const float w = (p >= 0) ? __expf(__ldg(lsepart + region + p) - mx) : 0.f;
+        wsum += w;
+        const int n = min(32, k - i0);
+        for (int s0 = 0; s0 < n; s0 += 8) {
+            uint2 u[8];
+            float wu[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int pq = __shfl_sync(0xffffffffu, p, (s0 + q) & 31);
+                wu[q] = __shfl_sync(0xffffffffu, w, (s0 + q) & 31);
+                u[q] = (s0 + q < n && pq >= 0)
+                           ? __ldg(reinterpret_cast<const uint2 *>(Opart + (region + pq) * 128) + lane)
+                           : make_uint2(0u, 0u);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                acc[0] += wu[q] * __uint_as_float(u[q].x << 16);
+                acc[1] += wu[q] * __uint_as_float(u[q].x & 0xFFFF0000u);
+                acc[2] += wu[q] * __uint_as_float(u[q].y << 16);
+                acc[3] += wu[q] * __uint_as_float(u[q].y & 0xFFFF0000u);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
     const float inv = 1.f / wsum;
     TO *dst = O + row * 128 + lane * 4;
     if constexpr (sizeof(TO) == 2) {

@@ -86,6 +86,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// Bounded wait used on exit paths to let this CTA's own copies in flight land
+// before its shared memory is released; ignores the abort flag, records nothing.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 <= kWaitLimitNs) {
+    }
+}
+
 // ----------------------------------------------------------------------------
 // Async-proxy fences and cp.async (16-byte, L2-only) row gathers.
 // ----------------------------------------------------------------------------
@@ -134,6 +142,42 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *ba
             smem_u32(dst)),
         "l"(map), "r"(col), "r"(row), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Per-head region of the inverse selection index (and of the block-major
+// partial outputs): T*k entries plus up to one tile of padding per key block,
+// so that every block's list starts on a 128-entry boundary.
+constexpr int kListPad = 128;
+__host__ __device__ __forceinline__ size_t list_stride(int T, int k, int nb) {
+    return static_cast<size_t>(T) * k + static_cast<size_t>(nb) * kListPad;
+}
+
+// TMA row gather: rows r0..r3 of a 2D tensor map whose box is one row high
+// (box = {64 columns, 1}), columns [col, col + 64), into 4 consecutive 128-byte
+// rows at dst (dst 512-byte aligned inside a 1024-byte aligned swizzle atom, so
+// the 128-byte swizzle lands exactly as for a 128-row box load).
+__device__ __forceinline__ void tma_gather4(const CUtensorMap *map, uint64_t *bar, uint32_t dst, int col, int r0,
+                                            int r1, int r2, int r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+        "l"(map), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Tiled TMA store of a box from shared memory (same swizzle as the tensor map),
+// tracked by this thread's bulk async-group.  Coordinates must be >= 0.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src_smem, int col, int row) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(col),
+                 "r"(row), "r"(src_smem)
+                 : "memory");
+}
+
+// Bulk copy shared -> global (both 16-byte aligned, bytes a multiple of 16),
+// tracked by this thread's bulk async-group.
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src_smem, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src_smem), "r"(bytes)
+                 : "memory");
 }
 
 // ----------------------------------------------------------------------------
@@ -318,6 +362,26 @@ __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): two lanes of work per instruction.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
 }
 
 // Pack two floats into a bf16x2 word, `lo` in the low half (round to nearest even).

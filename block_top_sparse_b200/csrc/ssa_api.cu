@@ -60,6 +60,8 @@ ssa_status_t check_dims(const ssa_dims_t *dims, Shape &S, bool need_k) {
     S.tc = S.dtype == SSA_DT_BF16 && S.d == 128;
     // the sparse index packs (t << 8) | slot into an int32
     if (need_k && S.tc && (S.k > 256 || S.T >= (1 << 23))) return SSA_ERR_UNSUPPORTED;
+    // list positions of the whole index (and TMA row coordinates of the partials) fit an int32
+    if (need_k && S.tc && S.BH * list_stride(S.T, S.k, S.nb) >= (size_t(1) << 31)) return SSA_ERR_UNSUPPORTED;
     return SSA_OK;
 }
 
@@ -68,13 +70,14 @@ inline size_t align_up(size_t x) { return (x + 255) & ~static_cast<size_t>(255);
 // Workspace layout of the sparse index.
 struct IndexWs {
     int *cnt, *lstart, *llen;
-    int32_t *entries;
+    int32_t *entries;  // per head: list_stride(T, k, nb) entries, block lists on 128-entry boundaries
     int nch;
 };
 
 size_t index_bytes(const Shape &S) {
     const size_t nch = (S.T + kIdxChunk - 1) / kIdxChunk;
-    return align_up(S.BH * nch * S.nb * 4) + 2 * align_up(S.BH * S.nb * 4) + align_up(S.rows * S.k * 4);
+    return align_up(S.BH * nch * S.nb * 4) + 2 * align_up(S.BH * S.nb * 4) +
+           align_up(S.BH * list_stride(S.T, S.k, S.nb) * 4);
 }
 
 uint8_t *carve_index(const Shape &S, uint8_t *p, IndexWs &W) {
@@ -86,7 +89,7 @@ uint8_t *carve_index(const Shape &S, uint8_t *p, IndexWs &W) {
     W.llen = reinterpret_cast<int *>(p);
     p += align_up(S.BH * S.nb * 4);
     W.entries = reinterpret_cast<int32_t *>(p);
-    p += align_up(S.rows * S.k * 4);
+    p += align_up(S.BH * list_stride(S.T, S.k, S.nb) * 4);
     return p;
 }
 
@@ -94,7 +97,9 @@ size_t ws_bytes_for(const Shape &S, int op) {
     switch (op) {
         case SSA_OP_SPARSE_FWD:
             if (!S.tc) return 0;
-            return index_bytes(S) + align_up(S.rows * S.k * 128 * 2) + align_up(S.rows * S.k * 4);
+            // index | partial outputs and lse by list position | list position of every (query, slot)
+            return index_bytes(S) + align_up(S.BH * list_stride(S.T, S.k, S.nb) * (128 * 2 + 4)) +
+                   align_up(S.rows * S.k * 4);
         case SSA_OP_SPARSE_BWD:
         case SSA_OP_FULL_BWD: {
             size_t b = align_up(S.rows * 4) + align_up(S.rows * S.d * 4);  // D, dQacc
@@ -174,15 +179,15 @@ ssa_status_t launch_select(const Shape &S, const void *Q, const float *Kbar, int
 }
 
 // Inverse selection index: entries of block j of head bh (query order).
-ssa_status_t build_index(const Shape &S, const int32_t *idx, IndexWs &W, cudaStream_t st) {
+ssa_status_t build_index(const Shape &S, const int32_t *idx, IndexWs &W, cudaStream_t st, int32_t *pos = nullptr) {
     const size_t hbytes = static_cast<size_t>(S.nb) * 4;
     if (!set_smem(index_count_kernel, hbytes)) return SSA_ERR_CUDA;
     index_count_kernel<<<dim3(W.nch, S.BH), 256, hbytes, st>>>(idx, W.cnt, S.T, S.k, S.nb, W.nch);
     index_scan_kernel<<<S.BH, 1024, 0, st>>>(W.cnt, W.lstart, W.llen, S.nb, W.nch);
     const size_t fbytes = static_cast<size_t>(S.nb) * 8 * 4;
     if (!set_smem(index_fill_kernel, fbytes)) return SSA_ERR_CUDA;
-    index_fill_kernel<<<dim3((W.nch + 3) / 4, S.BH), 128, fbytes, st>>>(idx, W.cnt, W.entries, S.T, S.k, S.nb,
-                                                                          W.nch);
+    index_fill_kernel<<<dim3((W.nch + 3) / 4, S.BH), 128, fbytes, st>>>(idx, W.cnt, W.entries, pos, S.T, S.k,
+                                                                          S.nb, W.nch);
     return launch_status();
 }
 
@@ -359,29 +364,32 @@ ssa_status_t ssa_sparse_attn_fwd(const ssa_dims_t *dims, const void *Q, const vo
     }
     IndexWs W{};
     uint8_t *p = carve_index(S, static_cast<uint8_t *>(ws), W);
+    const size_t nlist = S.BH * list_stride(S.T, S.k, S.nb);
     __nv_bfloat16 *Opart = reinterpret_cast<__nv_bfloat16 *>(p);
-    p += align_up(S.rows * S.k * 128 * 2);
-    float *lsepart = reinterpret_cast<float *>(p);
-    if ((e = build_index(S, idx, W, st)) != SSA_OK) return e;
-    CUtensorMap tmK, tmV;
-    if (!make_tmap(&tmK, K, S.rows, S.s) || !make_tmap(&tmV, V, S.rows, S.s)) return SSA_ERR_CUDA;
+    float *lsepart = reinterpret_cast<float *>(p + nlist * 128 * 2);
+    p += align_up(nlist * (128 * 2 + 4));
+    int32_t *pos = reinterpret_cast<int32_t *>(p);
+    if ((e = build_index(S, idx, W, st, pos)) != SSA_OK) return e;
+    CUtensorMap tmK, tmV, tmO;
+    if (!make_tmap(&tmK, K, S.rows, S.s) || !make_tmap(&tmV, V, S.rows, S.s) || !make_tmap(&tmO, Opart, nlist, 32))
+        return SSA_ERR_CUDA;
     const unsigned units = static_cast<unsigned>(S.BH * S.nb);
     const float sl2 = S.scale * kLog2e;
     if (S.s == 128) {
         const size_t sm = SparseFwdSmem<128>::kTotal + 1024;
         if (!set_smem(sparse_fwd_kernel<128>, sm)) return SSA_ERR_CUDA;
-        sparse_fwd_kernel<128><<<units, kSparseFwdThreads, sm, st>>>(tmK, tmV, (const __nv_bfloat16 *)Q, W.entries, W.lstart,
-                                                       W.llen, Opart, lsepart, static_cast<int>(S.BH), S.T, S.k,
-                                                       S.nb, sl2);
+        sparse_fwd_kernel<128><<<units, kSparseFwdThreads, sm, st>>>(tmK, tmV, tmO, (const __nv_bfloat16 *)Q,
+                                                                      W.entries, W.lstart, W.llen, lsepart,
+                                                                      static_cast<int>(S.BH), S.T, S.k, S.nb, sl2);
     } else {
         const size_t sm = SparseFwdSmem<64>::kTotal + 1024;
         if (!set_smem(sparse_fwd_kernel<64>, sm)) return SSA_ERR_CUDA;
-        sparse_fwd_kernel<64><<<units, kSparseFwdThreads, sm, st>>>(tmK, tmV, (const __nv_bfloat16 *)Q, W.entries, W.lstart,
-                                                      W.llen, Opart, lsepart, static_cast<int>(S.BH), S.T, S.k,
-                                                      S.nb, sl2);
+        sparse_fwd_kernel<64><<<units, kSparseFwdThreads, sm, st>>>(tmK, tmV, tmO, (const __nv_bfloat16 *)Q,
+                                                                     W.entries, W.lstart, W.llen, lsepart,
+                                                                     static_cast<int>(S.BH), S.T, S.k, S.nb, sl2);
     }
     sparse_merge_kernel<__nv_bfloat16><<<static_cast<unsigned>((S.rows + 7) / 8), 256, 0, st>>>(
-        idx, Opart, lsepart, (__nv_bfloat16 *)O, lse, S.rows, S.k);
+        pos, Opart, lsepart, (__nv_bfloat16 *)O, lse, S.rows, S.T, S.k, S.nb);
     return launch_status();
 }
 

@@ -24,7 +24,8 @@
  *    about two seconds) records SSA_ERR_TIMEOUT, read by ssa_get_device_error().
  *  - Supported: bf16 with d == 128 on the tensor-core path; fp32 (any op) and
  *    bf16 with d == 64 on a CUDA-core path; s in {64, 128}; T % s == 0;
- *    1 <= k <= nb; nb <= 1024 for ssa_block_select.
+ *    1 <= k <= nb; nb <= 1024 for ssa_block_select; on the tensor-core sparse
+ *    path also k <= 256, T < 2^23 and B*H*(T*k + 128*nb) < 2^31.
  *  - Workspace: calls that take `ws` need at least ssa_workspace_size(dims, op)
  *    bytes of device memory (16-byte aligned); its contents on entry are
  *    ignored and on exit undefined.  The library allocates nothing.
