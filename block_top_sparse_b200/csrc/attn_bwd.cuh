@@ -13,16 +13,22 @@
 // Paper: section 4.2 (keys outside S(t) get no gradient; the selection is a
 // constant), FlashAttention-2 style recomputation of P from the saved lse.
 //
-// Warp roles (320 threads):
-//   warps 0-7  two warpgroups; warp w owns query row (w & 3)*32 + lane and
-//              column half (w >> 2) of every row-wise phase;
-//   warp 8     MMA issuer (one thread);
-//   warp 9     TMA producer (K_j, V_j; contiguous Q / dO tiles of the full stream).
-// Overlap: Q/dO of the next tile are loaded as soon as the dV/dK MMAs of the
-// current tile have consumed them; dQ leaves tensor memory before its atomics,
-// so the next tile's S/dP MMAs run while the atomics drain.
+// Warp roles (640 threads, five warpgroups; registers rebalanced with setmaxnreg):
+//   warps 0-7    two warpgroups; warp w owns query row (w & 3)*32 + lane and
+//                column half (w >> 2) of the row-wise phase (P, dS), then the
+//                dV, dK epilogue;
+//   warps 8-11   dQ flush: thread <-> query row; dQ leaves tensor memory in two
+//                64-column halves through a 32 KB staging buffer of its own and
+//                is added with coalesced float4 reductions (two 256-byte row
+//                halves per warp instruction), so the next tile never waits for it;
+//   warp 12      MMA issuer (one thread);
+//   warp 13      TMA producer (K_j, V_j; contiguous Q / dO tiles of the full stream);
+//   warps 14-19  sparse stream: gather the next tile's Q and dO rows with
+//                cp.async (a half-warp per 256-byte row) once the dV / dK MMAs
+//                of the current tile have consumed the buffers.
 //
-// Shared memory: Q 32 KB | dO 32 KB | K, V NKV*256 B each | P, dS (NKV/64)*16 KB each
+// Shared memory: Q 32 KB | dO 32 KB | K, V NKV*256 B each | P, dS (NKV/64)*16 KB each |
+//                dQ staging 32 KB
 // Tensor memory: S / dQ at column 0, dP at 128, dV^T at 256, dK^T at 384 (512).
 #pragma once
 
@@ -38,7 +44,8 @@ struct BwdSmem {
     static constexpr int kV = kK + 2 * NKV * 128;
     static constexpr int kP = kV + 2 * NKV * 128;
     static constexpr int kdS = kP + (NKV / 64) * kChunkBytes;
-    static constexpr int kBar = kdS + (NKV / 64) * kChunkBytes;
+    static constexpr int kF = kdS + (NKV / 64) * kChunkBytes;  // dQ staging: 128 rows x 256 B
+    static constexpr int kBar = kF + 2 * kChunkBytes;
     static constexpr int kTotal = kBar + 256;
 };
 
@@ -52,7 +59,11 @@ struct BwdArgs {
     float scale, scale_log2;
 };
 
-constexpr int kBwdThreads = 320;
+// 640 threads launched with 96 registers each (61,440); setmaxnreg moves them to
+// softmax 2 x 152, flush 80, MMA / producer / gather 2 x 48: 128 * 480 = 61,440.
+constexpr int kBwdThreads = 640;
+constexpr int kBwdGatherWarps = 6;
+constexpr int kBwdGatherPairs = (64 + kBwdGatherWarps - 1) / kBwdGatherWarps;
 
 template <int NKV>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -61,22 +72,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const BwdArgs a) {
     using L = BwdSmem<NKV>;
     constexpr int HALF = NKV / 2;  // S / dP columns per warpgroup
-    // 128-key units stage the dQ tile (64 KB) through the P / dS buffers and add it
-    // with coalesced row reductions; 64-key units (buffers of 32 KB) add per row.
-    constexpr bool kCoalescedFlush = NKV == 128;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
     uint64_t *bar_kv = bars + 0, *bar_qdo_full = bars + 1, *bar_sdp_full = bars + 2, *bar_pds_full = bars + 3;
     uint64_t *bar_qdo_free = bars + 4, *bar_dq_full = bars + 5, *bar_dq_empty = bars + 6, *bar_final = bars + 7;
-    uint64_t *bar_staged = bars + 8, *bar_flushed = bars + 9;  // dQ staging in the P / dS buffers
+    uint64_t *bar_f_staged = bars + 8, *bar_f_free = bars + 9;  // dQ staging buffer handshakes
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 11);
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T;
-    // Head-major unit order, heaviest key block of each head first: the query
-    // rows and the dQ accumulator of the head being worked on stay in L2.
+    // Head-major unit order: the query rows and the dQ accumulator of the head
+    // being worked on stay in L2.
     const int units_per_head = a.sparse ? a.nb : (a.T + NKV - 1) / NKV;
     const int bh = blockIdx.x / units_per_head, kb = blockIdx.x % units_per_head;
     const int kv0 = kb * NKV;
@@ -96,19 +103,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int ntiles = (R.len + kTileQ - 1) / kTileQ;
 
     const uint32_t sQ = smem_u32(smem + L::kQ), sdO = smem_u32(smem + L::kdO), sK = smem_u32(smem + L::kK),
-                   sV = smem_u32(smem + L::kV), sP = smem_u32(smem + L::kP), sdS = smem_u32(smem + L::kdS);
+                   sV = smem_u32(smem + L::kV), sP = smem_u32(smem + L::kP), sdS = smem_u32(smem + L::kdS),
+                   sF = smem_u32(smem + L::kF);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
-        mbar_init(bar_qdo_full, sparse ? 256 : 1);
+        mbar_init(bar_qdo_full, sparse ? 32 * kBwdGatherWarps : 1);
         mbar_init(bar_sdp_full, 1);
         mbar_init(bar_pds_full, 256);
         mbar_init(bar_qdo_free, 1);
         mbar_init(bar_dq_full, 1);
-        mbar_init(bar_dq_empty, 256);
+        mbar_init(bar_dq_empty, 128);
         mbar_init(bar_final, 1);
-        mbar_init(bar_staged, 256);
-        mbar_init(bar_flushed, 256);
+        mbar_init(bar_f_staged, 128);
+        mbar_init(bar_f_free, 128);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -122,84 +130,185 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384, tdQ = tmem;
 
-    if (warp == 9) {
-        // ---------------- TMA producer ----------------
-        if (lane == 0) {
-            const int krow = static_cast<int>(head_rows) + kv0;
-            mbar_arrive_expect_tx(bar_kv, 4 * NKV * 128);
-            tma_load_2d(&tmK, bar_kv, smem + L::kK, 0, krow);
-            tma_load_2d(&tmK, bar_kv, smem + L::kK + NKV * 128, 64, krow);
-            tma_load_2d(&tmV, bar_kv, smem + L::kV, 0, krow);
-            tma_load_2d(&tmV, bar_kv, smem + L::kV + NKV * 128, 64, krow);
-            if (!sparse) {
+    if (warp >= 12) {
+        regs_shrink<48>();
+        if (warp >= 14) {
+            // ---------------- gather warps (sparse stream): Q and dO rows of each tile ----------------
+            if (sparse) {
+                const int gw = warp - 14, u = lane & 15;
+                int tn[kBwdGatherPairs];
+                auto load_rows = [&](int it) {
+#pragma unroll
+                    for (int q = 0; q < kBwdGatherPairs; ++q) {
+                        const int p = gw + kBwdGatherWarps * q;
+                        const int li = it * kTileQ + 2 * p + (lane >> 4);
+                        tn[q] = (p < 64 && li < R.len) ? (__ldg(R.list + li) >> 8) : -1;
+                    }
+                };
+                load_rows(0);
                 for (int it = 0; it < ntiles; ++it) {
-                    if (it > 0 && !mbar_wait(bar_qdo_free, (it - 1) & 1, abort_flag, 0x311)) break;
-                    const int qrow = static_cast<int>(head_rows) + kv0 + it * kTileQ;
-                    mbar_arrive_expect_tx(bar_qdo_full, 4 * kChunkBytes);
-                    tma_load_2d(&tmQ, bar_qdo_full, smem + L::kQ, 0, qrow);
-                    tma_load_2d(&tmQ, bar_qdo_full, smem + L::kQ + kChunkBytes, 64, qrow);
-                    tma_load_2d(&tmdO, bar_qdo_full, smem + L::kdO, 0, qrow);
-                    tma_load_2d(&tmdO, bar_qdo_full, smem + L::kdO + kChunkBytes, 64, qrow);
+                    // Q / dO are free once the dV / dK MMAs of the previous tile have completed
+                    bool ok = true;
+                    if (lane == 0 && it > 0) ok = mbar_wait(bar_qdo_free, (it - 1) & 1, abort_flag, 0x312);
+                    if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+#pragma unroll
+                    for (int q = 0; q < kBwdGatherPairs; ++q) {
+                        const int p = gw + kBwdGatherWarps * q;
+                        if (p < 64) {
+                            const int r = 2 * p + (lane >> 4);
+                            const uint32_t off = (u >> 3) * kChunkBytes + r * 128 + ((((u & 7) ^ (r & 7)) & 7) << 4);
+                            const bool valid = tn[q] >= 0;
+                            const size_t src = (head_rows + (valid ? tn[q] : 0)) * kD + u * 8;
+                            cp_async_16(sQ + off, a.Q + src, valid ? 16u : 0u);
+                            cp_async_16(sdO + off, a.dO + src, valid ? 16u : 0u);
+                        }
+                    }
+                    cp_async_mbar_arrive_noinc(bar_qdo_full);
+                    if (it + 1 < ntiles) load_rows(it + 1);  // in flight during the next wait
                 }
+                cp_async_wait_all();
+            }
+        } else if (warp == 13) {
+            // ---------------- TMA producer ----------------
+            if (lane == 0) {
+                const int krow = static_cast<int>(head_rows) + kv0;
+                mbar_arrive_expect_tx(bar_kv, 4 * NKV * 128);
+                tma_load_2d(&tmK, bar_kv, smem + L::kK, 0, krow);
+                tma_load_2d(&tmK, bar_kv, smem + L::kK + NKV * 128, 64, krow);
+                tma_load_2d(&tmV, bar_kv, smem + L::kV, 0, krow);
+                tma_load_2d(&tmV, bar_kv, smem + L::kV + NKV * 128, 64, krow);
+                if (!sparse) {
+                    for (int it = 0; it < ntiles; ++it) {
+                        if (it > 0 && !mbar_wait(bar_qdo_free, (it - 1) & 1, abort_flag, 0x311)) break;
+                        const int qrow = static_cast<int>(head_rows) + kv0 + it * kTileQ;
+                        mbar_arrive_expect_tx(bar_qdo_full, 4 * kChunkBytes);
+                        tma_load_2d(&tmQ, bar_qdo_full, smem + L::kQ, 0, qrow);
+                        tma_load_2d(&tmQ, bar_qdo_full, smem + L::kQ + kChunkBytes, 64, qrow);
+                        tma_load_2d(&tmdO, bar_qdo_full, smem + L::kdO, 0, qrow);
+                        tma_load_2d(&tmdO, bar_qdo_full, smem + L::kdO + kChunkBytes, 64, qrow);
+                    }
+                    // on an abort, let loads still in flight land before the CTA exits
+                    if (ntiles > 0) mbar_drain(bar_qdo_full, (ntiles - 1) & 1);
+                }
+            }
+        } else if (warp == 12) {
+            // ---------------- MMA issuer ----------------
+            if (lane == 0) {
+                const uint32_t idS = idesc_bf16(128, NKV, false, false);  // S, dP
+                const uint32_t idT = idesc_bf16(128, NKV, true, true);    // dV^T, dK^T
+                const uint32_t idQ = idesc_bf16(128, 128, false, true);   // dQ
+                bool ok = mbar_wait(bar_kv, 0, abort_flag, 0x301);
+                for (int it = 0; ok && it < ntiles; ++it) {
+                    if (!mbar_wait(bar_qdo_full, it & 1, abort_flag, 0x302)) break;
+                    if (it > 0 && !mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x303)) break;
+                    if (sparse) fence_proxy_async_smem();  // cp.async-written rows -> tensor-core reads
+                    tc_fence_after();
+                    mma_k128_kmajor(tS, sQ, sK, NKV * 128, idS);
+                    mma_k128_kmajor(tdP, sdO, sV, NKV * 128, idS);
+                    mma_commit(bar_sdp_full);
+                    if (!mbar_wait(bar_pds_full, it & 1, abort_flag, 0x304)) break;
+                    tc_fence_after();
+                    // dV^T[d x kv] += dO^T P ; dK^T[d x kv] += Q^T dS   (K = 128 query rows)
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        mma_bf16_ss(tdV, smem_desc_sw128(sdO + kk * 2048, kChunkBytes),
+                                    smem_desc_sw128(sP + kk * 2048, kChunkBytes), idT, (it > 0 || kk > 0) ? 1u : 0u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        mma_bf16_ss(tdK, smem_desc_sw128(sQ + kk * 2048, kChunkBytes),
+                                    smem_desc_sw128(sdS + kk * 2048, kChunkBytes), idT, (it > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(bar_qdo_free);
+                    // dQ[q x d] = dS K   (K = NKV keys)
+#pragma unroll
+                    for (int kk = 0; kk < NKV / 16; ++kk) {
+                        mma_bf16_ss(tdQ, smem_desc_sw128(sdS + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16),
+                                    smem_desc_sw128(sK + kk * 2048, NKV * 128), idQ, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar_dq_full);
+                }
+                mma_commit(bar_final);
+                mbar_wait(bar_final, 0, abort_flag, 0x305);
             }
         }
-    } else if (warp == 8) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            const uint32_t idS = idesc_bf16(128, NKV, false, false);  // S, dP
-            const uint32_t idT = idesc_bf16(128, NKV, true, true);    // dV^T, dK^T
-            const uint32_t idQ = idesc_bf16(128, 128, false, true);   // dQ
-            bool ok = mbar_wait(bar_kv, 0, abort_flag, 0x301);
-            for (int it = 0; ok && it < ntiles; ++it) {
-                if (!mbar_wait(bar_qdo_full, it & 1, abort_flag, 0x302)) break;
-                if (it > 0 && !mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x303)) break;
-                tc_fence_after();
-                mma_k128_kmajor(tS, sQ, sK, NKV * 128, idS);
-                mma_k128_kmajor(tdP, sdO, sV, NKV * 128, idS);
-                mma_commit(bar_sdp_full);
-                if (!mbar_wait(bar_pds_full, it & 1, abort_flag, 0x304)) break;
-                tc_fence_after();
-                // dV^T[d x kv] += dO^T P ; dK^T[d x kv] += Q^T dS   (K = 128 query rows)
+    } else if (warp >= 8) {
+        // ---------------- dQ flush (thread <-> query row of the tile) ----------------
+        regs_shrink<80>();
+        const int r = ((warp & 3) << 5) | lane;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        uint32_t fph = 0;  // staging rounds (two per tile)
+        for (int it = 0; it < ntiles; ++it) {
+            int t = 0, e = 0;
+            const bool valid = tile_row(R, T, it, r, t, e);
+            const int t_mine = valid ? t : -1;
+            if (!mbar_wait(bar_dq_full, it & 1, abort_flag, 0x307)) break;
+            tc_fence_after();
+            bool ok = true;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    mma_bf16_ss(tdV, smem_desc_sw128(sdO + kk * 2048, kChunkBytes),
-                                smem_desc_sw128(sP + kk * 2048, kChunkBytes), idT, (it > 0 || kk > 0) ? 1u : 0u);
+            for (int half = 0; half < 2; ++half) {
+                // the previous round's rows have been read by every flush warp
+                if (fph > 0 && !mbar_wait(bar_f_free, (fph - 1) & 1, abort_flag, 0x30b)) {
+                    ok = false;
+                    break;
                 }
+                // row r: 16 units of 16 bytes, unit q at position q ^ (r & 15) (conflict-free both ways);
+                // 32 columns at a time from tensor memory
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    mma_bf16_ss(tdK, smem_desc_sw128(sQ + kk * 2048, kChunkBytes),
-                                smem_desc_sw128(sdS + kk * 2048, kChunkBytes), idT, (it > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(bar_qdo_free);
-                // dQ[q x d] = dS K   (K = NKV keys)
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t g[32];
+                    tmem_ld32_async(tdQ + lane_off + 64 * half + 32 * c, g);
+                    tmem_ld_wait();
+                    if (half == 1 && c == 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar_dq_empty);  // dQ has left tensor memory: the next S may overwrite it
+                    }
 #pragma unroll
-                for (int kk = 0; kk < NKV / 16; ++kk) {
-                    mma_bf16_ss(tdQ, smem_desc_sw128(sdS + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16),
-                                smem_desc_sw128(sK + kk * 2048, NKV * 128), idQ, kk > 0 ? 1u : 0u);
+                    for (int q8 = 0; q8 < 8; ++q8) {
+                        const int q = 8 * c + q8;
+                        const uint32_t *x = g + 4 * q8;
+                        st_shared_v4(sF + r * 256 + (((q ^ r) & 15) << 4),
+                                     __float_as_uint(__uint_as_float(x[0]) * a.scale),
+                                     __float_as_uint(__uint_as_float(x[1]) * a.scale),
+                                     __float_as_uint(__uint_as_float(x[2]) * a.scale),
+                                     __float_as_uint(__uint_as_float(x[3]) * a.scale));
+                    }
                 }
-                mma_commit(bar_dq_full);
+                mbar_arrive(bar_f_staged);
+                if (!mbar_wait(bar_f_staged, fph & 1, abort_flag, 0x30a)) {
+                    ok = false;
+                    break;
+                }
+                // the warp's 32 rows, two per instruction: half-warp h2 takes row 2i + h2,
+                // lane l & 15 its 16-byte unit
+                const int u = lane & 15;
+#pragma unroll 4
+                for (int i = 0; i < 16; ++i) {
+                    const int rl = 2 * i + (lane >> 4);
+                    const int row = 32 * (warp & 3) + rl;
+                    const int t_dst = __shfl_sync(0xffffffffu, t_mine, rl);
+                    float4 v;
+                    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                                 : "r"(sF + row * 256 + (((u ^ row) & 15) << 4)));
+                    if (t_dst >= 0)
+                        atomicAdd(reinterpret_cast<float4 *>(a.dQacc + (head_rows + t_dst) * kD + 64 * half) + u, v);
+                }
+                mbar_arrive(bar_f_free);
+                ++fph;
             }
-            mma_commit(bar_final);
-            mbar_wait(bar_final, 0, abort_flag, 0x305);
+            if (!ok) break;
         }
     } else {
-        // ---------------- compute warps ----------------
+        // ---------------- softmax / dS warpgroups ----------------
+        regs_grow<152>();
         const int r = ((warp & 3) << 5) | lane;  // tile row
         const int h = warp >> 2;                 // column half
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        int t = 0, e = 0;
-        bool valid = ntiles > 0 && tile_row(R, T, 0, r, t, e);
-        if (sparse) {
-            // warpgroup 0 gathers Q rows, warpgroup 1 dO rows
-            const __nv_bfloat16 *src = (h == 0 ? a.Q : a.dO) + (head_rows + (valid ? t : 0)) * kD;
-            gather_row(h == 0 ? sQ : sdO, src, valid, r);
-            cp_async_commit();
-            cp_async_wait_all();
-            fence_proxy_async_smem();
-            mbar_arrive(bar_qdo_full);
-        }
         bool ok = true;
         for (int it = 0; it < ntiles; ++it) {
+            int t = 0, e = 0;
+            const bool valid = tile_row(R, T, it, r, t, e);
             const float lse2 = valid ? __ldg(a.lse + head_rows + t) * kLog2e : 0.f;
             const float Dt = valid ? __ldg(a.Dvec + head_rows + t) : 0.f;
             if (!mbar_wait(bar_sdp_full, it & 1, abort_flag, 0x306)) {
@@ -207,31 +316,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 break;
             }
             tc_fence_after();
-            // the previous tile's dQ flush staged through P / dS: wait until it has read them
-            if (kCoalescedFlush && it > 0 && !mbar_wait(bar_flushed, (it - 1) & 1, abort_flag, 0x309)) {
-                ok = false;
-                break;
-            }
-            // all tensor-memory loads of this row half in flight at once, one wait
-            uint32_t sraw[HALF / 32][32], draw[HALF / 32][32];
-#pragma unroll
-            for (int c = 0; c < HALF / 32; ++c) {
-                tmem_ld32_async(tS + lane_off + h * HALF + 32 * c, sraw[c]);
-                tmem_ld32_async(tdP + lane_off + h * HALF + 32 * c, draw[c]);
-            }
-            tmem_ld_wait();
             // key kv0 + col is attended when col <= lim (causal inside the diagonal block)
             const int lim = valid ? t - kv0 - h * HALF : -1;
 #pragma unroll
             for (int c = 0; c < HALF / 32; ++c) {
+                uint32_t sraw[32], draw[32];
+                tmem_ld32_async(tS + lane_off + h * HALF + 32 * c, sraw);
+                tmem_ld32_async(tdP + lane_off + h * HALF + 32 * c, draw);
+                tmem_ld_wait();
                 float sv[32], dp[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const float p = (32 * c + i <= lim)
-                                        ? fast_exp2(fmaf(__uint_as_float(sraw[c][i]), a.scale_log2, -lse2))
+                                        ? fast_exp2(fmaf(__uint_as_float(sraw[i]), a.scale_log2, -lse2))
                                         : 0.f;
                     sv[i] = p;
-                    dp[i] = p * (__uint_as_float(draw[c][i]) - Dt);
+                    dp[i] = p * (__uint_as_float(draw[i]) - Dt);
                 }
                 store_row32_bf16(sP, kChunkBytes, r, h * HALF + 32 * c, sv);
                 store_row32_bf16(sdS, kChunkBytes, r, h * HALF + 32 * c, dp);
@@ -239,86 +339,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(bar_pds_full);
-            // next tile's rows (sparse: gathered by these threads once Q/dO are consumed)
-            int t_next = 0, e_next = 0;
-            bool valid_next = false;
-            const bool more = it + 1 < ntiles;
-            if (more) valid_next = tile_row(R, T, it + 1, r, t_next, e_next);
-            if (sparse && more) {
-                if (!mbar_wait(bar_qdo_free, it & 1, abort_flag, 0x308)) {
-                    ok = false;
-                    break;
-                }
-                const __nv_bfloat16 *src = (h == 0 ? a.Q : a.dO) + (head_rows + (valid_next ? t_next : 0)) * kD;
-                gather_row(h == 0 ? sQ : sdO, src, valid_next, r);
-                cp_async_commit();
-            }
-            if (!mbar_wait(bar_dq_full, it & 1, abort_flag, 0x307)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            uint32_t g[2][32];
-            tmem_ld32_async(tdQ + lane_off + h * 64, g[0]);
-            tmem_ld32_async(tdQ + lane_off + h * 64 + 32, g[1]);
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive(bar_dq_empty);
-            if constexpr (kCoalescedFlush) {
-                // Stage the tile's dQ rows (fp32, 512 B per row, 16-byte units XOR-swizzled by
-                // row) in the P / dS buffers, free once every MMA of this tile has completed;
-                // then each warp adds 16 whole rows with coalesced float4 reductions.
-                auto stage_addr = [&](int row, int unit) -> uint32_t {
-                    const uint32_t base = row < 64 ? sP + row * 512 : sdS + (row - 64) * 512;
-                    return base + (((unit ^ row) & 31) << 4);
-                };
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const uint32_t *x = g[q >> 3] + 4 * (q & 7);
-                    st_shared_v4(stage_addr(r, 16 * h + q), __float_as_uint(__uint_as_float(x[0]) * a.scale),
-                                 __float_as_uint(__uint_as_float(x[1]) * a.scale),
-                                 __float_as_uint(__uint_as_float(x[2]) * a.scale),
-                                 __float_as_uint(__uint_as_float(x[3]) * a.scale));
-                }
-                mbar_arrive(bar_staged);
-                if (!mbar_wait(bar_staged, it & 1, abort_flag, 0x30a)) {
-                    ok = false;
-                    break;
-                }
-                const int t_mine = valid ? t : -1;
-#pragma unroll 4
-                for (int i = 0; i < 16; ++i) {
-                    const int row = 32 * (warp & 3) + 16 * h + i;
-                    const int t_dst = __shfl_sync(0xffffffffu, t_mine, 16 * h + i);
-                    if (t_dst >= 0) {
-                        float4 v;
-                        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                                     : "r"(stage_addr(row, lane)));
-                        atomicAdd(reinterpret_cast<float4 *>(a.dQacc + (head_rows + t_dst) * kD) + lane, v);
-                    }
-                }
-                mbar_arrive(bar_flushed);
-            } else if (valid) {
-                float4 *dq = reinterpret_cast<float4 *>(a.dQacc + (head_rows + t) * kD + h * 64);
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const uint32_t *x = g[q >> 3] + 4 * (q & 7);
-                    atomicAdd(dq + q, make_float4(__uint_as_float(x[0]) * a.scale, __uint_as_float(x[1]) * a.scale,
-                                                  __uint_as_float(x[2]) * a.scale, __uint_as_float(x[3]) * a.scale));
-                }
-            }
-            if (sparse && more) {
-                cp_async_wait_all();
-                fence_proxy_async_smem();
-                mbar_arrive(bar_qdo_full);
-            }
-            t = t_next;
-            e = e_next;
-            valid = valid_next;
         }
-        cp_async_wait_all();
         // Epilogue: thread <-> head-dim row r of dV^T / dK^T, key columns of its half.
+        if (ok && !mbar_wait(bar_final, 0, abort_flag, 0x30c)) ok = false;
+        tc_fence_after();
         if (ok) {
 #pragma unroll
             for (int c0 = h * HALF; c0 < (h + 1) * HALF; c0 += 32) {
@@ -326,24 +350,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tmem_ld32_async(tdV + lane_off + c0, rv);
                 tmem_ld32_async(tdK + lane_off + c0, rk);
                 tmem_ld_wait();
-                float gv[32], gk[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    gv[i] = __uint_as_float(rv[i]);
-                    gk[i] = __uint_as_float(rk[i]);
-                }
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int kv = kv0 + c0 + i;
                     if (kv < T) {
                         const size_t off = (head_rows + kv) * kD + r;
-                        float vv = ntiles > 0 ? gv[i] : 0.f, kk = ntiles > 0 ? gk[i] * a.scale : 0.f;
+                        float vv = ntiles > 0 ? __uint_as_float(rv[i]) : 0.f;
+                        float kq = ntiles > 0 ? __uint_as_float(rk[i]) * a.scale : 0.f;
                         if (a.accumulate) {
                             vv += __bfloat162float(a.dV[off]);
-                            kk += __bfloat162float(a.dK[off]);
+                            kq += __bfloat162float(a.dK[off]);
                         }
                         a.dV[off] = __float2bfloat16_rn(vv);
-                        a.dK[off] = __float2bfloat16_rn(kk);
+                        a.dK[off] = __float2bfloat16_rn(kq);
                     }
                 }
             }
