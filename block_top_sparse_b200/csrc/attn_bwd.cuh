@@ -17,10 +17,12 @@
 //   warps 0-7    two warpgroups; warp w owns query row (w & 3)*32 + lane and
 //                column half (w >> 2) of the row-wise phase (P, dS), then the
 //                dV, dK epilogue;
-//   warps 8-11   dQ flush: thread <-> query row; dQ leaves tensor memory in two
-//                64-column halves through a 32 KB staging buffer of its own and
-//                is added with coalesced float4 reductions (two 256-byte row
-//                halves per warp instruction), so the next tile never waits for it;
+//   warps 8-11   dQ flush: thread <-> query row; the whole dQ tile leaves tensor
+//                memory at once (columns 0-63 into a 32 KB staging buffer of its
+//                own, 64-127 into the P region, free once dQ is computed), so the
+//                next tile's S can start; the tile is then added with coalesced
+//                float4 reductions (two 256-byte row halves per warp instruction),
+//                the P-region half first so that the next tile's P is not held up;
 //   warp 12      MMA issuer (one thread);
 //   warp 13      TMA producer (K_j, V_j; contiguous Q / dO tiles of the full stream);
 //   warps 14-19  sparse stream: gather the next tile's Q and dO rows with
@@ -78,6 +80,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint64_t *bar_kv = bars + 0, *bar_qdo_full = bars + 1, *bar_sdp_full = bars + 2, *bar_pds_full = bars + 3;
     uint64_t *bar_qdo_free = bars + 4, *bar_dq_full = bars + 5, *bar_dq_empty = bars + 6, *bar_final = bars + 7;
     uint64_t *bar_f_staged = bars + 8, *bar_f_free = bars + 9;  // dQ staging buffer handshakes
+    uint64_t *bar_p_free = bars + 12;  // the P region's dQ half has been read by the flush
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 11);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -117,6 +120,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(bar_final, 1);
         mbar_init(bar_f_staged, 128);
         mbar_init(bar_f_free, 128);
+        mbar_init(bar_p_free, 128);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -237,51 +241,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         regs_shrink<80>();
         const int r = ((warp & 3) << 5) | lane;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        uint32_t fph = 0;  // staging rounds (two per tile)
         for (int it = 0; it < ntiles; ++it) {
             int t = 0, e = 0;
             const bool valid = tile_row(R, T, it, r, t, e);
             const int t_mine = valid ? t : -1;
             if (!mbar_wait(bar_dq_full, it & 1, abort_flag, 0x307)) break;
             tc_fence_after();
-            bool ok = true;
+            // this buffer's previous contents (columns 0-63 of tile it-1) have been read
+            if (it > 0 && !mbar_wait(bar_f_free, (it - 1) & 1, abort_flag, 0x30b)) break;
+            // row r of half hf: 16 units of 16 bytes, unit q at position q ^ (r & 15) (conflict-free
+            // both ways); half 0 -> sF, half 1 -> the P region; 32 columns at a time
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                // the previous round's rows have been read by every flush warp
-                if (fph > 0 && !mbar_wait(bar_f_free, (fph - 1) & 1, abort_flag, 0x30b)) {
-                    ok = false;
-                    break;
+            for (int c = 0; c < 4; ++c) {
+                uint32_t g[32];
+                tmem_ld32_async(tdQ + lane_off + 32 * c, g);
+                tmem_ld_wait();
+                if (c == 3) {
+                    tc_fence_before();
+                    mbar_arrive(bar_dq_empty);  // dQ has left tensor memory: the next S may overwrite it
                 }
-                // row r: 16 units of 16 bytes, unit q at position q ^ (r & 15) (conflict-free both ways);
-                // 32 columns at a time from tensor memory
+                const uint32_t base = (c < 2 ? sF : sP) + r * 256;
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t g[32];
-                    tmem_ld32_async(tdQ + lane_off + 64 * half + 32 * c, g);
-                    tmem_ld_wait();
-                    if (half == 1 && c == 1) {
-                        tc_fence_before();
-                        mbar_arrive(bar_dq_empty);  // dQ has left tensor memory: the next S may overwrite it
-                    }
+                for (int q8 = 0; q8 < 8; ++q8) {
+                    const int q = 8 * (c & 1) + q8;
+                    const uint32_t *x = g + 4 * q8;
+                    st_shared_v4(base + (((q ^ r) & 15) << 4), __float_as_uint(__uint_as_float(x[0]) * a.scale),
+                                 __float_as_uint(__uint_as_float(x[1]) * a.scale),
+                                 __float_as_uint(__uint_as_float(x[2]) * a.scale),
+                                 __float_as_uint(__uint_as_float(x[3]) * a.scale));
+                }
+            }
+            mbar_arrive(bar_f_staged);
+            if (!mbar_wait(bar_f_staged, it & 1, abort_flag, 0x30a)) break;
+            // the warp's 32 rows, two per instruction: half-warp h2 takes row 2i + h2, lane l & 15
+            // its 16-byte unit; the P-region half (columns 64-127) first
+            const int u = lane & 15;
 #pragma unroll
-                    for (int q8 = 0; q8 < 8; ++q8) {
-                        const int q = 8 * c + q8;
-                        const uint32_t *x = g + 4 * q8;
-                        st_shared_v4(sF + r * 256 + (((q ^ r) & 15) << 4),
-                                     __float_as_uint(__uint_as_float(x[0]) * a.scale),
-                                     __float_as_uint(__uint_as_float(x[1]) * a.scale),
-                                     __float_as_uint(__uint_as_float(x[2]) * a.scale),
-                                     __float_as_uint(__uint_as_float(x[3]) * a.scale));
-                    }
-                }
-                mbar_arrive(bar_f_staged);
-                if (!mbar_wait(bar_f_staged, fph & 1, abort_flag, 0x30a)) {
-                    ok = false;
-                    break;
-                }
-                // the warp's 32 rows, two per instruction: half-warp h2 takes row 2i + h2,
-                // lane l & 15 its 16-byte unit
-                const int u = lane & 15;
+            for (int hf = 1; hf >= 0; --hf) {
+                const uint32_t buf = hf ? sP : sF;
 #pragma unroll 4
                 for (int i = 0; i < 16; ++i) {
                     const int rl = 2 * i + (lane >> 4);
@@ -290,14 +287,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     float4 v;
                     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                                  : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                                 : "r"(sF + row * 256 + (((u ^ row) & 15) << 4)));
+                                 : "r"(buf + row * 256 + (((u ^ row) & 15) << 4)));
                     if (t_dst >= 0)
-                        atomicAdd(reinterpret_cast<float4 *>(a.dQacc + (head_rows + t_dst) * kD + 64 * half) + u, v);
+                        atomicAdd(reinterpret_cast<float4 *>(a.dQacc + (head_rows + t_dst) * kD + 64 * hf) + u, v);
                 }
-                mbar_arrive(bar_f_free);
-                ++fph;
+                mbar_arrive(hf ? bar_p_free : bar_f_free);
             }
-            if (!ok) break;
         }
     } else {
         // ---------------- softmax / dS warpgroups ----------------
@@ -312,6 +307,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float lse2 = valid ? __ldg(a.lse + head_rows + t) * kLog2e : 0.f;
             const float Dt = valid ? __ldg(a.Dvec + head_rows + t) : 0.f;
             if (!mbar_wait(bar_sdp_full, it & 1, abort_flag, 0x306)) {
+                ok = false;
+                break;
+            }
+            // the previous tile's dQ half staged over P (and dS for 64-key units) has been read
+            if (it > 0 && !mbar_wait(bar_p_free, (it - 1) & 1, abort_flag, 0x30d)) {
                 ok = false;
                 break;
             }
