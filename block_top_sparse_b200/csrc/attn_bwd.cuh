@@ -18,11 +18,14 @@
 //                column half (w >> 2) of the row-wise phase (P, dS), then the
 //                dV, dK epilogue;
 //   warps 8-11   dQ flush: thread <-> query row; the whole dQ tile leaves tensor
-//                memory at once (columns 0-63 into a 32 KB staging buffer of its
-//                own, 64-127 into the P region, free once dQ is computed), so the
-//                next tile's S can start; the tile is then added with coalesced
-//                float4 reductions (two 256-byte row halves per warp instruction),
-//                the P-region half first so that the next tile's P is not held up;
+//                memory at once, so the next tile's S can start.  Full stream (a
+//                tile's rows are contiguous): columns 0-63 into a 32 KB staging
+//                buffer of its own, 64-127 into the P region (free once dQ is
+//                computed), added by four TMA tensor reduce-adds issued by one
+//                thread.  Sparse stream (gathered rows): columns 64-127 wait in
+//                registers while 0-63 go through the staging buffer, each half
+//                added with coalesced float4 reductions (two 256-byte row halves
+//                per warp instruction);
 //   warp 12      MMA issuer (one thread);
 //   warp 13      TMA producer (K_j, V_j; contiguous Q / dO tiles of the full stream);
 //   warps 14-19  sparse stream: gather the next tile's Q and dO rows with
@@ -62,7 +65,7 @@ struct BwdArgs {
 };
 
 // 640 threads launched with 96 registers each (61,440); setmaxnreg moves them to
-// softmax 2 x 152, flush 80, MMA / producer / gather 2 x 48: 128 * 480 = 61,440.
+// softmax 2 x 144, flush 96, MMA / producer / gather 2 x 48: 128 * 480 = 61,440.
 constexpr int kBwdThreads = 640;
 constexpr int kBwdGatherWarps = 6;
 constexpr int kBwdGatherPairs = (64 + kBwdGatherWarps - 1) / kBwdGatherWarps;
@@ -71,7 +74,7 @@ template <int NKV>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
-                    const BwdArgs a) {
+                    const __grid_constant__ CUtensorMap tmdQ, const BwdArgs a) {
     using L = BwdSmem<NKV>;
     constexpr int HALF = NKV / 2;  // S / dP columns per warpgroup
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -119,8 +122,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(bar_dq_empty, 128);
         mbar_init(bar_final, 1);
         mbar_init(bar_f_staged, 128);
-        mbar_init(bar_f_free, 128);
-        mbar_init(bar_p_free, 128);
+        // staging buffers released by every flush thread (sparse: two rounds per tile through
+        // the staging buffer) or by the thread that issued the TMA reduce-adds once they have
+        // read shared memory (full: P region and staging buffer)
+        mbar_init(bar_f_free, sparse ? 128 : 1);
+        mbar_init(bar_p_free, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -238,65 +244,134 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     } else if (warp >= 8) {
         // ---------------- dQ flush (thread <-> query row of the tile) ----------------
-        regs_shrink<80>();
+        // (stays at the 96 registers it was launched with)
         const int r = ((warp & 3) << 5) | lane;
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        for (int it = 0; it < ntiles; ++it) {
-            int t = 0, e = 0;
-            const bool valid = tile_row(R, T, it, r, t, e);
-            const int t_mine = valid ? t : -1;
-            if (!mbar_wait(bar_dq_full, it & 1, abort_flag, 0x307)) break;
-            tc_fence_after();
-            // this buffer's previous contents (columns 0-63 of tile it-1) have been read
-            if (it > 0 && !mbar_wait(bar_f_free, (it - 1) & 1, abort_flag, 0x30b)) break;
-            // row r of half hf: 16 units of 16 bytes, unit q at position q ^ (r & 15) (conflict-free
-            // both ways); half 0 -> sF, half 1 -> the P region; 32 columns at a time
+        if (!sparse) {
+            for (int it = 0; it < ntiles; ++it) {
+                if (!mbar_wait(bar_dq_full, it & 1, abort_flag, 0x307)) break;
+                tc_fence_after();
+                // both staging buffers' previous contents (tile it-1) have been read by the TMA unit
+                if (it > 0 && !mbar_wait(bar_f_free, (it - 1) & 1, abort_flag, 0x30b)) break;
+                // Full stream: columns 32c .. 32c+31 as a 128-row x 128-byte swizzled chunk (chunks
+                // 0, 1 in sF, 2, 3 in the P region), added by four TMA tensor reduce-adds
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t g[32];
-                tmem_ld32_async(tdQ + lane_off + 32 * c, g);
-                tmem_ld_wait();
-                if (c == 3) {
-                    tc_fence_before();
-                    mbar_arrive(bar_dq_empty);  // dQ has left tensor memory: the next S may overwrite it
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t g[32];
+                    tmem_ld32_async(tdQ + lane_off + 32 * c, g);
+                    tmem_ld_wait();
+                    if (c == 3) {
+                        tc_fence_before();
+                        mbar_arrive(bar_dq_empty);  // dQ has left tensor memory: the next S may overwrite it
+                    }
+                    const uint32_t base = (c < 2 ? sF : sP) + (c & 1) * kChunkBytes + r * 128;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const uint32_t *x = g + 4 * q;
+                        st_shared_v4(base + (((q ^ r) & 7) << 4), __float_as_uint(__uint_as_float(x[0]) * a.scale),
+                                     __float_as_uint(__uint_as_float(x[1]) * a.scale),
+                                     __float_as_uint(__uint_as_float(x[2]) * a.scale),
+                                     __float_as_uint(__uint_as_float(x[3]) * a.scale));
+                    }
                 }
-                const uint32_t base = (c < 2 ? sF : sP) + r * 256;
+                fence_proxy_async_smem();  // generic-proxy staging writes -> TMA reads
+                mbar_arrive(bar_f_staged);
+                if (r == 0) {
+                    if (!mbar_wait(bar_f_staged, it & 1, abort_flag, 0x30a)) break;
+                    // rows past T in the last tile hold exact zeros (P = 0 there); rows past the
+                    // tensor are clipped by the TMA unit
+                    const int row0 = static_cast<int>(head_rows) + kv0 + it * kTileQ;
+                    // the P-region chunks first, in a group of their own, so that P is released early
+                    tma_reduce_add_2d(&tmdQ, sP, 64, row0);
+                    tma_reduce_add_2d(&tmdQ, sP + kChunkBytes, 96, row0);
+                    bulk_commit();
+                    tma_reduce_add_2d(&tmdQ, sF, 0, row0);
+                    tma_reduce_add_2d(&tmdQ, sF + kChunkBytes, 32, row0);
+                    bulk_commit();
+                    bulk_wait_read_all_but_1();
+                    mbar_arrive(bar_p_free);
+                    bulk_wait_read();
+                    mbar_arrive(bar_f_free);
+                }
+            }
+            if (r == 0) bulk_wait();  // the TMA reduce-adds have completed
+        } else {
+            // Sparse stream: columns 0-63 go to the staging buffer, 64-127 stay in registers (so
+            // dQ leaves tensor memory at once), then each half is added in turn.  Row r: 16 units of
+            // 16 bytes, unit q at position q ^ (r & 15) (conflict-free both ways).
+            uint32_t fph = 0;  // staging rounds (two per tile)
+            auto stage = [&](const uint32_t (&g)[32], int q0) {
 #pragma unroll
                 for (int q8 = 0; q8 < 8; ++q8) {
-                    const int q = 8 * (c & 1) + q8;
+                    const int q = q0 + q8;
                     const uint32_t *x = g + 4 * q8;
-                    st_shared_v4(base + (((q ^ r) & 15) << 4), __float_as_uint(__uint_as_float(x[0]) * a.scale),
+                    st_shared_v4(sF + r * 256 + (((q ^ r) & 15) << 4), __float_as_uint(__uint_as_float(x[0]) * a.scale),
                                  __float_as_uint(__uint_as_float(x[1]) * a.scale),
                                  __float_as_uint(__uint_as_float(x[2]) * a.scale),
                                  __float_as_uint(__uint_as_float(x[3]) * a.scale));
                 }
-            }
-            mbar_arrive(bar_f_staged);
-            if (!mbar_wait(bar_f_staged, it & 1, abort_flag, 0x30a)) break;
-            // the warp's 32 rows, two per instruction: half-warp h2 takes row 2i + h2, lane l & 15
-            // its 16-byte unit; the P-region half (columns 64-127) first
-            const int u = lane & 15;
+            };
+            for (int it = 0; it < ntiles; ++it) {
+                int t = 0, e = 0;
+                const bool valid = tile_row(R, T, it, r, t, e);
+                const int t_mine = valid ? t : -1;
+                if (!mbar_wait(bar_dq_full, it & 1, abort_flag, 0x307)) break;
+                tc_fence_after();
+                uint32_t hi[2][32];
+                bool ok = true;
 #pragma unroll
-            for (int hf = 1; hf >= 0; --hf) {
-                const uint32_t buf = hf ? sP : sF;
+                for (int hf = 0; hf < 2; ++hf) {
+                    // the previous round's rows have been read by every flush warp
+                    if (fph > 0 && !mbar_wait(bar_f_free, (fph - 1) & 1, abort_flag, 0x30b)) {
+                        ok = false;
+                        break;
+                    }
+                    if (hf == 0) {
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) {
+                            uint32_t g[32];
+                            tmem_ld32_async(tdQ + lane_off + 32 * c, g);
+                            tmem_ld_wait();
+                            stage(g, 8 * c);
+                        }
+                        tmem_ld32_async(tdQ + lane_off + 64, hi[0]);
+                        tmem_ld32_async(tdQ + lane_off + 96, hi[1]);
+                        tmem_ld_wait();
+                        tc_fence_before();
+                        mbar_arrive(bar_dq_empty);  // dQ has left tensor memory: the next S may overwrite it
+                    } else {
+                        stage(hi[0], 0);
+                        stage(hi[1], 8);
+                    }
+                    mbar_arrive(bar_f_staged);
+                    if (!mbar_wait(bar_f_staged, fph & 1, abort_flag, 0x30a)) {
+                        ok = false;
+                        break;
+                    }
+                    // the warp's 32 rows, two per instruction: half-warp h2 takes row 2i + h2,
+                    // lane l & 15 its 16-byte unit
+                    const int u = lane & 15;
 #pragma unroll 4
-                for (int i = 0; i < 16; ++i) {
-                    const int rl = 2 * i + (lane >> 4);
-                    const int row = 32 * (warp & 3) + rl;
-                    const int t_dst = __shfl_sync(0xffffffffu, t_mine, rl);
-                    float4 v;
-                    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                                 : "r"(buf + row * 256 + (((u ^ row) & 15) << 4)));
-                    if (t_dst >= 0)
-                        atomicAdd(reinterpret_cast<float4 *>(a.dQacc + (head_rows + t_dst) * kD + 64 * hf) + u, v);
+                    for (int i = 0; i < 16; ++i) {
+                        const int rl = 2 * i + (lane >> 4);
+                        const int row = 32 * (warp & 3) + rl;
+                        const int t_dst = __shfl_sync(0xffffffffu, t_mine, rl);
+                        float4 v;
+                        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                                     : "r"(sF + row * 256 + (((u ^ row) & 15) << 4)));
+                        if (t_dst >= 0)
+                            atomicAdd(reinterpret_cast<float4 *>(a.dQacc + (head_rows + t_dst) * kD + 64 * hf) + u, v);
+                    }
+                    mbar_arrive(bar_f_free);
+                    ++fph;
                 }
-                mbar_arrive(hf ? bar_p_free : bar_f_free);
+                if (!ok) break;
             }
         }
     } else {
         // ---------------- softmax / dS warpgroups ----------------
-        regs_grow<152>();
+        regs_grow<144>();
         const int r = ((warp & 3) << 5) | lane;  // tile row
         const int h = warp >> 2;                 // column half
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -307,11 +382,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float lse2 = valid ? __ldg(a.lse + head_rows + t) * kLog2e : 0.f;
             const float Dt = valid ? __ldg(a.Dvec + head_rows + t) : 0.f;
             if (!mbar_wait(bar_sdp_full, it & 1, abort_flag, 0x306)) {
-                ok = false;
-                break;
-            }
-            // the previous tile's dQ half staged over P (and dS for 64-key units) has been read
-            if (it > 0 && !mbar_wait(bar_p_free, (it - 1) & 1, abort_flag, 0x30d)) {
                 ok = false;
                 break;
             }
@@ -333,9 +403,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     sv[i] = p;
                     dp[i] = p * (__uint_as_float(draw[i]) - Dt);
                 }
+                // full stream: the previous tile's dQ staged over P (and dS for 64-key units) has been read
+                if (!sparse && c == 0 && it > 0) ok = mbar_wait(bar_p_free, (it - 1) & 1, abort_flag, 0x30d);
                 store_row32_bf16(sP, kChunkBytes, r, h * HALF + 32 * c, sv);
                 store_row32_bf16(sdS, kChunkBytes, r, h * HALF + 32 * c, dp);
             }
+            if (!ok) break;
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(bar_pds_full);

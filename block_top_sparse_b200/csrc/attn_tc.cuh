@@ -380,16 +380,19 @@ __global__ void __launch_bounds__(kFullFwdThreads, 1)
 //   warps 8-11 and 13-15 gather each tile's query rows with cp.async, a
 //   half-warp per 256-byte row (a gather's cost is set by the number of warp
 //   instructions in flight, so seven warps share it; completion on an mbarrier);
-//   warp 12 loads K_j, V_j (TMA) and issues the MMAs in the order
-//   S(it), PV(it-1), S(it+1), PV(it), ... so that one warpgroup's softmax
-//   overlaps the other's MMAs and epilogue.
-// smem: Q[2] 32 KB each | K, V NKV*256 each | O staging[2] 32 KB each | barriers
+//   warp 12 loads K_j, V_j (TMA) and issues each S(it) as soon as its query
+//   rows have landed and each PV(it) as soon as its P is ready (polling both,
+//   S(it) never ahead of PV(it-2), whose P it overwrites), so that one
+//   warpgroup's softmax overlaps the other's MMAs and epilogue.
+// smem: Q[3] 32 KB each | K, V NKV*256 each | O staging[2] 32 KB each | barriers
 // tmem: S/P[2] at 0 / 128, O[2] at 256 / 384 (512 allocated).
 // ---------------------------------------------------------------------------
+constexpr int kSparseFwdQStages = 3;
+
 template <int NKV>
 struct SparseFwdSmem {
-    static constexpr int kQ = 0;                          // [2]
-    static constexpr int kK = kQ + 2 * 2 * kChunkBytes;
+    static constexpr int kQ = 0;                          // [kSparseFwdQStages]
+    static constexpr int kK = kQ + kSparseFwdQStages * 2 * kChunkBytes;
     static constexpr int kV = kK + 2 * NKV * 128;
     static constexpr int kO = kV + 2 * NKV * 128;         // [2] 2 chunks x 128 rows x 128 B, swizzled
     static constexpr int kOStage = 2 * kChunkBytes;
@@ -443,11 +446,12 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBar);
     uint64_t *bar_kv = bars + 0;
-    uint64_t *bar_q_full = bars + 1;   // [2]
-    uint64_t *bar_s_full = bars + 3;   // [2]
+    uint64_t *bar_s_full = bars + 3;   // [2] tensor-memory buffers
     uint64_t *bar_p_full = bars + 5;   // [2]
     uint64_t *bar_o_full = bars + 7;   // [2]
     uint64_t *bar_final = bars + 11;
+    uint64_t *bar_q_full = bars + 16;  // [kSparseFwdQStages] query-row stages landed
+    uint64_t *bar_q_free = bars + 20;  // [kSparseFwdQStages] the S MMA reading a stage has completed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 15);
 
@@ -466,8 +470,11 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
+        for (int q = 0; q < kSparseFwdQStages; ++q) {
+            mbar_init(bar_q_full + q, 32 * kSparseFwdGatherWarps);  // one cp.async arrival per gather lane
+            mbar_init(bar_q_free + q, 1);
+        }
         for (int g = 0; g < 2; ++g) {
-            mbar_init(bar_q_full + g, 32 * kSparseFwdGatherWarps);  // one cp.async arrival per gather lane
             mbar_init(bar_s_full + g, 1);
             mbar_init(bar_p_full + g, 128);
             mbar_init(bar_o_full + g, 1);
@@ -493,17 +500,16 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
         int tn[kGatherPairs];
         gather_rows_load(R, 0, gw, lane, tn);
         for (int it = 0; it < ntiles; ++it) {
-            const int g = it & 1;
-            int tc[kGatherPairs];
-#pragma unroll
-            for (int q = 0; q < kGatherPairs; ++q) tc[q] = tn[q];
-            if (it + 1 < ntiles) gather_rows_load(R, it + 1, gw, lane, tn);  // one tile ahead
-            // Q[g] is free once the S MMA of tile it-2 has completed (one lane waits for the warp)
+            const int qs = it % kSparseFwdQStages;
+            // stage qs is free once the S MMA of tile it-3 has completed (one lane waits for the warp);
+            // the stage's own barrier completes once per use, so its phases cannot run ahead
             bool ok = true;
-            if (lane == 0 && it >= 2) ok = mbar_wait(bar_s_full + g, ((it - 2) >> 1) & 1, abort_flag, 0x208);
+            if (lane == 0 && it >= kSparseFwdQStages)
+                ok = mbar_wait(bar_q_free + qs, (it / kSparseFwdQStages - 1) & 1, abort_flag, 0x208);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            gather_rows_issue(smem_u32(smem + L::kQ + g * 2 * kChunkBytes), Q, head_rows, gw, lane, tc);
-            cp_async_mbar_arrive_noinc(bar_q_full + g);
+            gather_rows_issue(smem_u32(smem + L::kQ + qs * 2 * kChunkBytes), Q, head_rows, gw, lane, tn);
+            cp_async_mbar_arrive_noinc(bar_q_full + qs);
+            if (it + 1 < ntiles) gather_rows_load(R, it + 1, gw, lane, tn);  // in flight during the next wait
         }
         cp_async_wait_all();
     } else if (warp == 12) {
@@ -516,20 +522,14 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
             const uint32_t idS = idesc_bf16(128, NKV, false, false);
             const uint32_t idO = idesc_bf16(128, 128, false, true);
             bool ok = mbar_wait(bar_kv, 0, abort_flag, 0x201);
-            // S(it) overwrites the P of tile it-2 in the same tensor-memory columns; the PV MMA
-            // reading it was issued earlier and tensor-core operations run in issue order.
-            for (int it = 0; ok && it <= ntiles; ++it) {
-                if (it < ntiles) {
-                    const int g = it & 1, i = it >> 1;
-                    if (!mbar_wait(bar_q_full + g, i & 1, abort_flag, 0x202)) break;
-                    tc_fence_after();
-                    mma_k128_kmajor(tmem + 128 * g, smem_u32(smem + L::kQ + g * 2 * kChunkBytes), sK, NKV * 128,
-                                    idS);
-                    mma_commit(bar_s_full + g);
-                }
-                if (it >= 1) {
-                    const int g = (it - 1) & 1, i = (it - 1) >> 1;
-                    if (!mbar_wait(bar_p_full + g, i & 1, abort_flag, 0x204)) break;
+            // S(it) overwrites the P of tile it-2 in the same tensor-memory columns: it is issued
+            // only after PV(it-2) (tensor-core operations run in issue order).
+            int is = 0, ip = 0;  // next S and next PV to issue
+            uint64_t t_idle = globaltimer_ns();
+            while (ok && ip < ntiles) {
+                bool progressed = false;
+                if (ip < is && mbar_try_wait(bar_p_full + (ip & 1), (ip >> 1) & 1)) {
+                    const int g = ip & 1;
                     tc_fence_after();
                     // O_g = P_g V : A = P from tensor memory (bf16 pairs over S_g), B = V [NKV x d] MN-major
 #pragma unroll
@@ -537,6 +537,30 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
                         mma_bf16_ts(tmem + 256 + 128 * g, tmem + 128 * g + kk * 8,
                                     smem_desc_sw128(sV + kk * 2048, NKV * 128), idO, kk > 0 ? 1u : 0u);
                     mma_commit(bar_o_full + g);
+                    ++ip;
+                    progressed = true;
+                }
+                if (is < ntiles && is < ip + 2 &&
+                    mbar_try_wait(bar_q_full + is % kSparseFwdQStages, (is / kSparseFwdQStages) & 1)) {
+                    const int g = is & 1;
+                    fence_proxy_async_smem();  // cp.async-written rows -> tensor-core reads
+                    tc_fence_after();
+                    mma_k128_kmajor(tmem + 128 * g,
+                                    smem_u32(smem + L::kQ + (is % kSparseFwdQStages) * 2 * kChunkBytes), sK,
+                                    NKV * 128, idS);
+                    mma_commit(bar_s_full + g);
+                    mma_commit(bar_q_free + is % kSparseFwdQStages);
+                    ++is;
+                    progressed = true;
+                }
+                if (progressed) {
+                    t_idle = globaltimer_ns();
+                } else if (*abort_flag) {
+                    ok = false;
+                } else if (globaltimer_ns() - t_idle > kWaitLimitNs) {
+                    *abort_flag = 1;
+                    record_error(ERR_TIMEOUT, 0x202);
+                    ok = false;
                 }
             }
             mma_commit(bar_final);

@@ -129,6 +129,12 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // Wait until every bulk operation of this thread has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
+// Wait until all but the most recent bulk async-group of this thread have finished
+// reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all_but_1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 // Wait until every bulk operation of this thread has completed.
 __device__ __forceinline__ void bulk_wait() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -170,6 +176,15 @@ __device__ __forceinline__ void tma_gather4(const CUtensorMap *map, uint64_t *ba
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src_smem, int col, int row) {
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(col),
                  "r"(row), "r"(src_smem)
+                 : "memory");
+}
+
+// Tiled TMA reduce-add of a box from shared memory into global memory (element
+// type and swizzle of the tensor map; the additions are performed in L2),
+// tracked by this thread's bulk async-group.  Coordinates must be >= 0.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, uint32_t src_smem, int col, int row) {
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map),
+                 "r"(col), "r"(row), "r"(src_smem)
                  : "memory");
 }
 

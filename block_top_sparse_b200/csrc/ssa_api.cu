@@ -159,6 +159,19 @@ bool make_tmap(CUtensorMap *m, const void *base, size_t rows, int box_rows) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 view [rows, 128] of the dQ accumulator, box 32 columns x 128 rows (128-byte rows, swizzled).
+bool make_tmap_f32(CUtensorMap *m, const void *base, size_t rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    const cuuint64_t gdim[2] = {128, rows};
+    const cuuint64_t gstride[1] = {128 * 4};
+    const cuuint32_t box[2] = {32, 128};
+    const cuuint32_t estride[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), gdim, gstride, box, estride,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename K>
 bool set_smem(K kernel, size_t bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) ==
@@ -253,9 +266,9 @@ ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V,
     bwd_prep_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16 *)dO, (const __nv_bfloat16 *)O, Dvec,
                                                        dQacc, S.rows, S.d);
     const int nkv = sparse ? S.s : 128;
-    CUtensorMap tmK, tmV, tmQ, tmdO;
+    CUtensorMap tmK, tmV, tmQ, tmdO, tmdQ;
     if (!make_tmap(&tmK, K, S.rows, nkv) || !make_tmap(&tmV, V, S.rows, nkv) || !make_tmap(&tmQ, Q, S.rows, 128) ||
-        !make_tmap(&tmdO, dO, S.rows, 128))
+        !make_tmap(&tmdO, dO, S.rows, 128) || !make_tmap_f32(&tmdQ, dQacc, S.rows))
         return SSA_ERR_CUDA;
     BwdArgs a{};
     a.Q = (const __nv_bfloat16 *)Q;
@@ -280,11 +293,11 @@ ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V,
     if (nkv == 128) {
         const size_t sm = BwdSmem<128>::kTotal + 1024;
         if (!set_smem(attn_bwd_kernel<128>, sm)) return SSA_ERR_CUDA;
-        attn_bwd_kernel<128><<<units, kBwdThreads, sm, st>>>(tmK, tmV, tmQ, tmdO, a);
+        attn_bwd_kernel<128><<<units, kBwdThreads, sm, st>>>(tmK, tmV, tmQ, tmdO, tmdQ, a);
     } else {
         const size_t sm = BwdSmem<64>::kTotal + 1024;
         if (!set_smem(attn_bwd_kernel<64>, sm)) return SSA_ERR_CUDA;
-        attn_bwd_kernel<64><<<units, kBwdThreads, sm, st>>>(tmK, tmV, tmQ, tmdO, a);
+        attn_bwd_kernel<64><<<units, kBwdThreads, sm, st>>>(tmK, tmV, tmQ, tmdO, tmdQ, a);
     }
     const size_t n = S.rows * S.d;
     acc_to_out_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, st>>>(dQacc, (__nv_bfloat16 *)dQ, n, accumulate);
