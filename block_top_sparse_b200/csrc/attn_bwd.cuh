@@ -256,22 +256,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 // Full stream: columns 32c .. 32c+31 as a 128-row x 128-byte swizzled chunk (chunks
                 // 0, 1 in sF, 2, 3 in the P region), added by four TMA tensor reduce-adds
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t g[32];
-                    tmem_ld32_async(tdQ + lane_off + 32 * c, g);
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    uint32_t g[2][32];
+                    tmem_ld32_async(tdQ + lane_off + 64 * c2, g[0]);
+                    tmem_ld32_async(tdQ + lane_off + 64 * c2 + 32, g[1]);
                     tmem_ld_wait();
-                    if (c == 3) {
+                    if (c2 == 1) {
                         tc_fence_before();
                         mbar_arrive(bar_dq_empty);  // dQ has left tensor memory: the next S may overwrite it
                     }
-                    const uint32_t base = (c < 2 ? sF : sP) + (c & 1) * kChunkBytes + r * 128;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint32_t *x = g + 4 * q;
-                        st_shared_v4(base + (((q ^ r) & 7) << 4), __float_as_uint(__uint_as_float(x[0]) * a.scale),
-                                     __float_as_uint(__uint_as_float(x[1]) * a.scale),
-                                     __float_as_uint(__uint_as_float(x[2]) * a.scale),
-                                     __float_as_uint(__uint_as_float(x[3]) * a.scale));
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const uint32_t base = (c2 == 0 ? sF : sP) + cc * kChunkBytes + r * 128;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const uint32_t *x = g[cc] + 4 * q;
+                            st_shared_v4(base + (((q ^ r) & 7) << 4), __float_as_uint(__uint_as_float(x[0]) * a.scale),
+                                         __float_as_uint(__uint_as_float(x[1]) * a.scale),
+                                         __float_as_uint(__uint_as_float(x[2]) * a.scale),
+                                         __float_as_uint(__uint_as_float(x[3]) * a.scale));
+                        }
                     }
                 }
                 fence_proxy_async_smem();  // generic-proxy staging writes -> TMA reads
@@ -388,20 +392,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after();
             // key kv0 + col is attended when col <= lim (causal inside the diagonal block)
             const int lim = valid ? t - kv0 - h * HALF : -1;
+            const uint64_t sl2 = f2_pack(a.scale_log2, a.scale_log2), nl2 = f2_pack(-lse2, -lse2),
+                           nD = f2_pack(-Dt, -Dt);
 #pragma unroll
             for (int c = 0; c < HALF / 32; ++c) {
                 uint32_t sraw[32], draw[32];
                 tmem_ld32_async(tS + lane_off + h * HALF + 32 * c, sraw);
                 tmem_ld32_async(tdP + lane_off + h * HALF + 32 * c, draw);
                 tmem_ld_wait();
+                // masked scores become -inf (only warps holding a masked column pay for it)
+                if (!__all_sync(0xffffffffu, lim >= 32 * c + 31)) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (32 * c + i > lim) sraw[i] = 0xff800000u;
+                }
+                // p = 2^(s * scale_log2 - lse2), ds = p * (dp - D), in packed pairs
                 float sv[32], dp[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float p = (32 * c + i <= lim)
-                                        ? fast_exp2(fmaf(__uint_as_float(sraw[i]), a.scale_log2, -lse2))
-                                        : 0.f;
-                    sv[i] = p;
-                    dp[i] = p * (__uint_as_float(draw[i]) - Dt);
+                for (int i = 0; i < 32; i += 2) {
+                    float x0, x1;
+                    f2_unpack(ffma2(f2_pack(__uint_as_float(sraw[i]), __uint_as_float(sraw[i + 1])), sl2, nl2), x0, x1);
+                    sv[i] = fast_exp2(x0);
+                    sv[i + 1] = fast_exp2(x1);
+                    f2_unpack(fmul2(f2_pack(sv[i], sv[i + 1]),
+                                    fadd2(f2_pack(__uint_as_float(draw[i]), __uint_as_float(draw[i + 1])), nD)),
+                              dp[i], dp[i + 1]);
                 }
                 // full stream: the previous tile's dQ staged over P (and dS for 64-key units) has been read
                 if (!sparse && c == 0 && it > 0) ok = mbar_wait(bar_p_free, (it - 1) & 1, abort_flag, 0x30d);

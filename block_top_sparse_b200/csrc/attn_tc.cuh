@@ -281,14 +281,21 @@ __global__ void __launch_bounds__(kFullFwdThreads, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_ld32_async(tS + 32 * c, sr[c]);
             tmem_ld_wait();
-            // key n*128 + col is attended when col <= lim (causal on the diagonal tile)
+            // key n*128 + col is attended when col <= lim (causal on the diagonal tile); masked
+            // scores become -inf, on the diagonal tile only
             const int lim = (n == nkv - 1) ? t - n * kTileQ : 127;
+            if (n == nkv - 1) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (32 * c + i > lim) sr[c][i] = 0xff800000u;
+            }
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int c = 0; c < 4; ++c)
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    mx4[i & 3] = fmaxf(mx4[i & 3], (32 * c + i <= lim) ? __uint_as_float(sr[c][i]) : -INFINITY);
+                for (int i = 0; i < 32; ++i) mx4[i & 3] = fmaxf(mx4[i & 3], __uint_as_float(sr[c][i]));
             const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * scale_log2;
             float alpha = 1.f;
             if (n == 0) {
@@ -315,23 +322,29 @@ __global__ void __launch_bounds__(kFullFwdThreads, 1)
             l *= alpha;
             // probabilities -> P (bf16 pairs) in tensor memory, over the first 64 columns of S
             // (chunk c of S lands in packed columns 16c .. 16c+15; every S value is already in registers)
-            float l4[4] = {0.f, 0.f, 0.f, 0.f};
+            // p = 2^(s * scale_log2 - m) in packed pairs
+            const uint64_t sl2 = f2_pack(scale_log2, scale_log2), nm = f2_pack(-m_used, -m_used);
+            uint64_t l2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t pw[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
-                    const float p0 =
-                        (32 * c + i <= lim) ? fast_exp2(fmaf(__uint_as_float(sr[c][i]), scale_log2, -m_used)) : 0.f;
-                    const float p1 = (32 * c + i + 1 <= lim)
-                                         ? fast_exp2(fmaf(__uint_as_float(sr[c][i + 1]), scale_log2, -m_used))
-                                         : 0.f;
-                    l4[(i >> 1) & 3] += p0 + p1;
+                    float x0, x1;
+                    f2_unpack(ffma2(f2_pack(__uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1])), sl2, nm), x0,
+                              x1);
+                    const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                    l2[(i >> 1) & 1] = fadd2(l2[(i >> 1) & 1], f2_pack(p0, p1));
                     pw[i >> 1] = pack_bf16x2(p0, p1);
                 }
                 tmem_st16_u(tS + 16 * c, pw);
             }
-            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            {
+                float la, lb, lc, ld;
+                f2_unpack(l2[0], la, lb);
+                f2_unpack(l2[1], lc, ld);
+                l += (la + lb) + (lc + ld);
+            }
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(bar_p_full + x);

@@ -96,8 +96,9 @@ __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ K, floa
 //           l + 32 of the chunk for the warp's 4 queries;
 //   top-(k-1): the (k-1)-th largest order-preserving 32-bit key is built bit by
 //           bit from the most significant end (count of keys >= candidate by
-//           warp reduction); keys above it are kept, keys equal to it are kept
-//           in ascending block order until k-1 are chosen; a ballot compaction
+//           warp reduction), stopping early at a candidate with exactly k-1 keys
+//           at or above it; otherwise keys above it are kept, keys equal to it
+//           are kept in ascending block order until k-1 are chosen; a ballot compaction
 //           writes the chosen blocks in ascending order, then b(t), then -1.
 // ---------------------------------------------------------------------------
 constexpr int kSelQ = 32;
@@ -123,8 +124,12 @@ __device__ __forceinline__ void select_row(const float *row, int n, int want, in
         const int j = 32 * i + lane;
         key[i] = j < n ? order_key(row[j]) : 0u;  // 0 is below every real key
     }
+    // Invariant: at least `want` keys are >= tau.  A candidate with exactly `want`
+    // keys at or above it separates the top `want` from the rest: stop there
+    // (no key equal to the threshold is left out).
     uint32_t tau = 0u;
     int need_eq = 0;
+    bool exact = false;
     if (want > 0 && want < n) {
 #pragma unroll 1
         for (int b = 31; b >= 0; --b) {
@@ -132,12 +137,21 @@ __device__ __forceinline__ void select_row(const float *row, int n, int want, in
             unsigned c = 0;
 #pragma unroll
             for (int i = 0; i < KPL; ++i) c += key[i] >= cand ? 1u : 0u;
-            if (__reduce_add_sync(0xffffffffu, c) >= static_cast<unsigned>(want)) tau = cand;
+            const unsigned tot = __reduce_add_sync(0xffffffffu, c);
+            if (tot >= static_cast<unsigned>(want)) {
+                tau = cand;
+                if (tot == static_cast<unsigned>(want)) {
+                    exact = true;
+                    break;
+                }
+            }
         }
-        unsigned gt = 0;
+        if (!exact) {
+            unsigned gt = 0;
 #pragma unroll
-        for (int i = 0; i < KPL; ++i) gt += key[i] > tau ? 1u : 0u;
-        need_eq = want - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+            for (int i = 0; i < KPL; ++i) gt += key[i] > tau ? 1u : 0u;
+            need_eq = want - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+        }
     }
     int taken = 0, eq_seen = 0;
     if (want > 0) {
@@ -147,7 +161,9 @@ __device__ __forceinline__ void select_row(const float *row, int n, int want, in
             const bool in = 32 * i + lane < n;
             bool sel;
             uint32_t eqb = 0u;
-            if (want < n) {
+            if (want < n && exact) {
+                sel = in && key[i] >= tau;
+            } else if (want < n) {
                 const bool eq = in && key[i] == tau;
                 eqb = __ballot_sync(0xffffffffu, eq);
                 sel = (in && key[i] > tau) || (eq && (eq_seen + __popc(eqb & lt_mask)) < need_eq);
