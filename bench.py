@@ -245,6 +245,15 @@ def ours(args, rank, world, local_rank):
     # ---- per-op breakdown (separate, untimed-for-value pass) ----
     for i in range(max(2, min(args.steps, 4))):
         run_step(i, timed_ops=True)
+    # Pooling bandwidth from back-to-back launches: the events around the first call of a step
+    # also hold the host's launch latency.  K (268 MB) exceeds L2, so every launch streams it from HBM.
+    pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pa.record(stream)
+    for _ in range(10):
+        L.ssa_block_pool(steps[0].dims, d["K"], steps[0].Kbar)
+    pb.record(stream)
+    torch.cuda.synchronize(dev)
+    pool_kernel_ms = pa.elapsed_time(pb) / 10
 
     # ---- end to end: pinned host inputs -> device, step, loss back to host ----
     loss_host = torch.empty((), dtype=torch.float32).pin_memory()
@@ -281,10 +290,13 @@ def ours(args, rank, world, local_rank):
     full_ms = op_ms["full_fwd"] + op_ms["full_bwd"]
     op_flops = {"full_fwd": ff, "full_bwd": fb, "sparse_fwd": sf, "sparse_bwd": sb}
     dominant = max(op_ms, key=op_ms.get)
-    traffic = None
+    # DRAM bytes per launch of the dominant kernel from one ncu capture of the same build
+    # (profiles/attn_bwd_full_long_H4.md: the 4-head case, read 203.2 MB + write 96.0 MB; heads are
+    # independent units of the grid, so traffic scales by 32/4 to the benchmarked launch).
+    traffic = (203.203328e6 + 96.020736e6) * (wl.H / 4) if dominant == "full_bwd" else None
     roof = {"kernel": "ssa_%s call" % dominant, "bound": "tensor",
             "achieved": op_flops.get(dominant, 0.0) / (op_ms[dominant] / 1e3) / 1e12, "peak": peak_sust,
-            "unit": "TFLOP/s", "traffic": traffic,
+            "unit": "TFLOP/s", "traffic": traffic, "traffic_unit": "DRAM bytes per launch (ncu)",
             "peak_basis": "%s bf16 dense, sustained (kernel timed inside a long step)" % peak_kind}
     roof["frac"] = roof["achieved"] / roof["peak"]
     line = {
@@ -300,8 +312,9 @@ def ours(args, rank, world, local_rank):
         "op_ms": op_ms,
         "select_hbm": {"gbs": (wl.B * wl.H * wl.T * (2 * wl.d + 4 * K_SEL)) / (op_ms["select"] / 1e3) / 1e9,
                        "frac": (wl.B * wl.H * wl.T * (2 * wl.d + 4 * K_SEL)) / (op_ms["select"] / 1e3) / 1e9 / hbm},
-        "pool_hbm": {"gbs": (wl.B * wl.H * wl.T * 2 * wl.d) / (op_ms["pool"] / 1e3) / 1e9,
-                     "frac": (wl.B * wl.H * wl.T * 2 * wl.d) / (op_ms["pool"] / 1e3) / 1e9 / hbm},
+        "pool_hbm": {"gbs": (wl.B * wl.H * wl.T * 2 * wl.d) / (pool_kernel_ms / 1e3) / 1e9,
+                     "frac": (wl.B * wl.H * wl.T * 2 * wl.d) / (pool_kernel_ms / 1e3) / 1e9 / hbm,
+                     "ms": pool_kernel_ms, "timing": "mean of 10 back-to-back launches"},
         "roofline": roof,
         "e2e": {"value": tokens / (e_ms / args.steps / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(host[k].numel() * 2 for k in host), "d2h_bytes_per_step": 4},
@@ -378,7 +391,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-tokens", type=int, default=4096, help="prefix length of the oracle sample")
+    ap.add_argument("--ref-tokens", type=int, default=16384, help="prefix length of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", default=None,
                     choices=["pool", "select", "full_fwd", "sparse_fwd", "full_bwd", "sparse_bwd"],

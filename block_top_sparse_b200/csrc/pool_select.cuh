@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ K, floa
     float acc[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = 0.f;
-#pragma unroll 4
+#pragma unroll 8
     for (int r = g; r < s; r += G) {
         float f[V];
         Vec16<T>::load(base + static_cast<size_t>(r) * d, f);
