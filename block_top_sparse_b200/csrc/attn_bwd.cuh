@@ -84,6 +84,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint64_t *bar_qdo_free = bars + 4, *bar_dq_full = bars + 5, *bar_dq_empty = bars + 6, *bar_final = bars + 7;
     uint64_t *bar_f_staged = bars + 8, *bar_f_free = bars + 9;  // dQ staging buffer handshakes
     uint64_t *bar_p_free = bars + 12;  // the P region's dQ half has been read by the flush
+    uint64_t *bar_epi = bars + 13;     // the dV / dK staging of the epilogue is complete
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 11);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -127,6 +128,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // read shared memory (full: P region and staging buffer)
         mbar_init(bar_f_free, sparse ? 128 : 1);
         mbar_init(bar_p_free, 1);
+        mbar_init(bar_epi, 256);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -428,9 +430,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_before();
             mbar_arrive(bar_pds_full);
         }
-        // Epilogue: thread <-> head-dim row r of dV^T / dK^T, key columns of its half.
+        // Epilogue.  dV^T / dK^T (thread <-> head-dim row r, key columns of its half) are restaged in
+        // fp32 as [key][dim] rows over the idle operand buffers (dV over Q/dO, dK over K/V, NKV rows of
+        // 512 bytes each), then every warp writes whole 256-byte bf16 rows with 16-byte accesses, adding
+        // the existing gradient in fp32 first when asked (one rounding).
         if (ok && !mbar_wait(bar_final, 0, abort_flag, 0x30c)) ok = false;
         tc_fence_after();
+        const uint32_t sdv = sQ, sdk = sK;
         if (ok) {
 #pragma unroll
             for (int c0 = h * HALF; c0 < (h + 1) * HALF; c0 += 32) {
@@ -440,19 +446,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int kv = kv0 + c0 + i;
-                    if (kv < T) {
-                        const size_t off = (head_rows + kv) * kD + r;
-                        float vv = ntiles > 0 ? __uint_as_float(rv[i]) : 0.f;
-                        float kq = ntiles > 0 ? __uint_as_float(rk[i]) * a.scale : 0.f;
-                        if (a.accumulate) {
-                            vv += __bfloat162float(a.dV[off]);
-                            kq += __bfloat162float(a.dK[off]);
-                        }
-                        a.dV[off] = __float2bfloat16_rn(vv);
-                        a.dK[off] = __float2bfloat16_rn(kq);
-                    }
+                    const float vv = ntiles > 0 ? __uint_as_float(rv[i]) : 0.f;
+                    const float kq = ntiles > 0 ? __uint_as_float(rk[i]) * a.scale : 0.f;
+                    // a warp stores 32 consecutive dims of one key row: 128 contiguous bytes
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(sdv + (c0 + i) * 512 + r * 4), "f"(vv) : "memory");
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(sdk + (c0 + i) * 512 + r * 4), "f"(kq) : "memory");
                 }
+            }
+        }
+        mbar_arrive(bar_epi);
+        if (ok && !mbar_wait(bar_epi, 0, abort_flag, 0x30e)) ok = false;
+        if (ok) {
+            // warp w writes key rows w, w+8, ...: lane l the dims 4l .. 4l+3 of both gradients
+            for (int kr = warp; kr < NKV; kr += 8) {
+                if (kv0 + kr >= T) break;
+                float4 v4, k4;
+                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(v4.x), "=f"(v4.y), "=f"(v4.z), "=f"(v4.w)
+                             : "r"(sdv + kr * 512 + lane * 16));
+                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(k4.x), "=f"(k4.y), "=f"(k4.z), "=f"(k4.w)
+                             : "r"(sdk + kr * 512 + lane * 16));
+                const size_t off = (head_rows + kv0 + kr) * kD + 4 * lane;
+                uint2 *dv2 = reinterpret_cast<uint2 *>(a.dV + off);
+                uint2 *dk2 = reinterpret_cast<uint2 *>(a.dK + off);
+                if (a.accumulate) {
+                    const uint2 ov = *dv2, ok2 = *dk2;
+                    v4.x += __uint_as_float(ov.x << 16);
+                    v4.y += __uint_as_float(ov.x & 0xFFFF0000u);
+                    v4.z += __uint_as_float(ov.y << 16);
+                    v4.w += __uint_as_float(ov.y & 0xFFFF0000u);
+                    k4.x += __uint_as_float(ok2.x << 16);
+                    k4.y += __uint_as_float(ok2.x & 0xFFFF0000u);
+                    k4.z += __uint_as_float(ok2.y << 16);
+                    k4.w += __uint_as_float(ok2.y & 0xFFFF0000u);
+                }
+                *dv2 = make_uint2(pack_bf16x2(v4.x, v4.y), pack_bf16x2(v4.z, v4.w));
+                *dk2 = make_uint2(pack_bf16x2(k4.x, k4.y), pack_bf16x2(k4.z, k4.w));
             }
         }
     }
