@@ -59,7 +59,7 @@ def _load():
     lib.ora_check_selection.argtypes = [i64, i64, i64, i64, p]
     lib.ora_check_selection.restype = ctypes.c_int
     lib.ora_attn_fwd.argtypes = [i64, i64, i64, i64, i64, dbl, p, p, p, p, i64, p, p, p]
-    lib.ora_attn_bwd.argtypes = [i64, i64, i64, i64, i64, dbl, p, p, p, p, p, i64, p, i64, p, p, p, p]
+    lib.ora_attn_bwd.argtypes = [i64, i64, i64, i64, i64, dbl, p, p, p, p, p, i64, p, i64, p, p, p, p, ctypes.c_int]
     lib.ora_align_fwd.argtypes = [i64, p, p, dbl, dbl, dbl]
     lib.ora_align_fwd.restype = dbl
     lib.ora_align_bwd.argtypes = [i64, p, p, dbl, dbl, dbl, dbl, p, p]
@@ -125,8 +125,12 @@ def attn_fwd(Q, K, V, s: int, scale: float, idx: Optional[np.ndarray] = None, ro
     return O, lse
 
 
-def attn_bwd(Q, K, V, dO, s: int, scale: float, idx: Optional[np.ndarray] = None, qrows=None, krows=None):
-    """Gradients of sum(dO * O) -> (dQ [BH, nq, d], dK [BH, nk, d], dV [BH, nk, d])."""
+def attn_bwd(Q, K, V, dO, s: int, scale: float, idx: Optional[np.ndarray] = None, qrows=None, krows=None,
+             stored_o: str = "exact"):
+    """Gradients of sum(dO * O) -> (dQ [BH, nq, d], dK [BH, nk, d], dV [BH, nk, d]).
+
+    stored_o="bf16": D_t = dO_t . o_t is formed with the oracle's own output rounded to bfloat16, the value
+    a backward pass is given when the forward stores its output in bfloat16; "exact" uses o_t itself."""
     Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
     BH, T, d = Q.shape
     k = 0 if idx is None else idx.shape[-1]
@@ -139,7 +143,8 @@ def attn_bwd(Q, K, V, dO, s: int, scale: float, idx: Optional[np.ndarray] = None
     dK = np.empty((BH, nk, d), dtype=np.float64)
     dV = np.empty((BH, nk, d), dtype=np.float64)
     _load().ora_attn_bwd(BH, T, d, s, k, float(scale), _ptr(Q), _ptr(K), _ptr(V), _ptr(dO), _ptr(idx),
-                         nq, _ptr(qrows), nk, _ptr(krows), _ptr(dQ), _ptr(dK), _ptr(dV))
+                         nq, _ptr(qrows), nk, _ptr(krows), _ptr(dQ), _ptr(dK), _ptr(dV),
+                         1 if stored_o == "bf16" else 0)
     return dQ, dK, dV
 
 

@@ -218,9 +218,20 @@ void ora_attn_fwd(i64 BH, i64 T, i64 d, i64 s, i64 k, double scale, const double
  * Computes dQ for query rows qrows[0..nq) and dK, dV for key rows krows[0..nk)
  * (NULL: all rows); outputs are [BH, nq, d] and [BH, nk, d].
  * ------------------------------------------------------------------------- */
+/* x rounded to the nearest bfloat16 value (8 significant bits, ties to even), as a forward output
+ * stored in bfloat16 holds it. */
+static double round_bf16(double x) {
+    if (x == 0.0 || !isfinite(x)) return x;
+    int e;
+    const double m = frexp(x, &e);            /* x = m * 2^e, 0.5 <= |m| < 1 */
+    return ldexp(nearbyint(ldexp(m, 8)), e - 8); /* default rounding mode: to nearest, ties to even */
+}
+
+/* round_o != 0: D_t = dO_t . o_t uses o_t rounded to bfloat16 -- the value a backward pass receives
+ * when the forward stores its output in bfloat16 (the backward takes the stored output as input). */
 void ora_attn_bwd(i64 BH, i64 T, i64 d, i64 s, i64 k, double scale, const double *Q, const double *K,
                   const double *V, const double *dO, const int32_t *idx, i64 nq, const i64 *qrows, i64 nk,
-                  const i64 *krows, double *dQ, double *dK, double *dV) {
+                  const i64 *krows, double *dQ, double *dK, double *dV, int round_o) {
     i64 nQ = qrows ? nq : T, nK = krows ? nk : T;
     double *lse = (double *)malloc(sizeof(double) * (size_t)(BH * T));
     double *Dt = (double *)malloc(sizeof(double) * (size_t)(BH * T));
@@ -243,7 +254,7 @@ void ora_attn_bwd(i64 BH, i64 T, i64 d, i64 s, i64 k, double scale, const double
                 lse[bh * T + t] =
                     attend_row(d, s, k, scale, Q + bh * T * d, K + bh * T * d, V + bh * T * d, sel_row, t, o, pos);
                 double acc = 0.0;
-                for (i64 c = 0; c < d; ++c) acc += dO[(bh * T + t) * d + c] * o[c];
+                for (i64 c = 0; c < d; ++c) acc += dO[(bh * T + t) * d + c] * (round_o ? round_bf16(o[c]) : o[c]);
                 Dt[bh * T + t] = acc;
             }
         }

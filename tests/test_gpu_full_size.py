@@ -98,8 +98,9 @@ def _run(wlname, k, heads, n_rows, backward, main="full"):
             # The main stream's backward with the seeded dO.  The other stream receives only the
             # alignment slope, |dL/do| <= max(w) / (B*H*T*d) ~ 1e-8 here, far below the tolerance,
             # so the oracle leaves it out.
+            # the backward is given the forward's output as stored (bf16): D = dO . bf16(o)
             a = ora.attn_bwd(f["Q"], f["K"], f["V"], f["dO"], s, dims.scale,
-                             idx_ref if main == "sparse" else None, rows, rows)
+                             idx_ref if main == "sparse" else None, rows, rows, stored_o="bf16")
             for nm, got, ref in zip(("dQ", "dK", "dV"), (step.dQ, step.dK, step.dV), a):
                 check_close("%s.h%d.%s" % (wlname, bh, nm), _pick(got, B, H, T, bh, rows), ref, True)
     return report

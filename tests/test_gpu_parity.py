@@ -68,7 +68,8 @@ def _attn_check(w, dims, f, dev, idx_ref, tag):
     check_close(tag + ".O", to_np(O).reshape(BH, w.T, w.d), O_ref, bf16)
     np.testing.assert_allclose(to_np(lse).reshape(BH, w.T), lse_ref, rtol=0, atol=2e-3)
     dQ, dK, dV = ops.attn_bwd(dims, dev["Q"], dev["K"], dev["V"], O, lse, dev["dO"], idx_dev)
-    gref = ora.attn_bwd(f["Q"], f["K"], f["V"], f["dO"], w.s, scale, idx_ref)
+    # the backward is given the forward's output as stored: D = dO . o with o in the output dtype
+    gref = ora.attn_bwd(f["Q"], f["K"], f["V"], f["dO"], w.s, scale, idx_ref, stored_o="bf16" if bf16 else "exact")
     for nm, g, r in zip(("dQ", "dK", "dV"), (dQ, dK, dV), gref):
         check_close(tag + "." + nm, to_np(g).reshape(BH, w.T, w.d), r, bf16)
     assert L.ssa_get_device_error() == L.SSA_OK
@@ -172,8 +173,8 @@ def test_step_both_streams_matches_oracle():
         gf, gs = ora.align_bwd(Of_ref, Os_ref)
         dOf = f["dO"] + gf if main == "full" else gf
         dOs = f["dO"] + gs if main == "sparse" else gs
-        g_full = ora.attn_bwd(f["Q"], f["K"], f["V"], dOf, s, scale)
-        g_sparse = ora.attn_bwd(f["Q"], f["K"], f["V"], dOs, s, scale, idx_ref)
+        g_full = ora.attn_bwd(f["Q"], f["K"], f["V"], dOf, s, scale, stored_o="bf16")
+        g_sparse = ora.attn_bwd(f["Q"], f["K"], f["V"], dOs, s, scale, idx_ref, stored_o="bf16")
         if rep["differ"] == 0:
             for nm, g, a, b in zip(("dQ", "dK", "dV"), (step.dQ, step.dK, step.dV), g_full, g_sparse):
                 check_close("step.%s.%s" % (main, nm), to_np(g).reshape(a.shape), a + b, True)

@@ -393,3 +393,25 @@ def test_planted_blocks_are_found(ora):
     pool_mean = np.array([sc[tt, :b].mean() for tt, b in zip(t, bt)]).mean()
     pool_std = np.array([sc[tt, :b].std() for tt, b in zip(t, bt)]).mean()
     assert chosen > pool_mean + 1.5 * pool_std
+
+
+def test_bwd_with_stored_bf16_output_matches_dense_formulas(ora):
+    # The backward given the forward's output as stored in bfloat16: D_t = dO_t . bf16(o_t), the rest of the
+    # gradient formulas unchanged.  Dense numpy formulas with torch's bfloat16 rounding as the pin.
+    T, d, s, scale = 16, 4, 4, 0.5
+    Q, K, V, dO = (_rand((1, T, d), i) for i in (40, 41, 42, 43))
+    q, k, v, g = Q[0], K[0], V[0], dO[0]
+    S = scale * q @ k.T
+    S[np.triu_indices(T, 1)] = -np.inf
+    P = np.exp(S - S.max(axis=1, keepdims=True))
+    P /= P.sum(axis=1, keepdims=True)
+    o_b = torch.from_numpy(P @ v).to(torch.bfloat16).double().numpy()
+    D = (g * o_b).sum(axis=1, keepdims=True)
+    dS = P * (g @ v.T - D)
+    want = (scale * dS @ k, scale * dS.T @ q, P.T @ g)
+    got = ora.attn_bwd(Q, K, V, dO, s, scale, stored_o="bf16")
+    exact = ora.attn_bwd(Q, K, V, dO, s, scale)
+    for gg, w in zip(got, want):
+        np.testing.assert_allclose(gg[0], w, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got[2], exact[2], rtol=0, atol=1e-12)  # dV does not involve D
+    assert np.abs(got[0] - exact[0]).max() > 0  # the rounding is visible in dQ
