@@ -243,4 +243,145 @@ __global__ void __launch_bounds__(256) select_kernel(const T *__restrict__ Q, co
     }
 }
 
+// ---------------------------------------------------------------------------
+// Selection with the block scores on the tensor cores (bf16 Q, d = 128, nb <= 256).
+// One CTA (256 threads) per 128 consecutive queries of one head:
+//   scores: r[q][j] = q . Kbar_j as one dense contraction S = Q Kbar^T (M = 128 queries,
+//           N = 64 blocks per group, K = d) in tensor memory.  Kbar (fp32) is split into
+//           three bf16 terms, hi = bf16(x), mid = bf16(x - hi), lo = bf16(x - hi - mid),
+//           which carry its 24 significant bits; the products with the bf16 query are
+//           exact and the three contractions accumulate in fp32;
+//   top-(k-1): the scores are staged row-major in shared memory and each warp runs the
+//           threshold search of select_row on 16 of the 128 rows.
+// ---------------------------------------------------------------------------
+constexpr int kSelTcRows = 128;
+constexpr int kSelTcMaxBlocks = 256;
+constexpr int kSelTcPitch = kSelTcMaxBlocks + 4;  // fp32 score row pitch: conflict-free staging
+
+struct SelTcSmem {
+    static constexpr int kQ = 0;                      // 128 rows x 128 bf16: 2 swizzled 16 KB chunks
+    static constexpr int kB = 2 * 16384;              // hi / mid / lo: 3 x (64 blocks x 128 bf16), 16 KB each
+    static constexpr int kS = kB + 3 * 16384;         // 128 x kSelTcPitch fp32 scores
+    static constexpr int kBar = kS + kSelTcRows * kSelTcPitch * 4;
+    static constexpr int kTotal = kBar + 64;
+};
+
+__device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b) {
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
+
+__global__ void __launch_bounds__(256, 1) select_tc_kernel(const __nv_bfloat16 *__restrict__ Q,
+                                                           const float *__restrict__ Kbar, int32_t *__restrict__ idx,
+                                                           int T_len, int s, int k, int nb) {
+    using L = SelTcSmem;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bar_mma = reinterpret_cast<uint64_t *>(smem + L::kBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBar + 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kBar + 16);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.y, t0 = blockIdx.x * kSelTcRows;
+    const size_t head_rows = static_cast<size_t>(bh) * T_len;
+    const int last = min(t0 + kSelTcRows, T_len) - 1;
+    const int nbc = min(last / s, nb);  // blocks scored by some row of the tile (j < b(t))
+    const int ngroups = (nbc + 63) / 64;
+    const uint32_t sQ = smem_u32(smem + L::kQ), sB = smem_u32(smem + L::kB);
+    float *sS = reinterpret_cast<float *>(smem + L::kS);
+
+    if (tid == 0) {
+        mbar_init(bar_mma, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    {
+        // query rows -> K-major 128-byte-swizzled tile; rows past T are zero-filled
+        const int u = tid & 15;
+        for (int row = tid >> 4; row < kSelTcRows; row += 16) {
+            const int t = t0 + row;
+            const bool valid = t < T_len;
+            const uint32_t dst = sQ + (u >> 3) * 16384 + row * 128 + ((((u & 7) ^ (row & 7)) & 7) << 4);
+            cp_async_16(dst, Q + (head_rows + (valid ? t : 0)) * 128 + u * 8, valid ? 16u : 0u);
+        }
+        cp_async_wait_all();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+    for (int gi = 0; gi < ngroups; ++gi) {
+        // Kbar rows 64gi .. 64gi+63 -> hi / mid / lo tiles (K-major, swizzled); rows >= nbc are zero.
+        // Lane c4 of a warp takes dims 4c4 .. 4c4+3 of one row: two 128-byte row halves per store.
+        const int c4 = lane;
+        for (int jj = warp; jj < 64; jj += 8) {
+            const int j = 64 * gi + jj;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (j < nbc) v = __ldg(reinterpret_cast<const float4 *>(Kbar + (static_cast<size_t>(bh) * nb + j) * 128) + c4);
+            const uint32_t h01 = pack_bf16x2(v.x, v.y), h23 = pack_bf16x2(v.z, v.w);
+            const float r0 = v.x - __uint_as_float(h01 << 16), r1 = v.y - __uint_as_float(h01 & 0xFFFF0000u);
+            const float r2 = v.z - __uint_as_float(h23 << 16), r3 = v.w - __uint_as_float(h23 & 0xFFFF0000u);
+            const uint32_t m01 = pack_bf16x2(r0, r1), m23 = pack_bf16x2(r2, r3);
+            const uint32_t l01 = pack_bf16x2(r0 - __uint_as_float(m01 << 16), r1 - __uint_as_float(m01 & 0xFFFF0000u));
+            const uint32_t l23 = pack_bf16x2(r2 - __uint_as_float(m23 << 16), r3 - __uint_as_float(m23 & 0xFFFF0000u));
+            const uint32_t off = (c4 >> 4) * 8192 + jj * 128 + (((((c4 & 15) >> 1) ^ (jj & 7)) & 7) << 4) + (c4 & 1) * 8;
+            st_shared_v2(sB + off, h01, h23);
+            st_shared_v2(sB + 16384 + off, m01, m23);
+            st_shared_v2(sB + 2 * 16384 + off, l01, l23);
+        }
+        fence_proxy_async_smem();  // generic-proxy tile writes -> tensor-core reads
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int sp = 0; sp < 3; ++sp)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ss(tmem + 64 * gi, smem_desc_sw128(sQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
+                                smem_desc_sw128(sB + sp * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32, 16), id,
+                                (sp > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(bar_mma);
+        }
+        // the next group rewrites the split tiles only after these MMAs have read them
+        if (!mbar_wait(bar_mma, gi & 1, abort_flag, 0x501)) {
+            ok = false;
+            break;
+        }
+    }
+    tc_fence_after();
+    // scores -> shared memory: warps 0-3, thread <-> row (tensor-memory lane)
+    if (ok && warp < 4) {
+        const int row = warp * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t dst = smem_u32(sS + row * kSelTcPitch);
+        for (int gi = 0; gi < ngroups; ++gi) {
+            uint32_t v[2][32];
+            tmem_ld32_async(tmem + lane_off + 64 * gi, v[0]);
+            tmem_ld32_async(tmem + lane_off + 64 * gi + 32, v[1]);
+            tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const uint32_t *x = v[q >> 3] + 4 * (q & 7);
+                st_shared_v4(dst + (64 * gi + 4 * q) * 4, x[0], x[1], x[2], x[3]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+    // top-(k-1) per row: warp w takes rows w, w+8, ...
+    for (int row = warp; row < kSelTcRows; row += 8) {
+        const int t = t0 + row;
+        if (t >= T_len) break;
+        const int bt = t / s;
+        select_row<8>(sS + row * kSelTcPitch, bt, min(k - 1, bt), bt, k, idx + (head_rows + t) * k, lane);
+    }
+}
+
 }  // namespace ssa

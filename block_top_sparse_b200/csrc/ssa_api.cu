@@ -340,6 +340,14 @@ ssa_status_t ssa_block_select(const ssa_dims_t *dims, const void *Q, const float
     const size_t sm = select_smem_bytes(S.d, S.nb);
     if (S.nb > 1024 || sm > 227 * 1024) return SSA_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (S.tc && S.nb <= kSelTcMaxBlocks) {
+        // scores on the tensor cores
+        const size_t smt = SelTcSmem::kTotal + 1024;
+        if (!set_smem(select_tc_kernel, smt)) return SSA_ERR_CUDA;
+        select_tc_kernel<<<dim3((S.T + kSelTcRows - 1) / kSelTcRows, S.BH), 256, smt, st>>>(
+            (const __nv_bfloat16 *)Q, Kbar, idx, S.T, S.s, S.k, S.nb);
+        return launch_status();
+    }
     if (S.dtype == SSA_DT_BF16) {
         if (S.nb <= 256)
             e = launch_select<__nv_bfloat16, 8>(S, Q, Kbar, idx, sm, st);
