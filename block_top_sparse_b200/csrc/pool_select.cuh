@@ -245,16 +245,19 @@ __global__ void __launch_bounds__(256) select_kernel(const T *__restrict__ Q, co
 
 // ---------------------------------------------------------------------------
 // Selection with the block scores on the tensor cores (bf16 Q, d = 128, nb <= 256).
-// One CTA (256 threads) per 128 consecutive queries of one head:
+// One CTA (512 threads) per 128 consecutive queries of one head:
 //   scores: r[q][j] = q . Kbar_j as one dense contraction S = Q Kbar^T (M = 128 queries,
 //           N = 64 blocks per group, K = d) in tensor memory.  Kbar (fp32) is split into
 //           three bf16 terms, hi = bf16(x), mid = bf16(x - hi), lo = bf16(x - hi - mid),
 //           which carry its 24 significant bits; the products with the bf16 query are
 //           exact and the three contractions accumulate in fp32;
-//   top-(k-1): the scores are staged row-major in shared memory and each warp runs the
-//           threshold search of select_row on 16 of the 128 rows.
+//   top-(k-1): the scores are staged row-major in shared memory and each of the 16 warps runs
+//           the threshold search of select_row on 8 of the 128 rows (a search is a chain of
+//           dependent warp reductions, so many rows are kept in flight).
 // ---------------------------------------------------------------------------
 constexpr int kSelTcRows = 128;
+constexpr int kSelTcThreads = 512;
+constexpr int kSelTcWarps = kSelTcThreads / 32;
 constexpr int kSelTcMaxBlocks = 256;
 constexpr int kSelTcPitch = kSelTcMaxBlocks + 4;  // fp32 score row pitch: conflict-free staging
 
@@ -270,7 +273,7 @@ __device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t
     asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
 
-__global__ void __launch_bounds__(256, 1) select_tc_kernel(const __nv_bfloat16 *__restrict__ Q,
+__global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_bfloat16 *__restrict__ Q,
                                                            const float *__restrict__ Kbar, int32_t *__restrict__ idx,
                                                            int T_len, int s, int k, int nb) {
     using L = SelTcSmem;
@@ -300,7 +303,7 @@ __global__ void __launch_bounds__(256, 1) select_tc_kernel(const __nv_bfloat16 *
     {
         // query rows -> K-major 128-byte-swizzled tile; rows past T are zero-filled
         const int u = tid & 15;
-        for (int row = tid >> 4; row < kSelTcRows; row += 16) {
+        for (int row = tid >> 4; row < kSelTcRows; row += kSelTcThreads / 16) {
             const int t = t0 + row;
             const bool valid = t < T_len;
             const uint32_t dst = sQ + (u >> 3) * 16384 + row * 128 + ((((u & 7) ^ (row & 7)) & 7) << 4);
@@ -318,7 +321,7 @@ __global__ void __launch_bounds__(256, 1) select_tc_kernel(const __nv_bfloat16 *
         // Kbar rows 64gi .. 64gi+63 -> hi / mid / lo tiles (K-major, swizzled); rows >= nbc are zero.
         // Lane c4 of a warp takes dims 4c4 .. 4c4+3 of one row: two 128-byte row halves per store.
         const int c4 = lane;
-        for (int jj = warp; jj < 64; jj += 8) {
+        for (int jj = warp; jj < 64; jj += kSelTcWarps) {
             const int j = 64 * gi + jj;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
             if (j < nbc) v = __ldg(reinterpret_cast<const float4 *>(Kbar + (static_cast<size_t>(bh) * nb + j) * 128) + c4);
@@ -359,24 +362,20 @@ __global__ void __launch_bounds__(256, 1) select_tc_kernel(const __nv_bfloat16 *
         const int row = warp * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
         const uint32_t dst = smem_u32(sS + row * kSelTcPitch);
-        for (int gi = 0; gi < ngroups; ++gi) {
-            uint32_t v[2][32];
-            tmem_ld32_async(tmem + lane_off + 64 * gi, v[0]);
-            tmem_ld32_async(tmem + lane_off + 64 * gi + 32, v[1]);
+        for (int c = 0; c < 2 * ngroups; ++c) {
+            uint32_t v[32];
+            tmem_ld32_async(tmem + lane_off + 32 * c, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const uint32_t *x = v[q >> 3] + 4 * (q & 7);
-                st_shared_v4(dst + (64 * gi + 4 * q) * 4, x[0], x[1], x[2], x[3]);
-            }
+            for (int q = 0; q < 8; ++q) st_shared_v4(dst + (32 * c + 4 * q) * 4, v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, 256);
-    // top-(k-1) per row: warp w takes rows w, w+8, ...
-    for (int row = warp; row < kSelTcRows; row += 8) {
+    // top-(k-1) per row: warp w takes rows w, w + 16, ...
+    for (int row = warp; row < kSelTcRows; row += kSelTcWarps) {
         const int t = t0 + row;
         if (t >= T_len) break;
         const int bt = t / s;

@@ -344,7 +344,7 @@ ssa_status_t ssa_block_select(const ssa_dims_t *dims, const void *Q, const float
         // scores on the tensor cores
         const size_t smt = SelTcSmem::kTotal + 1024;
         if (!set_smem(select_tc_kernel, smt)) return SSA_ERR_CUDA;
-        select_tc_kernel<<<dim3((S.T + kSelTcRows - 1) / kSelTcRows, S.BH), 256, smt, st>>>(
+        select_tc_kernel<<<dim3((S.T + kSelTcRows - 1) / kSelTcRows, S.BH), kSelTcThreads, smt, st>>>(
             (const __nv_bfloat16 *)Q, Kbar, idx, S.T, S.s, S.k, S.nb);
         return launch_status();
     }
