@@ -115,44 +115,61 @@ __device__ __forceinline__ uint32_t order_key(float x) {
 }
 
 // Top-(want) of row[0..n) for one warp; KPL keys per lane (n <= 32*KPL).
+// Invariant of the search: at least `want` keys are >= tau.  A candidate with exactly
+// `want` keys at or above it separates the top `want` from the rest: stop there (no key
+// equal to the threshold is left out); otherwise tau ends as the want-th largest key and
+// need_eq of the keys equal to it are taken in ascending block order.
+struct SelSearch {
+    uint32_t tau = 0u;
+    int need_eq = 0;
+    bool exact = false;
+    bool done = true;
+};
+
 template <int KPL>
-__device__ __forceinline__ void select_row(const float *row, int n, int want, int bt, int k, int32_t *out, int lane) {
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    uint32_t key[KPL];
+__device__ __forceinline__ void select_load(const float *row, int n, uint32_t (&key)[KPL], int lane) {
 #pragma unroll
     for (int i = 0; i < KPL; ++i) {
         const int j = 32 * i + lane;
         key[i] = j < n ? order_key(row[j]) : 0u;  // 0 is below every real key
     }
-    // Invariant: at least `want` keys are >= tau.  A candidate with exactly `want`
-    // keys at or above it separates the top `want` from the rest: stop there
-    // (no key equal to the threshold is left out).
-    uint32_t tau = 0u;
-    int need_eq = 0;
-    bool exact = false;
-    if (want > 0 && want < n) {
-#pragma unroll 1
-        for (int b = 31; b >= 0; --b) {
-            const uint32_t cand = tau | (1u << b);
-            unsigned c = 0;
+}
+
+template <int KPL>
+__device__ __forceinline__ unsigned select_count(const uint32_t (&key)[KPL], uint32_t cand) {
+    unsigned c = 0;
 #pragma unroll
-            for (int i = 0; i < KPL; ++i) c += key[i] >= cand ? 1u : 0u;
-            const unsigned tot = __reduce_add_sync(0xffffffffu, c);
-            if (tot >= static_cast<unsigned>(want)) {
-                tau = cand;
-                if (tot == static_cast<unsigned>(want)) {
-                    exact = true;
-                    break;
-                }
-            }
-        }
-        if (!exact) {
-            unsigned gt = 0;
-#pragma unroll
-            for (int i = 0; i < KPL; ++i) gt += key[i] > tau ? 1u : 0u;
-            need_eq = want - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+    for (int i = 0; i < KPL; ++i) c += key[i] >= cand ? 1u : 0u;
+    return __reduce_add_sync(0xffffffffu, c);
+}
+
+// One step (bit b) of the search; a finished search is left unchanged.
+__device__ __forceinline__ void select_step(SelSearch &st, int want, int b, unsigned tot) {
+    if (st.done) return;
+    if (tot >= static_cast<unsigned>(want)) {
+        st.tau |= 1u << b;
+        if (tot == static_cast<unsigned>(want)) {
+            st.exact = true;
+            st.done = true;
         }
     }
+}
+
+template <int KPL>
+__device__ __forceinline__ void select_finish(const uint32_t (&key)[KPL], SelSearch &st, int want, int n) {
+    if (want > 0 && want < n && !st.exact) {
+        unsigned gt = 0;
+#pragma unroll
+        for (int i = 0; i < KPL; ++i) gt += key[i] > st.tau ? 1u : 0u;
+        st.need_eq = want - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+    }
+}
+
+// Writes the chosen blocks ascending, then b(t), then -1 padding up to k.
+template <int KPL>
+__device__ __forceinline__ void select_emit(const uint32_t (&key)[KPL], const SelSearch &st, int n, int want, int bt,
+                                            int k, int32_t *out, int lane) {
+    const uint32_t lt_mask = (1u << lane) - 1u;
     int taken = 0, eq_seen = 0;
     if (want > 0) {
 #pragma unroll
@@ -161,12 +178,12 @@ __device__ __forceinline__ void select_row(const float *row, int n, int want, in
             const bool in = 32 * i + lane < n;
             bool sel;
             uint32_t eqb = 0u;
-            if (want < n && exact) {
-                sel = in && key[i] >= tau;
+            if (want < n && st.exact) {
+                sel = in && key[i] >= st.tau;
             } else if (want < n) {
-                const bool eq = in && key[i] == tau;
+                const bool eq = in && key[i] == st.tau;
                 eqb = __ballot_sync(0xffffffffu, eq);
-                sel = (in && key[i] > tau) || (eq && (eq_seen + __popc(eqb & lt_mask)) < need_eq);
+                sel = (in && key[i] > st.tau) || (eq && (eq_seen + __popc(eqb & lt_mask)) < st.need_eq);
             } else {
                 sel = in;
             }
@@ -178,6 +195,42 @@ __device__ __forceinline__ void select_row(const float *row, int n, int want, in
         }
     }
     for (int i = want + lane; i < k; i += 32) out[i] = (i == want) ? bt : -1;
+}
+
+template <int KPL>
+__device__ __forceinline__ void select_row(const float *row, int n, int want, int bt, int k, int32_t *out, int lane) {
+    uint32_t key[KPL];
+    select_load<KPL>(row, n, key, lane);
+    SelSearch st;
+    st.done = !(want > 0 && want < n);
+#pragma unroll 1
+    for (int b = 31; b >= 0 && !st.done; --b) select_step(st, want, b, select_count<KPL>(key, st.tau | (1u << b)));
+    select_finish<KPL>(key, st, want, n);
+    select_emit<KPL>(key, st, n, want, bt, k, out, lane);
+}
+
+// Two rows' searches interleaved in one warp: their chains of dependent warp reductions overlap.
+template <int KPL>
+__device__ __forceinline__ void select_row2(const float *rowA, int nA, int wantA, int btA, int32_t *outA,
+                                            const float *rowB, int nB, int wantB, int btB, int32_t *outB, int k,
+                                            int lane) {
+    uint32_t ka[KPL], kb[KPL];
+    select_load<KPL>(rowA, nA, ka, lane);
+    select_load<KPL>(rowB, nB, kb, lane);
+    SelSearch sa, sb;
+    sa.done = !(wantA > 0 && wantA < nA);
+    sb.done = !(wantB > 0 && wantB < nB);
+#pragma unroll 1
+    for (int b = 31; b >= 0 && !(sa.done && sb.done); --b) {
+        const unsigned ta = select_count<KPL>(ka, sa.tau | (1u << b));
+        const unsigned tb = select_count<KPL>(kb, sb.tau | (1u << b));
+        select_step(sa, wantA, b, ta);
+        select_step(sb, wantB, b, tb);
+    }
+    select_finish<KPL>(ka, sa, wantA, nA);
+    select_finish<KPL>(kb, sb, wantB, nB);
+    if (outA) select_emit<KPL>(ka, sa, nA, wantA, btA, k, outA, lane);
+    if (outB) select_emit<KPL>(kb, sb, nB, wantB, btB, k, outB, lane);
 }
 
 template <typename T, int KPL>
@@ -374,12 +427,15 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
     __syncthreads();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, 256);
-    // top-(k-1) per row: warp w takes rows w, w + 16, ...
-    for (int row = warp; row < kSelTcRows; row += kSelTcWarps) {
-        const int t = t0 + row;
-        if (t >= T_len) break;
-        const int bt = t / s;
-        select_row<8>(sS + row * kSelTcPitch, bt, min(k - 1, bt), bt, k, idx + (head_rows + t) * k, lane);
+    // top-(k-1) per row: warp w takes rows w, w + 16, ..., two at a time (rows past T write nothing)
+    for (int row = warp; row < kSelTcRows; row += 2 * kSelTcWarps) {
+        const int ta = t0 + row, tb = t0 + row + kSelTcWarps;
+        const int bta = ta / s, btb = tb / s;
+        const bool va = ta < T_len, vb = tb < T_len;
+        select_row2<8>(sS + row * kSelTcPitch, va ? bta : 0, va ? min(k - 1, bta) : 0, bta,
+                       va ? idx + (head_rows + ta) * k : nullptr, sS + (row + kSelTcWarps) * kSelTcPitch,
+                       vb ? btb : 0, vb ? min(k - 1, btb) : 0, btb, vb ? idx + (head_rows + tb) * k : nullptr, k,
+                       lane);
     }
 }
 
