@@ -85,6 +85,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint64_t *bar_f_staged = bars + 8, *bar_f_free = bars + 9;  // dQ staging buffer handshakes
     uint64_t *bar_p_free = bars + 12;  // the P region's dQ half has been read by the flush
     uint64_t *bar_epi = bars + 13;     // the dV / dK staging of the epilogue is complete
+    // full stream: dO has its own load / release barriers (released after the dV MMAs, before
+    // Q, which the dK MMAs still read); the sparse gather brings Q and dO together on bar_qdo_full
+    uint64_t *bar_do_full = bars + 14, *bar_do_free = bars + 15;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 11);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -119,6 +122,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(bar_sdp_full, 1);
         mbar_init(bar_pds_full, 256);
         mbar_init(bar_qdo_free, 1);
+        mbar_init(bar_do_full, 1);
+        mbar_init(bar_do_free, 1);
         mbar_init(bar_dq_full, 1);
         mbar_init(bar_dq_empty, 128);
         mbar_init(bar_final, 1);
@@ -190,17 +195,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tma_load_2d(&tmV, bar_kv, smem + L::kV, 0, krow);
                 tma_load_2d(&tmV, bar_kv, smem + L::kV + NKV * 128, 64, krow);
                 if (!sparse) {
+                    int do_issued = 0, q_issued = 0;
                     for (int it = 0; it < ntiles; ++it) {
-                        if (it > 0 && !mbar_wait(bar_qdo_free, (it - 1) & 1, abort_flag, 0x311)) break;
                         const int qrow = static_cast<int>(head_rows) + kv0 + it * kTileQ;
-                        mbar_arrive_expect_tx(bar_qdo_full, 4 * kChunkBytes);
+                        // dO of tile it once the dV MMAs of tile it-1 have read dO
+                        if (it > 0 && !mbar_wait(bar_do_free, (it - 1) & 1, abort_flag, 0x314)) break;
+                        mbar_arrive_expect_tx(bar_do_full, 2 * kChunkBytes);
+                        tma_load_2d(&tmdO, bar_do_full, smem + L::kdO, 0, qrow);
+                        tma_load_2d(&tmdO, bar_do_full, smem + L::kdO + kChunkBytes, 64, qrow);
+                        do_issued = it + 1;
+                        // Q of tile it once the dK MMAs of tile it-1 have read Q
+                        if (it > 0 && !mbar_wait(bar_qdo_free, (it - 1) & 1, abort_flag, 0x311)) break;
+                        mbar_arrive_expect_tx(bar_qdo_full, 2 * kChunkBytes);
                         tma_load_2d(&tmQ, bar_qdo_full, smem + L::kQ, 0, qrow);
                         tma_load_2d(&tmQ, bar_qdo_full, smem + L::kQ + kChunkBytes, 64, qrow);
-                        tma_load_2d(&tmdO, bar_qdo_full, smem + L::kdO, 0, qrow);
-                        tma_load_2d(&tmdO, bar_qdo_full, smem + L::kdO + kChunkBytes, 64, qrow);
+                        q_issued = it + 1;
                     }
                     // on an abort, let loads still in flight land before the CTA exits
-                    if (ntiles > 0) mbar_drain(bar_qdo_full, (ntiles - 1) & 1);
+                    if (do_issued > 0) mbar_drain(bar_do_full, (do_issued - 1) & 1);
+                    if (q_issued > 0) mbar_drain(bar_qdo_full, (q_issued - 1) & 1);
                 }
             }
         } else if (warp == 12) {
@@ -211,12 +224,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const uint32_t idQ = idesc_bf16(128, 128, false, true);   // dQ
                 bool ok = mbar_wait(bar_kv, 0, abort_flag, 0x301);
                 for (int it = 0; ok && it < ntiles; ++it) {
-                    if (!mbar_wait(bar_qdo_full, it & 1, abort_flag, 0x302)) break;
-                    if (it > 0 && !mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x303)) break;
+                    // dP first (its columns are free once the previous tile's P/dS were formed), then S,
+                    // which overwrites the previous tile's dQ once the flush has taken it out
+                    if (!mbar_wait(sparse ? bar_qdo_full : bar_do_full, it & 1, abort_flag, 0x302)) break;
                     if (sparse) fence_proxy_async_smem();  // cp.async-written rows -> tensor-core reads
                     tc_fence_after();
-                    mma_k128_kmajor(tS, sQ, sK, NKV * 128, idS);
                     mma_k128_kmajor(tdP, sdO, sV, NKV * 128, idS);
+                    if (!sparse && !mbar_wait(bar_qdo_full, it & 1, abort_flag, 0x315)) break;
+                    if (it > 0 && !mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x303)) break;
+                    tc_fence_after();
+                    mma_k128_kmajor(tS, sQ, sK, NKV * 128, idS);
                     mma_commit(bar_sdp_full);
                     if (!mbar_wait(bar_pds_full, it & 1, abort_flag, 0x304)) break;
                     tc_fence_after();
@@ -226,6 +243,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         mma_bf16_ss(tdV, smem_desc_sw128(sdO + kk * 2048, kChunkBytes),
                                     smem_desc_sw128(sP + kk * 2048, kChunkBytes), idT, (it > 0 || kk > 0) ? 1u : 0u);
                     }
+                    mma_commit(bar_do_free);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         mma_bf16_ss(tdK, smem_desc_sw128(sQ + kk * 2048, kChunkBytes),
