@@ -1,7 +1,8 @@
 """GPU parity: every step of the path through the C ABI against the fp64 oracle,
 on seeded inputs at sizes the oracle finishes in seconds that still span several
 tiles and a ragged tail (T not a multiple of the 128-row tile, lists whose
-length is not a multiple of 128, -1 padded selections, k = 1 and k = nb)."""
+length is not a multiple of 128, -1 padded selections, k = 1 and k = nb, a single
+block, many short heads)."""
 import numpy as np
 import pytest
 
@@ -23,6 +24,8 @@ CASES = [
     ("prefill_planted", "prefill", dict(H=2, T=2048), 16),
     ("k_equals_nb", "train", dict(B=1, H=1, T=512), 8),
     ("k_one", "long", dict(H=1, T=1024), 1),
+    ("single_block", "long", dict(H=1, T=128), 1),  # nb = 1: every query attends its own block only
+    ("many_heads_short", "long", dict(B=2, H=8, T=384), 3),
 ]
 
 
