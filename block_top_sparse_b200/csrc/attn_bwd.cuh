@@ -95,7 +95,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // Head-major unit order: the query rows and the dQ accumulator of the head
     // being worked on stay in L2.
     const int units_per_head = a.sparse ? a.nb : (a.T + NKV - 1) / NKV;
-    const int bh = blockIdx.x / units_per_head, kb = blockIdx.x % units_per_head;
+    int bh, kb;
+    unit_order(blockIdx.x, a.BH, units_per_head, bh, kb);
     const int kv0 = kb * NKV;
     const size_t head_rows = static_cast<size_t>(bh) * T;
     const bool sparse = a.sparse != 0;

@@ -135,7 +135,7 @@ constexpr int kFullFwdThreads = 384;
 __global__ void __launch_bounds__(kFullFwdThreads, 1)
     full_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ O, float *__restrict__ lse,
-                    int T, float scale_log2) {
+                    int BH, int T, float scale_log2) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + FullFwdSmem::kBar);
@@ -151,8 +151,9 @@ __global__ void __launch_bounds__(kFullFwdThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nqb = (T + 255) / 256;
-    const int qb = nqb - 1 - blockIdx.x;  // heaviest query blocks first
-    const int bh = blockIdx.y;
+    int bh, u;
+    unit_order(blockIdx.x, BH, nqb, bh, u);
+    const int qb = nqb - 1 - u;  // heaviest query blocks first
     const int row0 = bh * T;              // first tensor-map row of this head
     const int q0 = qb * 256;              // first query of tile a; tile b starts at q0 + 128
     // key tiles 0 .. diag: tile a ends at key tile 2qb, tile b at 2qb+1
@@ -469,7 +470,8 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 15);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.x / nb, j = blockIdx.x % nb;
+    int bh, j;
+    unit_order(blockIdx.x, BH, nb, bh, j);
     const int kv0 = j * NKV;
     const size_t head_rows = static_cast<size_t>(bh) * T;
     // this block's list (and partial-output rows) start at list position obase

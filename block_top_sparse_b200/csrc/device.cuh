@@ -150,6 +150,32 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *ba
         : "memory");
 }
 
+// Order of the (head, unit) work items of a grid of nh * per_head CTAs: head-major (a head's rows
+// stay in L2 while its units run), with every head's first unit -- its heaviest: the first key
+// block, which every query may select, or the longest query range -- pulled one head earlier, so
+// that the last head's heaviest unit does not start at the very end of the grid.
+__device__ __forceinline__ void unit_order(int u, int nh, int per_head, int &h, int &j) {
+    if (u == 0) {
+        h = 0;
+        j = 0;
+        return;
+    }
+    const int v = u - 1, full = (nh - 1) * per_head;
+    if (v < full) {
+        h = v / per_head;
+        const int r = v % per_head;
+        if (r == 0) {
+            h += 1;  // the next head's first unit
+            j = 0;
+        } else {
+            j = r;
+        }
+    } else {
+        h = nh - 1;
+        j = v - full + 1;
+    }
+}
+
 // Per-head region of the inverse selection index (and of the block-major
 // partial outputs): T*k entries plus up to one tile of padding per key block,
 // so that every block's list starts on a 128-entry boundary.

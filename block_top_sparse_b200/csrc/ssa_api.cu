@@ -451,9 +451,9 @@ ssa_status_t ssa_full_attn_fwd(const ssa_dims_t *dims, const void *Q, const void
         return SSA_ERR_CUDA;
     const size_t sm = FullFwdSmem::kTotal + 1024;
     if (!set_smem(full_fwd_kernel, sm)) return SSA_ERR_CUDA;
-    const dim3 grid((S.T + 255) / 256, S.BH);
-    full_fwd_kernel<<<grid, kFullFwdThreads, sm, st>>>(tmQ, tmK, tmV, (__nv_bfloat16 *)O, lse, S.T,
-                                                      S.scale * kLog2e);
+    const unsigned grid = static_cast<unsigned>(S.BH * ((S.T + 255) / 256));
+    full_fwd_kernel<<<grid, kFullFwdThreads, sm, st>>>(tmQ, tmK, tmV, (__nv_bfloat16 *)O, lse,
+                                                      static_cast<int>(S.BH), S.T, S.scale * kLog2e);
     return launch_status();
 }
 
