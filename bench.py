@@ -150,6 +150,61 @@ def reference_arm(args, rank):
     print(json.dumps(line), flush=True)
 
 
+def exact_attended_flops(B, H, T, d, s, k):
+    """Forward FLOPs by the attended-token count: query t sees (t mod s) + 1 keys of its own block and s keys
+    of each of min(k-1, b(t)) earlier blocks."""
+    t = np.arange(T, dtype=np.int64)
+    n = (t % s) + 1 + s * np.minimum(k - 1, t // s)
+    return 4.0 * B * H * d * float(n.sum())
+
+
+def sweep(args):
+    """Config 5: sparse forward tokens/s at T = 131072 for k in {4, 8, 16, 32, 64}, with the dropped mass
+    delta_t = 1 - exp(lse_s - lse_f) (mean, p99, max) and max_t |o_f - o_s| / (2 delta_t max|v|), which the
+    exact identity o_f = (1 - delta) o_s + delta u_drop bounds by 1.  One JSON line per k."""
+    import torch
+    from block_top_sparse_b200 import _lib as L
+    from block_top_sparse_b200 import build, inputs, ops
+    build.build()
+    wl = inputs.WORKLOADS["sweep"]
+    g = inputs.generate(wl)
+    dev = {key: torch.from_numpy(g[key].view(np.int16)).view(torch.bfloat16).cuda() for key in ("Q", "K", "V")}
+    Q, K, V = dev["Q"], dev["K"], dev["V"]
+    B, H, T, d, s = wl.B, wl.H, wl.T, wl.d, wl.s
+    dims0 = L.make_dims(B, H, T, d, s, 1)
+    Of, lf = ops.attn_fwd(dims0, Q, K, V)
+    vmax = torch.linalg.vector_norm(V.float(), dim=-1).amax(dim=-1, keepdim=True)
+    for k in (4, 8, 16, 32, 64):
+        dims = L.make_dims(B, H, T, d, s, k)
+        idx = ops.block_select(dims, Q, ops.block_pool(dims, K))
+        Os = torch.empty_like(Q)
+        lse = torch.empty(B, H, T, dtype=torch.float32, device=Q.device)
+        ws = ops._ws(dims, L.SSA_OP_SPARSE_FWD, Q.device)
+        call = lambda: L.ssa_sparse_attn_fwd(dims, Q, K, V, idx, Os, lse, ws)
+        for _ in range(args.warmup):
+            call()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(args.steps):
+            call()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / args.steps
+        delta = ops.dropped_mass(dims, lse, lf).float()
+        gap = torch.linalg.vector_norm(Of.float() - Os.float(), dim=-1)
+        ratio = gap / (2 * delta.clamp(min=1e-30) * vmax)
+        ratio = torch.where(delta > 1e-6, ratio, torch.zeros_like(ratio))  # rows with nothing dropped
+        fl = flops(B, H, T, d, s, k)[0]
+        print(json.dumps({"sweep": "sparse fwd, T=%d H=%d s=%d" % (T, H, s), "k": k, "receptive_field": k * s,
+                          "sparse_fwd_ms": ms, "tokens_per_s": B * T / (ms / 1e3), "tflops": fl / (ms / 1e3) / 1e12,
+                          "delta_mean": float(delta.mean()), "delta_p99": float(torch.quantile(delta.flatten()[::97], 0.99)),
+                          "delta_max": float(delta.max()), "bound_ratio_max": float(ratio.max()),
+                          "device_error": L.ssa_get_device_error()}), flush=True)
+        del idx, Os, lse, ws
+        torch.cuda.empty_cache()
+
+
 def config_block(wl):
     return {"workload": "long-context fwd+bwd, both streams + alignment: B=%d H=%d T=%d d=%d s=%d k=%d, sink block"
                         % (wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL),
@@ -304,6 +359,8 @@ def ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_block(wl),
         "sparse_attn": {"fwd_bwd_ms": sparse_ms, "tflops": (sf + sb) / (sparse_ms / 1e3) / 1e12,
+                        "tflops_exact_attended": 3.5 * exact_attended_flops(wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL)
+                        / (sparse_ms / 1e3) / 1e12,
                         "frac_of_peak": (sf + sb) / (sparse_ms / 1e3) / 1e12 / peak_sust,
                         "frac_of_burst_peak": (sf + sb) / (sparse_ms / 1e3) / 1e12 / peak_burst,
                         "tokens_per_s": wl.B * wl.T / (sparse_ms / 1e3), "flop_per_step": sf + sb},
@@ -311,7 +368,9 @@ def ours(args, rank, world, local_rank):
                       "frac_of_peak": (ff + fb) / (full_ms / 1e3) / 1e12 / peak_sust},
         "op_ms": op_ms,
         "select_hbm": {"gbs": (wl.B * wl.H * wl.T * (2 * wl.d + 4 * K_SEL)) / (op_ms["select"] / 1e3) / 1e9,
-                       "frac": (wl.B * wl.H * wl.T * (2 * wl.d + 4 * K_SEL)) / (op_ms["select"] / 1e3) / 1e9 / hbm},
+                       "frac": (wl.B * wl.H * wl.T * (2 * wl.d + 4 * K_SEL)) / (op_ms["select"] / 1e3) / 1e9 / hbm,
+                       "frac_of_nominal_8tbs": (wl.B * wl.H * wl.T * (2 * wl.d + 4 * K_SEL))
+                       / (op_ms["select"] / 1e3) / 1e9 / 8000.0},
         "pool_hbm": {"gbs": (wl.B * wl.H * wl.T * 2 * wl.d) / (pool_kernel_ms / 1e3) / 1e9,
                      "frac": (wl.B * wl.H * wl.T * 2 * wl.d) / (pool_kernel_ms / 1e3) / 1e9 / hbm,
                      "ms": pool_kernel_ms, "timing": "mean of 10 back-to-back launches"},
@@ -393,6 +452,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=16384, help="prefix length of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="the k sweep at T = 131072 (one JSON line per k)")
     ap.add_argument("--op", default=None,
                     choices=["pool", "select", "full_fwd", "sparse_fwd", "full_bwd", "sparse_bwd"],
                     help="time one library call instead of the whole step (profiling)")
@@ -401,6 +461,9 @@ def main():
     ap.add_argument("--H", type=int, default=0)
     ap.add_argument("--k", type=int, default=0)
     args = ap.parse_args()
+    if args.sweep:
+        sweep(args)
+        return
     if args.op:
         single_op(args)
         return

@@ -182,3 +182,14 @@ def test_step_both_streams_matches_oracle():
             for nm, g, a, b in zip(("dQ", "dK", "dV"), (step.dQ, step.dK, step.dV), g_full, g_sparse):
                 check_close("step.%s.%s" % (main, nm), to_np(g).reshape(a.shape), a + b, True)
     assert L.ssa_get_device_error() == L.SSA_OK
+
+
+@pytest.mark.parametrize("name,wlname,over,k", [CASES[1], CASES[3]], ids=[CASES[1][0], CASES[3][0]])
+def test_attention_at_unit_scale(name, wlname, over, k):
+    # The other reading of the softmax scale: the inputs' d^-1/4 already folds it in (unit-variance logits).
+    w, _, f, dev = _setup(wlname, over, k)
+    dims = L.make_dims(w.B, w.H, w.T, w.d, w.s, k, dtype=w.dtype, scale=1.0)
+    Kbar = ora.block_pool(f["K"], w.s)
+    idx_ref, _, _ = ora.block_select(f["Q"], Kbar, w.s, k)
+    _attn_check(w, dims, f, dev, None, name + ".unit_scale.full")
+    _attn_check(w, dims, f, dev, idx_ref, name + ".unit_scale.sparse")
