@@ -88,15 +88,26 @@ __global__ void __launch_bounds__(1024) index_scan_kernel(int *__restrict__ cnt,
 
 // Pass 3: one warp per chunk writes entries (t << 8) | slot at their final
 // position, in ascending query order (ranks within a 32-query step come from
-// lane bitmasks).  k <= 256 and T < 2^23 keep the encoding in an int32.
+// lane bitmasks).  k <= 256 and T < 2^23 keep the encoding in an int32.  Each
+// 32-query step's selection rows are staged in shared memory by one coalesced
+// load (rows padded to k + 1 ints: conflict-free per-lane reads), and the list
+// positions (pos, when asked) leave through the same staging, coalesced.
+// Shared memory per warp: 2 * nb + 2 * 32 * (k + 1) ints.
+__host__ __device__ constexpr size_t index_fill_warp_ints(int nb, int k) {
+    return 2 * static_cast<size_t>(nb) + 64 * static_cast<size_t>(k + 1);
+}
+
 __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t *__restrict__ idx,
                                                          const int *__restrict__ off, int32_t *__restrict__ entries,
                                                          int32_t *__restrict__ pos, int T, int k, int nb, int nch) {
     extern __shared__ int sm_fill[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.y, c = blockIdx.x * 4 + warp;
-    uint32_t *bits = reinterpret_cast<uint32_t *>(sm_fill) + warp * 2 * nb;
-    int *run = sm_fill + warp * 2 * nb + nb;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, wpc = blockDim.x >> 5;
+    const int bh = blockIdx.y, c = blockIdx.x * wpc + warp;
+    int *wsm = sm_fill + warp * index_fill_warp_ints(nb, k);
+    uint32_t *bits = reinterpret_cast<uint32_t *>(wsm);
+    int *run = wsm + nb;
+    int *rows = wsm + 2 * nb;              // [32][k + 1] selections of the step's queries
+    int *prow = rows + 32 * (k + 1);       // [32][k + 1] their list positions
     if (c < nch) {
         for (int j = lane; j < nb; j += 32) {
             bits[j] = 0u;
@@ -108,30 +119,44 @@ __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t *__restri
     int32_t *dst = entries + static_cast<size_t>(bh) * list_stride(T, k, nb);
     const uint32_t lt_mask = (1u << lane) - 1u;
     const int t_end = min(T, (c + 1) * kIdxChunk);
+    const int *mine = rows + lane * (k + 1);
+    int *mpos = prow + lane * (k + 1);
     for (int tb = c * kIdxChunk; tb < t_end; tb += 32) {
         const int t = tb + lane;
-        const bool valid = t < t_end;
-        const int32_t *row = idx + (static_cast<size_t>(bh) * T + t) * k;
+        const size_t base = (static_cast<size_t>(bh) * T + tb) * k;
+        const int n = min(32, t_end - tb) * k;  // the step's selections, contiguous in idx
+        for (int e = lane; e < 32 * k; e += 32) {
+            const int r = e / k;
+            rows[r * (k + 1) + (e - r * k)] = e < n ? __ldg(idx + base + e) : -1;
+        }
+        __syncwarp();
         for (int i = 0; i < k; ++i) {
-            const int j = valid ? __ldg(row + i) : -1;
+            const int j = mine[i];
             if (j >= 0 && j < nb) atomicOr(&bits[j], 1u << lane);
         }
         __syncwarp();
         for (int i = 0; i < k; ++i) {
-            const int j = valid ? __ldg(row + i) : -1;
+            const int j = mine[i];
             const int at = (j >= 0 && j < nb) ? run[j] + __popc(bits[j] & lt_mask) : -1;
             if (at >= 0) dst[at] = (t << 8) | i;
-            if (pos && valid) pos[(static_cast<size_t>(bh) * T + t) * k + i] = at;
+            mpos[i] = at;
         }
         __syncwarp();
         for (int i = 0; i < k; ++i) {
-            const int j = valid ? __ldg(row + i) : -1;
+            const int j = mine[i];
             if (j >= 0 && j < nb) {
                 const uint32_t b = bits[j];
                 if (b != 0u && lane == __ffs(b) - 1) {
                     run[j] += __popc(b);
                     bits[j] = 0u;
                 }
+            }
+        }
+        if (pos) {
+            __syncwarp();
+            for (int e = lane; e < n; e += 32) {
+                const int r = e / k;
+                pos[base + e] = prow[r * (k + 1) + (e - r * k)];
             }
         }
         __syncwarp();

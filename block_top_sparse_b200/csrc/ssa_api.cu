@@ -62,6 +62,8 @@ ssa_status_t check_dims(const ssa_dims_t *dims, Shape &S, bool need_k) {
     if (need_k && S.tc && (S.k > 256 || S.T >= (1 << 23))) return SSA_ERR_UNSUPPORTED;
     // list positions of the whole index (and TMA row coordinates of the partials) fit an int32
     if (need_k && S.tc && S.BH * list_stride(S.T, S.k, S.nb) >= (size_t(1) << 31)) return SSA_ERR_UNSUPPORTED;
+    // one warp's staging of the index fill must fit in shared memory
+    if (need_k && S.tc && index_fill_warp_ints(S.nb, S.k) * 4 > 227 * 1024) return SSA_ERR_UNSUPPORTED;
     return SSA_OK;
 }
 
@@ -197,10 +199,12 @@ ssa_status_t build_index(const Shape &S, const int32_t *idx, IndexWs &W, cudaStr
     if (!set_smem(index_count_kernel, hbytes)) return SSA_ERR_CUDA;
     index_count_kernel<<<dim3(W.nch, S.BH), 256, hbytes, st>>>(idx, W.cnt, S.T, S.k, S.nb, W.nch);
     index_scan_kernel<<<S.BH, 1024, 0, st>>>(W.cnt, W.lstart, W.llen, S.nb, W.nch);
-    const size_t fbytes = static_cast<size_t>(S.nb) * 8 * 4;
-    if (!set_smem(index_fill_kernel, fbytes)) return SSA_ERR_CUDA;
-    index_fill_kernel<<<dim3((W.nch + 3) / 4, S.BH), 128, fbytes, st>>>(idx, W.cnt, W.entries, pos, S.T, S.k,
-                                                                          S.nb, W.nch);
+    // four warps (chunks) per CTA while their staging fits comfortably, else one
+    const size_t wbytes = index_fill_warp_ints(S.nb, S.k) * 4;
+    const int wpc = wbytes * 4 <= 160 * 1024 ? 4 : 1;
+    if (!set_smem(index_fill_kernel, wbytes * wpc)) return SSA_ERR_CUDA;
+    index_fill_kernel<<<dim3((W.nch + wpc - 1) / wpc, S.BH), 32 * wpc, wbytes * wpc, st>>>(
+        idx, W.cnt, W.entries, pos, S.T, S.k, S.nb, W.nch);
     return launch_status();
 }
 
