@@ -34,11 +34,6 @@ struct Rows {
     int k;
 };
 
-// Row of the [.., T, k] per-(query, slot) arrays addressed by an index entry.
-__device__ __forceinline__ size_t entry_row(int entry, int k) {
-    return static_cast<size_t>(entry >> 8) * k + (entry & 255);
-}
-
 // Query position and global selection entry of tile row r of tile `it`.
 __device__ __forceinline__ bool tile_row(const Rows &R, int T, int it, int r, int &t, int &entry) {
     if (R.list) {
@@ -51,30 +46,6 @@ __device__ __forceinline__ bool tile_row(const Rows &R, int T, int it, int r, in
     t = R.first + it * kTileQ + r;
     entry = -1;
     return t < T;
-}
-
-// cp.async one 256-byte row (128 bf16) into row r of a 2-chunk swizzled tile.
-// Invalid rows are zero-filled (source size 0).
-__device__ __forceinline__ void gather_row(uint32_t tile, const __nv_bfloat16 *src, bool valid, int r) {
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-        const uint32_t dst = tile + (u >> 3) * kChunkBytes + r * 128 + ((((u & 7) ^ (r & 7)) & 7) << 4);
-        cp_async_16(dst, src + u * 8, valid ? 16u : 0u);
-    }
-}
-
-// One warp gathers the 128 rows of a query tile (4 rows per lane) into a
-// 2-chunk swizzled tile; rows past the list are zero-filled.  The caller then
-// signals completion with cp_async_mbar_arrive_noinc().
-__device__ __forceinline__ void warp_gather_tile(uint32_t tile, const __nv_bfloat16 *base, const Rows &R, int T,
-                                                 int it, size_t head_rows, int lane) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int r = lane + 32 * q;
-        int t = 0, e = 0;
-        const bool valid = tile_row(R, T, it, r, t, e);
-        gather_row(tile, base + (head_rows + (valid ? t : 0)) * kD, valid, r);
-    }
 }
 
 // Write 32 fp32 values as bf16 into row r, columns [c0, c0+32) of a swizzled

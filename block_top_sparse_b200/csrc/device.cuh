@@ -106,8 +106,6 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void *src, 
                  : "memory");
 }
 
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
 // Arrive on `bar` once every cp.async this thread issued so far has landed; the
 // arrival is pre-counted in the barrier's expected count (.noinc).
 __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
@@ -115,14 +113,6 @@ __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
 }
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// Bulk fp32 add of `bytes` contiguous bytes of shared memory into global memory
-// (performed in L2), tracked by this thread's bulk async-group.
-__device__ __forceinline__ void bulk_reduce_add_f32(float *dst, uint32_t src_smem, uint32_t bytes) {
-    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
-                 "r"(src_smem), "r"(bytes)
-                 : "memory");
-}
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
@@ -184,19 +174,6 @@ __host__ __device__ __forceinline__ size_t list_stride(int T, int k, int nb) {
     return static_cast<size_t>(T) * k + static_cast<size_t>(nb) * kListPad;
 }
 
-// TMA row gather: rows r0..r3 of a 2D tensor map whose box is one row high
-// (box = {64 columns, 1}), columns [col, col + 64), into 4 consecutive 128-byte
-// rows at dst (dst 512-byte aligned inside a 1024-byte aligned swizzle atom, so
-// the 128-byte swizzle lands exactly as for a 128-row box load).
-__device__ __forceinline__ void tma_gather4(const CUtensorMap *map, uint64_t *bar, uint32_t dst, int col, int r0,
-                                            int r1, int r2, int r3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-        "l"(map), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
-        : "memory");
-}
-
 // Tiled TMA store of a box from shared memory (same swizzle as the tensor map),
 // tracked by this thread's bulk async-group.  Coordinates must be >= 0.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src_smem, int col, int row) {
@@ -211,13 +188,6 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t sr
 __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, uint32_t src_smem, int col, int row) {
     asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map),
                  "r"(col), "r"(row), "r"(src_smem)
-                 : "memory");
-}
-
-// Bulk copy shared -> global (both 16-byte aligned, bytes a multiple of 16),
-// tracked by this thread's bulk async-group.
-__device__ __forceinline__ void bulk_store(void *dst, uint32_t src_smem, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src_smem), "r"(bytes)
                  : "memory");
 }
 
@@ -301,11 +271,6 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
-// Byte offset of element (row r, column c) inside a 128B-swizzled chunk of 64 bf16 columns.
-__device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c) {
-    return r * 128u + ((((c >> 3) ^ (r & 7u)) & 7u) << 4) + ((c & 7u) << 1);
-}
-
 // tcgen05.ld / st, 32 lanes x 32 bit, 32 consecutive columns per thread.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     uint32_t r[32];
@@ -338,19 +303,6 @@ __device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, uint32_t (&r)[32
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// Store 32 consecutive 32-bit columns per thread (e.g. 64 bf16 packed in pairs).
-__device__ __forceinline__ void tmem_st32_u(uint32_t taddr, const uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
-        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
-        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-        : "memory");
-}
 
 // Store 16 consecutive 32-bit columns per thread.
 __device__ __forceinline__ void tmem_st16_u(uint32_t taddr, const uint32_t (&v)[16]) {
