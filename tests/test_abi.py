@@ -81,6 +81,9 @@ BAD_DIMS = [
     (dict(dtype=7), L.SSA_ERR_INVALID_ARG),
     (dict(scale=0.0), L.SSA_ERR_INVALID_ARG),
     (dict(scale=float("nan")), L.SSA_ERR_INVALID_ARG),
+    (dict(T=64 * 300, k=257), L.SSA_ERR_UNSUPPORTED),                # slot index above the entry encoding
+    (dict(B=1, H=512, T=131072, s=128, k=32), L.SSA_ERR_UNSUPPORTED),  # list positions beyond int32
+    (dict(H=1, T=64 * 21000, k=256), L.SSA_ERR_UNSUPPORTED),         # index-fill staging beyond shared memory
 ]
 
 
