@@ -415,3 +415,22 @@ def test_bwd_with_stored_bf16_output_matches_dense_formulas(ora):
         np.testing.assert_allclose(gg[0], w, rtol=0, atol=1e-12)
     np.testing.assert_allclose(got[2], exact[2], rtol=0, atol=1e-12)  # dV does not involve D
     assert np.abs(got[0] - exact[0]).max() > 0  # the rounding is visible in dQ
+
+
+def test_oracle_regression_against_committed_golden(ora):
+    # tests/golden/tiny_case.json: the oracle's outputs on a tiny seeded case, written by make_golden.py
+    import json
+    import os
+    import importlib.util
+    here = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+    spec = importlib.util.spec_from_file_location("make_golden", os.path.join(here, "make_golden.py"))
+    mg = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mg)
+    doc = json.load(open(os.path.join(here, "tiny_case.json")))
+    x = {k: np.array(v) for k, v in doc["inputs"].items()}
+    for k, v in mg.inputs().items():
+        np.testing.assert_array_equal(x[k], v)  # the generator still produces the stored inputs
+    got = mg.compute(x)
+    for k, v in doc["outputs"].items():
+        np.testing.assert_allclose(np.asarray(got[k], dtype=np.float64), np.array(v, dtype=np.float64),
+                                   rtol=1e-12, atol=1e-12, err_msg=k)
