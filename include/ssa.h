@@ -83,9 +83,10 @@ enum {
 size_t ssa_workspace_size(const ssa_dims_t *dims, int op);
 
 /*
- * Block pooling (paper section 3: "scores preceding blocks using mean-pooled
- * keys").  Kbar[b,h,j,:] = (1/s) * sum_{t in block j} K[b,h,t,:], fp32
- * accumulation, unweighted.
+ * Block pooling (paper section 3: each block of keys is summarised by the mean
+ * of its keys, which the queries are scored against).
+ * Kbar[b,h,j,:] = (1/s) * sum_{t in block j} K[b,h,t,:], fp32 accumulation,
+ * unweighted.
  *   K    in   [B,H,T,d] dtype
  *   Kbar out  [B,H,T/s,d] fp32
  */

@@ -116,7 +116,7 @@ void ora_block_select(i64 BH, i64 T, i64 d, i64 s, i64 k, const double *Q, const
 
 /* ---------------------------------------------------------------------------
  * Attended set S(t).
- * Full attention (page section 3: "uses all preceding tokens"): S(t) = {0..t}.
+ * Full attention (paper section 3: every preceding token takes part): S(t) = {0..t}.
  * Sparse attention (page section 3: the selected blocks' tokens form the
  * reduced key/value matrices): S(t) = union over the selected blocks of their
  * tokens, restricted to positions <= t (causal inside the query's own block).
