@@ -9,7 +9,8 @@
 //   S = Q K^T, dP = dO V^T                      (M = 128 query rows)
 //   P = exp(scale S - lse), dS = P o (dP - D)   -> shared memory, bf16
 //   dV^T += dO^T P, dK^T += Q^T dS              (M = head dim 128)
-//   dQ = dS K                                    -> fp32 vector atomics, * scale
+//   dQ = dS K, * scale                           -> full: added into an fp32 accumulator;
+//                                                   sparse: a bf16 partial row per (query, slot)
 // Paper: section 4.2 (keys outside S(t) get no gradient; the selection is a
 // constant), FlashAttention-2 style recomputation of P from the saved lse.
 //
@@ -22,10 +23,10 @@
 //                tile's rows are contiguous): columns 0-63 into a 32 KB staging
 //                buffer of its own, 64-127 into the P region (free once dQ is
 //                computed), added by four TMA tensor reduce-adds issued by one
-//                thread.  Sparse stream (gathered rows): columns 64-127 wait in
-//                registers while 0-63 go through the staging buffer, each half
-//                added with coalesced float4 reductions (two 256-byte row halves
-//                per warp instruction);
+//                thread.  Sparse stream (gathered rows): the tile is rounded to
+//                bf16 and written by TMA tile stores as partial rows at the list
+//                positions of the block's entries (contiguous there); a merge
+//                kernel later sums each query's k partials;
 //   warp 12      MMA issuer (one thread);
 //   warp 13      TMA producer (K_j, V_j; contiguous Q / dO tiles of the full stream);
 //   warps 14-19  sparse stream: gather the next tile's Q and dO rows with
@@ -57,7 +58,6 @@ struct BwdSmem {
 struct BwdArgs {
     const __nv_bfloat16 *Q, *dO;
     const float *lse, *Dvec;
-    float *dQacc;
     __nv_bfloat16 *dK, *dV;
     const int32_t *entries, *lstart, *llen;  // sparse only
     int BH, T, k, nb, sparse, accumulate;
@@ -129,10 +129,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(bar_dq_empty, 128);
         mbar_init(bar_final, 1);
         mbar_init(bar_f_staged, 128);
-        // staging buffers released by every flush thread (sparse: two rounds per tile through
-        // the staging buffer) or by the thread that issued the TMA reduce-adds once they have
-        // read shared memory (full: P region and staging buffer)
-        mbar_init(bar_f_free, sparse ? 128 : 1);
+        // full stream: staging buffers released by the thread that issued the TMA reduce-adds
+        // once they have read shared memory (P region and staging buffer)
+        mbar_init(bar_f_free, 1);
         mbar_init(bar_p_free, 1);
         mbar_init(bar_epi, 256);
         *abort_flag = 0;
@@ -321,78 +320,50 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             if (r == 0) bulk_wait();  // the TMA reduce-adds have completed
         } else {
-            // Sparse stream: columns 0-63 go to the staging buffer, 64-127 stay in registers (so
-            // dQ leaves tensor memory at once), then each half is added in turn.  Row r: 16 units of
-            // 16 bytes, unit q at position q ^ (r & 15) (conflict-free both ways).
-            uint32_t fph = 0;  // staging rounds (two per tile)
-            auto stage = [&](const uint32_t (&g)[32], int q0) {
-#pragma unroll
-                for (int q8 = 0; q8 < 8; ++q8) {
-                    const int q = q0 + q8;
-                    const uint32_t *x = g + 4 * q8;
-                    st_shared_v4(sF + r * 256 + (((q ^ r) & 15) << 4), __float_as_uint(__uint_as_float(x[0]) * a.scale),
-                                 __float_as_uint(__uint_as_float(x[1]) * a.scale),
-                                 __float_as_uint(__uint_as_float(x[2]) * a.scale),
-                                 __float_as_uint(__uint_as_float(x[3]) * a.scale));
-                }
-            };
+            // Sparse stream: the tile's dQ (scaled, rounded to bf16) is one partial row per
+            // (query, slot) at the entry's list position, so nothing is reduced here: each warp
+            // stages its 32 rows in the 128-byte-swizzled layout (columns 0-63 | 64-127 in the two
+            // halves of the staging buffer) and writes them with two TMA tile stores.  The list
+            // region of every block is padded to whole tiles, so the rows of a partial last tile
+            // stay inside this block's region (and are never read).
+            const size_t lbase = static_cast<size_t>(bh) * list_stride(T, a.k, a.nb) + a.lstart[bh * a.nb + kb];
+            const uint32_t wrow = static_cast<uint32_t>((warp & 3) * 32);
             for (int it = 0; it < ntiles; ++it) {
-                int t = 0, e = 0;
-                const bool valid = tile_row(R, T, it, r, t, e);
-                const int t_mine = valid ? t : -1;
                 if (!mbar_wait(bar_dq_full, it & 1, abort_flag, 0x307)) break;
                 tc_fence_after();
-                uint32_t hi[2][32];
-                bool ok = true;
+                // the previous tile's stores have read this warp's staging rows
+                if (lane == 0) bulk_wait_read();
+                __syncwarp();
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    // the previous round's rows have been read by every flush warp
-                    if (fph > 0 && !mbar_wait(bar_f_free, (fph - 1) & 1, abort_flag, 0x30b)) {
-                        ok = false;
-                        break;
-                    }
-                    if (hf == 0) {
-#pragma unroll
-                        for (int c = 0; c < 2; ++c) {
-                            uint32_t g[32];
-                            tmem_ld32_async(tdQ + lane_off + 32 * c, g);
-                            tmem_ld_wait();
-                            stage(g, 8 * c);
-                        }
-                        tmem_ld32_async(tdQ + lane_off + 64, hi[0]);
-                        tmem_ld32_async(tdQ + lane_off + 96, hi[1]);
-                        tmem_ld_wait();
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t g[2][32];
+                    tmem_ld32_async(tdQ + lane_off + 64 * hh, g[0]);
+                    tmem_ld32_async(tdQ + lane_off + 64 * hh + 32, g[1]);
+                    tmem_ld_wait();
+                    if (hh == 1) {
                         tc_fence_before();
                         mbar_arrive(bar_dq_empty);  // dQ has left tensor memory: the next S may overwrite it
-                    } else {
-                        stage(hi[0], 0);
-                        stage(hi[1], 8);
                     }
-                    mbar_arrive(bar_f_staged);
-                    if (!mbar_wait(bar_f_staged, fph & 1, abort_flag, 0x30a)) {
-                        ok = false;
-                        break;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const uint32_t *x = g[u >> 2] + 8 * (u & 3);
+                        st_shared_v4(sF + hh * kChunkBytes + r * 128 + (((u ^ (r & 7)) & 7) << 4),
+                                     pack_bf16x2(__uint_as_float(x[0]) * a.scale, __uint_as_float(x[1]) * a.scale),
+                                     pack_bf16x2(__uint_as_float(x[2]) * a.scale, __uint_as_float(x[3]) * a.scale),
+                                     pack_bf16x2(__uint_as_float(x[4]) * a.scale, __uint_as_float(x[5]) * a.scale),
+                                     pack_bf16x2(__uint_as_float(x[6]) * a.scale, __uint_as_float(x[7]) * a.scale));
                     }
-                    // the warp's 32 rows, two per instruction: half-warp h2 takes row 2i + h2,
-                    // lane l & 15 its 16-byte unit
-                    const int u = lane & 15;
-#pragma unroll 4
-                    for (int i = 0; i < 16; ++i) {
-                        const int rl = 2 * i + (lane >> 4);
-                        const int row = 32 * (warp & 3) + rl;
-                        const int t_dst = __shfl_sync(0xffffffffu, t_mine, rl);
-                        float4 v;
-                        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                                     : "r"(sF + row * 256 + (((u ^ row) & 15) << 4)));
-                        if (t_dst >= 0)
-                            atomicAdd(reinterpret_cast<float4 *>(a.dQacc + (head_rows + t_dst) * kD + 64 * hf) + u, v);
-                    }
-                    mbar_arrive(bar_f_free);
-                    ++fph;
                 }
-                if (!ok) break;
+                fence_proxy_async_smem();  // generic-proxy staging writes -> TMA reads
+                __syncwarp();
+                if (lane == 0) {
+                    const int row0 = static_cast<int>(lbase + static_cast<size_t>(it) * kTileQ + wrow);
+                    tma_store_2d(&tmdQ, sF + wrow * 128, 0, row0);
+                    tma_store_2d(&tmdQ, sF + kChunkBytes + wrow * 128, 64, row0);
+                    bulk_commit();
+                }
             }
+            if (lane == 0) bulk_wait();  // the stores have completed
         }
     } else {
         // ---------------- softmax / dS warpgroups ----------------
@@ -401,11 +372,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int h = warp >> 2;                 // column half
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         bool ok = true;
+        // Row data is fetched ahead: the query position of tile it+2 and the lse, D of tile it+1
+        // are loaded while tile it is processed (the sparse stream's lse / D addresses depend on
+        // the position loaded from the list), so no dependent global load sits between two tiles.
+        int e = 0, t_n1 = 0, t_n2 = 0;
+        bool v_n1 = ntiles > 0 && tile_row(R, T, 0, r, t_n1, e);
+        float lse_n = v_n1 ? __ldg(a.lse + head_rows + t_n1) : 0.f;
+        float D_n = v_n1 ? __ldg(a.Dvec + head_rows + t_n1) : 0.f;
+        bool v_n2 = ntiles > 1 && tile_row(R, T, 1, r, t_n2, e);
         for (int it = 0; it < ntiles; ++it) {
-            int t = 0, e = 0;
-            const bool valid = tile_row(R, T, it, r, t, e);
-            const float lse2 = valid ? __ldg(a.lse + head_rows + t) * kLog2e : 0.f;
-            const float Dt = valid ? __ldg(a.Dvec + head_rows + t) : 0.f;
+            const bool valid = v_n1;
+            const int t = t_n1;
+            const float lse2 = lse_n * kLog2e;
+            const float Dt = D_n;
+            v_n1 = v_n2;
+            t_n1 = t_n2;
+            lse_n = v_n1 ? __ldg(a.lse + head_rows + t_n1) : 0.f;
+            D_n = v_n1 ? __ldg(a.Dvec + head_rows + t_n1) : 0.f;
+            v_n2 = it + 2 < ntiles && tile_row(R, T, it + 2, r, t_n2, e);
             if (!mbar_wait(bar_sdp_full, it & 1, abort_flag, 0x306)) {
                 ok = false;
                 break;

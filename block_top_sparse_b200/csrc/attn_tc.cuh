@@ -559,12 +559,17 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t sO = smem_u32(smem + L::kO + g * L::kOStage);  // this warpgroup's staging tile
         const uint32_t tS = tmem + 128 * g + lane_off, tO = tmem + 256 + 128 * g + lane_off;
+        // this row's list entry (t << 8 | slot, or -1 past the list) is loaded one tile ahead
+        int ent_n = (g < ntiles && g * kTileQ + r < R.len) ? __ldg(R.list + g * kTileQ + r) : -1;
         for (int it = g; it < ntiles; it += 2) {
             const int i = it >> 1;
-            const bool valid = it * kTileQ + r < R.len;
-            const int lim = valid ? (__ldg(R.list + it * kTileQ + r) >> 8) - kv0 : -1;  // overlaps the wait
+            const int ent = ent_n;
+            if (it + 2 < ntiles)
+                ent_n = (it + 2) * kTileQ + r < R.len ? __ldg(R.list + (it + 2) * kTileQ + r) : -1;
+            const bool valid = ent >= 0;
             if (!mbar_wait(bar_s_full + g, i & 1, abort_flag, 0x206)) break;
             tc_fence_after();
+            const int lim = valid ? (ent >> 8) - kv0 : -1;
             uint32_t sr[NKV / 32][32];
 #pragma unroll
             for (int c = 0; c < NKV / 32; ++c) tmem_ld32_async(tS + 32 * c, sr[c]);

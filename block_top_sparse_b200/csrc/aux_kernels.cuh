@@ -225,7 +225,56 @@ __global__ void __launch_bounds__(256) sparse_merge_kernel(const int32_t *__rest
     if (lane == 0) lse[row] = mx + __logf(wsum);
 }
 
-// D[row] = sum_c dO[row,c] * O[row,c] (one warp per row) and zero the fp32 dQ accumulator row.
+// Sparse-stream dQ from its partials (head dimension 128):
+//   dQ[row] = (accumulate ? dQ[row] : 0) + sum_i dQpart[pos[row * k + i]]
+// summed in fp32 and rounded once.  The partial of (query, slot i) sits at list
+// position pos[row * k + i] of its head's region (-1: slot not attended).  Lane i
+// holds slot i's position, so the slots' row loads are all in flight at once; lane
+// l then owns columns 4l .. 4l+3.
+__global__ void __launch_bounds__(256) dq_merge_kernel(const int32_t *__restrict__ pos,
+                                                       const __nv_bfloat16 *__restrict__ dQpart,
+                                                       __nv_bfloat16 *__restrict__ dQ, size_t rows, int T, int k,
+                                                       int nb, int accumulate) {
+    const size_t row = static_cast<size_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const size_t region = (row / T) * list_stride(T, k, nb);
+    const int32_t *ps = pos + row * k;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    uint2 *dst = reinterpret_cast<uint2 *>(dQ + row * 128) + lane;
+    if (accumulate) {
+        const uint2 o = *dst;
+        acc[0] = __uint_as_float(o.x << 16);
+        acc[1] = __uint_as_float(o.x & 0xFFFF0000u);
+        acc[2] = __uint_as_float(o.y << 16);
+        acc[3] = __uint_as_float(o.y & 0xFFFF0000u);
+    }
+    for (int i0 = 0; i0 < k; i0 += 32) {
+        const int p = (i0 + lane < k) ? __ldg(ps + i0 + lane) : -1;
+        const int n = min(32, k - i0);
+        for (int s0 = 0; s0 < n; s0 += 8) {
+            uint2 u[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int pq = __shfl_sync(0xffffffffu, p, (s0 + q) & 31);
+                u[q] = (s0 + q < n && pq >= 0)
+                           ? __ldg(reinterpret_cast<const uint2 *>(dQpart + (region + pq) * 128) + lane)
+                           : make_uint2(0u, 0u);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                acc[0] += __uint_as_float(u[q].x << 16);
+                acc[1] += __uint_as_float(u[q].x & 0xFFFF0000u);
+                acc[2] += __uint_as_float(u[q].y << 16);
+                acc[3] += __uint_as_float(u[q].y & 0xFFFF0000u);
+            }
+        }
+    }
+    *dst = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
+}
+
+// D[row] = sum_c dO[row,c] * O[row,c] (one warp per row); zero the fp32 dQ
+// accumulator row when there is one (the sparse tensor-core stream has partials instead).
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const T *__restrict__ dO, const T *__restrict__ O,
                                                        float *__restrict__ Dvec, float *__restrict__ dQacc,
@@ -236,7 +285,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const T *__restrict__ dO,
     float acc = 0.f;
     for (int c = lane; c < d; c += 32) {
         acc += to_f32(dO[row * d + c]) * to_f32(O[row * d + c]);
-        dQacc[row * d + c] = 0.f;
+        if (dQacc) dQacc[row * d + c] = 0.f;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);

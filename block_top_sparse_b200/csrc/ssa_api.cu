@@ -103,10 +103,14 @@ size_t ws_bytes_for(const Shape &S, int op) {
             return index_bytes(S) + align_up(S.BH * list_stride(S.T, S.k, S.nb) * (128 * 2 + 4)) +
                    align_up(S.rows * S.k * 4);
         case SSA_OP_SPARSE_BWD:
+            // D | index | list position of every (query, slot) | bf16 dQ partials by list position
+            if (S.tc)
+                return align_up(S.rows * 4) + index_bytes(S) + align_up(S.rows * S.k * 4) +
+                       align_up(S.BH * list_stride(S.T, S.k, S.nb) * 128 * 2);
+            [[fallthrough]];
         case SSA_OP_FULL_BWD: {
             size_t b = align_up(S.rows * 4) + align_up(S.rows * S.d * 4);  // D, dQacc
             if (!S.tc) b += 2 * align_up(S.rows * S.d * 4);                // dKacc, dVacc
-            if (op == SSA_OP_SPARSE_BWD && S.tc) b += index_bytes(S);
             return b;
         }
         case SSA_OP_FULL_FWD:
@@ -257,14 +261,23 @@ ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V,
     uint8_t *p = static_cast<uint8_t *>(ws);
     float *Dvec = reinterpret_cast<float *>(p);
     p += align_up(S.rows * 4);
-    float *dQacc = reinterpret_cast<float *>(p);
-    p += align_up(S.rows * S.d * 4);
     const bool sparse = idx != nullptr;
+    // full stream: an fp32 dQ accumulator (TMA reduce-adds); sparse stream: one bf16 dQ
+    // partial per (query, slot) at its list position, summed by dq_merge_kernel
+    float *dQacc = nullptr;
+    __nv_bfloat16 *dQpart = nullptr;
+    int32_t *pos = nullptr;
+    const size_t nlist = sparse ? S.BH * list_stride(S.T, S.k, S.nb) : 0;
     IndexWs W{};
     if (sparse) {
-        carve_index(S, p, W);
-        const ssa_status_t e = build_index(S, idx, W, st);
+        p = carve_index(S, p, W);
+        pos = reinterpret_cast<int32_t *>(p);
+        p += align_up(S.rows * S.k * 4);
+        dQpart = reinterpret_cast<__nv_bfloat16 *>(p);
+        const ssa_status_t e = build_index(S, idx, W, st, pos);
         if (e != SSA_OK) return e;
+    } else {
+        dQacc = reinterpret_cast<float *>(p);
     }
     const unsigned g = static_cast<unsigned>((S.rows + 7) / 8);
     bwd_prep_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16 *)dO, (const __nv_bfloat16 *)O, Dvec,
@@ -272,14 +285,14 @@ ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V,
     const int nkv = sparse ? S.s : 128;
     CUtensorMap tmK, tmV, tmQ, tmdO, tmdQ;
     if (!make_tmap(&tmK, K, S.rows, nkv) || !make_tmap(&tmV, V, S.rows, nkv) || !make_tmap(&tmQ, Q, S.rows, 128) ||
-        !make_tmap(&tmdO, dO, S.rows, 128) || !make_tmap_f32(&tmdQ, dQacc, S.rows))
+        !make_tmap(&tmdO, dO, S.rows, 128) ||
+        !(sparse ? make_tmap(&tmdQ, dQpart, nlist, 32) : make_tmap_f32(&tmdQ, dQacc, S.rows)))
         return SSA_ERR_CUDA;
     BwdArgs a{};
     a.Q = (const __nv_bfloat16 *)Q;
     a.dO = (const __nv_bfloat16 *)dO;
     a.lse = lse;
     a.Dvec = Dvec;
-    a.dQacc = dQacc;
     a.dK = (__nv_bfloat16 *)dK;
     a.dV = (__nv_bfloat16 *)dV;
     a.entries = W.entries;
@@ -303,8 +316,13 @@ ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V,
         if (!set_smem(attn_bwd_kernel<64>, sm)) return SSA_ERR_CUDA;
         attn_bwd_kernel<64><<<units, kBwdThreads, sm, st>>>(tmK, tmV, tmQ, tmdO, tmdQ, a);
     }
-    const size_t n = S.rows * S.d;
-    acc_to_out_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, st>>>(dQacc, (__nv_bfloat16 *)dQ, n, accumulate);
+    if (sparse) {
+        dq_merge_kernel<<<g, 256, 0, st>>>(pos, dQpart, (__nv_bfloat16 *)dQ, S.rows, S.T, S.k, S.nb, accumulate);
+    } else {
+        const size_t n = S.rows * S.d;
+        acc_to_out_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, st>>>(dQacc, (__nv_bfloat16 *)dQ, n,
+                                                                           accumulate);
+    }
     return launch_status();
 }
 
