@@ -346,9 +346,9 @@ def ours(args, rank, world, local_rank):
     op_flops = {"full_fwd": ff, "full_bwd": fb, "sparse_fwd": sf, "sparse_bwd": sb}
     dominant = max(op_ms, key=op_ms.get)
     # DRAM bytes per launch of the dominant kernel from one ncu capture of the same build
-    # (profiles/attn_bwd_full_long_H4.md: the 4-head case, read 221.0 MB + write 105.8 MB; heads are
+    # (profiles/attn_bwd_full_long_H4.md: the 4-head case, read 221.7 MB + write 106.3 MB; heads are
     # independent units of the grid, so traffic scales by 32/4 to the benchmarked launch).
-    traffic = (220.960512e6 + 105.816320e6) * (wl.H / 4) if dominant == "full_bwd" else None
+    traffic = (221.727488e6 + 106.342656e6) * (wl.H / 4) if dominant == "full_bwd" else None
     roof = {"kernel": "ssa_%s call" % dominant, "bound": "tensor",
             "achieved": op_flops.get(dominant, 0.0) / (op_ms[dominant] / 1e3) / 1e12, "peak": peak_sust,
             "unit": "TFLOP/s", "traffic": traffic, "traffic_unit": "DRAM bytes per launch (ncu)",
