@@ -44,6 +44,26 @@ def flops(B, H, T, d, s, k):
     return sparse_fwd, 2.5 * sparse_fwd, full_fwd, 2.5 * full_fwd
 
 
+def max_over_ranks(vals, device):
+    """Element-wise maximum of per-rank timings over every rank of the default process group.
+
+    The whole job finishes when its slowest replica does, so a job time is the max over ranks.
+    With no process group (one GPU) the values come back unchanged.
+    """
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def whole_job_tokens_per_s(tokens_per_rank, world, ms_per_step):
+    """Throughput of the whole job: the tokens every replica processed in one step over the step time."""
+    return tokens_per_rank * world / (ms_per_step / 1e3)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -328,18 +348,14 @@ def ours(args, rank, world, local_rank):
     if L.ssa_get_device_error() != L.SSA_OK:
         raise RuntimeError("device error during timing")
 
-    if dist is not None:
-        t = torch.tensor([ms, e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e_ms = float(t[0]), float(t[1])
+    ms, e_ms = max_over_ranks([ms, e_ms], dev)
     if rank != 0:
         return
 
     hbm, peak_burst, peak_sust, peak_kind = measured_peaks()
     sf, sb, ff, fb = flops(wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL)
     ms_step = ms / args.steps
-    tokens = wl.B * wl.T * world
-    value = tokens / (ms_step / 1e3)
+    value = whole_job_tokens_per_s(wl.B * wl.T, world, ms_step)
     op_ms = {name: statistics.median(v) for name, v in per_op.items()}
     sparse_ms = op_ms["sparse_fwd"] + op_ms["sparse_bwd"]
     full_ms = op_ms["full_fwd"] + op_ms["full_bwd"]
@@ -375,7 +391,7 @@ def ours(args, rank, world, local_rank):
                      "frac": (wl.B * wl.H * wl.T * 2 * wl.d) / (pool_kernel_ms / 1e3) / 1e9 / hbm,
                      "ms": pool_kernel_ms, "timing": "mean of 10 back-to-back launches"},
         "roofline": roof,
-        "e2e": {"value": tokens / (e_ms / args.steps / 1e3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_tokens_per_s(wl.B * wl.T, world, e_ms / args.steps), "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(host[k].numel() * 2 for k in host), "d2h_bytes_per_step": 4},
         "gpu_launches": args.steps * (ops.SSAStep.KERNELS_FWD + ops.SSAStep.KERNELS_BWD),
         "clocks": clocks,
