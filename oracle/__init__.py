@@ -12,10 +12,12 @@ Aligning Full and Sparse Attention Outputs in Feature Space", paperlayer.ai
 summary of v4):
   block_pool    section 3  mean-pooled block keys
   block_select  section 3  current block + top-(k-1) preceding blocks by q.Kbar
+  block_scores  section 3  the candidate scores q.Kbar of chosen rows
   attn_fwd      sections 3 full causal attention / attention over the selected
                            blocks' tokens
   attn_bwd      section 4.2 gradients; dropped keys get none
-  align_fwd/bwd section 5  bidirectional SmoothL1 output alignment
+  align_fwd/bwd section 5  bidirectional SmoothL1 output alignment; section 7.5
+                           the adjusted L2 variant (kind="l2")
   dropped_mass  section 4.2 / Appendix B  delta = 1 - exp(lse_s - lse_f)
 
 Parity pins: see tests/test_oracle_pins.py.  Every function there is pinned
@@ -56,13 +58,14 @@ def _load():
     lib.ora_num_threads.restype = ctypes.c_int
     lib.ora_block_pool.argtypes = [i64, i64, i64, i64, p, p]
     lib.ora_block_select.argtypes = [i64, i64, i64, i64, i64, p, p, p, p, p]
+    lib.ora_block_scores.argtypes = [i64, i64, i64, i64, i64, p, p, p, p, p]
     lib.ora_check_selection.argtypes = [i64, i64, i64, i64, p]
     lib.ora_check_selection.restype = ctypes.c_int
     lib.ora_attn_fwd.argtypes = [i64, i64, i64, i64, i64, dbl, p, p, p, p, i64, p, p, p]
     lib.ora_attn_bwd.argtypes = [i64, i64, i64, i64, i64, dbl, p, p, p, p, p, i64, p, i64, p, p, p, p, ctypes.c_int]
-    lib.ora_align_fwd.argtypes = [i64, p, p, dbl, dbl, dbl]
+    lib.ora_align_fwd.argtypes = [i64, p, p, dbl, dbl, dbl, ctypes.c_int]
     lib.ora_align_fwd.restype = dbl
-    lib.ora_align_bwd.argtypes = [i64, p, p, dbl, dbl, dbl, dbl, p, p]
+    lib.ora_align_bwd.argtypes = [i64, p, p, dbl, dbl, dbl, dbl, p, p, ctypes.c_int]
     _lib = lib
     return lib
 
@@ -101,6 +104,18 @@ def block_select(Q: np.ndarray, Kbar: np.ndarray, s: int, k: int) -> Tuple[np.nd
     r2 = np.empty((BH, T), dtype=np.float64)
     _load().ora_block_select(BH, T, d, s, k, _ptr(Q), _ptr(Kbar), _ptr(idx), _ptr(r1), _ptr(r2))
     return idx, r1, r2
+
+
+def block_scores(Q: np.ndarray, Kbar: np.ndarray, s: int, bh, t) -> np.ndarray:
+    """Candidate scores q_t . Kbar_j of the rows (bh[i], t[i]) -> [n, nb] (NaN for j >= b(t))."""
+    Q, Kbar = _f64(Q), _f64(Kbar)
+    BH, T, d = Q.shape
+    nb = T // s
+    bh = np.ascontiguousarray(bh, dtype=np.int64)
+    t = np.ascontiguousarray(t, dtype=np.int64)
+    out = np.empty((bh.shape[0], nb), dtype=np.float64)
+    _load().ora_block_scores(BH, T, d, s, bh.shape[0], _ptr(bh), _ptr(t), _ptr(Q), _ptr(Kbar), _ptr(out))
+    return out
 
 
 def check_selection(idx: np.ndarray, s: int) -> bool:
@@ -148,17 +163,24 @@ def attn_bwd(Q, K, V, dO, s: int, scale: float, idx: Optional[np.ndarray] = None
     return dQ, dK, dV
 
 
-def align_fwd(Of, Os, beta: float = 1.0, w_sparsity: float = 1.0, w_commit: float = 1.0) -> float:
+ALIGN_KINDS = {"smooth_l1": 0, "l2": 1}
+
+
+def align_fwd(Of, Os, beta: float = 1.0, w_sparsity: float = 1.0, w_commit: float = 1.0,
+              kind: str = "smooth_l1") -> float:
+    """Alignment loss; kind "smooth_l1" (section 5) or "l2" (the adjusted L2 variant of section 7.5)."""
     Of, Os = _f64(Of).ravel(), _f64(Os).ravel()
-    return float(_load().ora_align_fwd(Of.size, _ptr(Of), _ptr(Os), beta, w_sparsity, w_commit))
+    return float(_load().ora_align_fwd(Of.size, _ptr(Of), _ptr(Os), beta, w_sparsity, w_commit, ALIGN_KINDS[kind]))
 
 
-def align_bwd(Of, Os, beta: float = 1.0, w_sparsity: float = 1.0, w_commit: float = 1.0, g: float = 1.0):
+def align_bwd(Of, Os, beta: float = 1.0, w_sparsity: float = 1.0, w_commit: float = 1.0, g: float = 1.0,
+              kind: str = "smooth_l1"):
     shape = np.shape(Of)
     Of, Os = _f64(Of).ravel(), _f64(Os).ravel()
     dOf = np.empty_like(Of)
     dOs = np.empty_like(Os)
-    _load().ora_align_bwd(Of.size, _ptr(Of), _ptr(Os), beta, w_sparsity, w_commit, g, _ptr(dOf), _ptr(dOs))
+    _load().ora_align_bwd(Of.size, _ptr(Of), _ptr(Os), beta, w_sparsity, w_commit, g, _ptr(dOf), _ptr(dOs),
+                          ALIGN_KINDS[kind])
     return dOf.reshape(shape), dOs.reshape(shape)
 
 

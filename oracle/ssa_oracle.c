@@ -114,6 +114,32 @@ void ora_block_select(i64 BH, i64 T, i64 d, i64 s, i64 k, const double *Q, const
     }
 }
 
+/* Candidate scores of listed rows -- page section 3: every strictly preceding
+ * block j < b(t) is scored r_j = q_t . Kbar_j.  For the n (head, query) pairs
+ * (bh_list[i], t_list[i]), out[i * nb + j] = r_j for j < b(t) and NaN for the
+ * blocks that are not candidates.  Used to check that a selection which differs
+ * from block_select's on a near-tie row is still a valid top set. */
+void ora_block_scores(i64 BH, i64 T, i64 d, i64 s, i64 n, const i64 *bh_list, const i64 *t_list, const double *Q,
+                      const double *Kbar, double *out) {
+    i64 nb = T / s;
+    (void)BH;
+#pragma omp parallel for schedule(static)
+    for (i64 i = 0; i < n; ++i) {
+        i64 bh = bh_list[i], t = t_list[i], bt = t / s;
+        const double *q = Q + (bh * T + t) * d;
+        for (i64 j = 0; j < nb; ++j) {
+            if (j >= bt) {
+                out[i * nb + j] = NAN;
+                continue;
+            }
+            const double *kb = Kbar + (bh * nb + j) * d;
+            double r = 0.0;
+            for (i64 c = 0; c < d; ++c) r += q[c] * kb[c];
+            out[i * nb + j] = r;
+        }
+    }
+}
+
 /* ---------------------------------------------------------------------------
  * Attended set S(t).
  * Full attention (paper section 3: every preceding token takes part): S(t) = {0..t}.
@@ -356,21 +382,37 @@ static double huber_slope(double x, double beta) {
     return x > 0 ? 1.0 : -1.0;
 }
 
-double ora_align_fwd(i64 n, const double *of, const double *os, double beta, double w_s, double w_c) {
+/* Adjusted L2 variant -- page section 7.5 (ablation, Table 3: an "adjusted L2"
+ * alignment in place of SmoothL1; the pages do not print it).  Reading: the
+ * quadratic branch of the SmoothL1 above kept for every x,
+ *   l2adj(x) = 0.5 x^2 / beta,
+ * which equals SmoothL1 wherever |x| < beta, so the weights need no retuning. */
+static double l2adj(double x, double beta) { return 0.5 * x * x / beta; }
+
+static double l2adj_slope(double x, double beta) { return x / beta; }
+
+/* kind 0: SmoothL1 (the default of section 5); kind 1: adjusted L2. */
+static double align_elem(int kind, double x, double beta) { return kind ? l2adj(x, beta) : huber(x, beta); }
+
+static double align_slope(int kind, double x, double beta) {
+    return kind ? l2adj_slope(x, beta) : huber_slope(x, beta);
+}
+
+double ora_align_fwd(i64 n, const double *of, const double *os, double beta, double w_s, double w_c, int kind) {
     double a = 0.0, b = 0.0;
     for (i64 i = 0; i < n; ++i) {
-        a += huber(of[i] - os[i], beta);
-        b += huber(os[i] - of[i], beta);
+        a += align_elem(kind, of[i] - os[i], beta);
+        b += align_elem(kind, os[i] - of[i], beta);
     }
     return w_s * a / (double)n + w_c * b / (double)n;
 }
 
-/* dL/do_f = g * w_s * huber'(o_f - o_s) / n   (o_s is a constant in the sparsity term)
- * dL/do_s = g * w_c * huber'(o_s - o_f) / n   (o_f is a constant in the commitment term) */
+/* dL/do_f = g * w_s * loss'(o_f - o_s) / n   (o_s is a constant in the sparsity term)
+ * dL/do_s = g * w_c * loss'(o_s - o_f) / n   (o_f is a constant in the commitment term) */
 void ora_align_bwd(i64 n, const double *of, const double *os, double beta, double w_s, double w_c, double g,
-                   double *dof, double *dos) {
+                   double *dof, double *dos, int kind) {
     for (i64 i = 0; i < n; ++i) {
-        dof[i] = g * w_s * huber_slope(of[i] - os[i], beta) / (double)n;
-        dos[i] = g * w_c * huber_slope(os[i] - of[i], beta) / (double)n;
+        dof[i] = g * w_s * align_slope(kind, of[i] - os[i], beta) / (double)n;
+        dos[i] = g * w_c * align_slope(kind, os[i] - of[i], beta) / (double)n;
     }
 }

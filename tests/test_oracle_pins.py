@@ -103,6 +103,36 @@ def test_select_scale_invariance(ora):
     np.testing.assert_array_equal(a, b)
 
 
+def test_block_scores_hand_example(ora):
+    # the hand example above: q = 1, Kbar = [0.5, 3, 1, 7]; query 6 (block 3) scores blocks 0-2
+    K = np.array([0, 1, 3, 3, 1, 1, 7, 7], dtype=np.float64)[None, :, None]
+    Q = np.ones((1, 8, 1))
+    sc = ora.block_scores(Q, ora.block_pool(K, 2), 2, [0, 0], [6, 1])
+    np.testing.assert_array_equal(sc[0, :3], [0.5, 3.0, 1.0])
+    assert np.isnan(sc[0, 3]) and np.all(np.isnan(sc[1]))  # not candidates: j >= b(t)
+
+
+@pytest.mark.parametrize("s,k", [(4, 3), (8, 5)])
+def test_block_scores_rank_to_the_brute_force_selection(ora, s, k):
+    # Sorting a row's candidate scores (score desc, index asc) and keeping k-1 plus b(t) gives the
+    # brute-force selection, and ranks k-1, k are the r_(k-1), r_(k) block_select reports.
+    Q = _rand((2, 64, 6), 12)
+    K = _rand((2, 64, 6), 13)
+    Kbar = ora.block_pool(K, s)
+    idx, r1, r2 = ora.block_select(Q, Kbar, s, k)
+    brute = _brute_select(Q, K, s, k)
+    bh, t = np.meshgrid(np.arange(2), np.arange(64), indexing="ij")
+    sc = ora.block_scores(Q, Kbar, s, bh.ravel(), t.ravel())
+    for i, (b, tt) in enumerate(zip(bh.ravel(), t.ravel())):
+        bt = tt // s
+        cand = np.arange(bt)
+        order = cand[np.lexsort((cand, -sc[i, :bt]))]
+        pick = sorted(list(order[:k - 1]) + [bt])
+        np.testing.assert_array_equal(brute[b, tt, :len(pick)], pick)
+        if bt >= k:
+            assert sc[i, order[k - 2]] == r1[b, tt] and sc[i, order[k - 1]] == r2[b, tt]
+
+
 def test_check_selection_rejects_bad_rows(ora):
     good = np.array([[[0, -1], [0, 1]]], dtype=np.int32)  # T=2, s=1
     assert ora.check_selection(good, 1)
@@ -348,6 +378,29 @@ def test_align_finite_differences(ora):
             b[i, j] -= eps
             fd = (ora.align_fwd(Of, a, 1.0, 0.0, wc) - ora.align_fwd(Of, b, 1.0, 0.0, wc)) / (2 * eps)
             assert gs[i, j] == pytest.approx(fd, rel=1e-5, abs=1e-9)
+
+
+@pytest.mark.parametrize("beta,ws,wc", [(1.0, 1.0, 1.0), (0.5, 0.3, 2.0)])
+def test_align_l2_matches_torch_mse(ora, beta, ws, wc):
+    # adjusted L2 (section 7.5): 0.5 x^2 / beta for every x = mse_loss / (2 beta), both directions
+    Of, Os = _rand((2, 3, 7, 5), 51) * 2.0, _rand((2, 3, 7, 5), 52)
+    of, os_ = torch.tensor(Of, requires_grad=True), torch.tensor(Os, requires_grad=True)
+    L = (ws * F.mse_loss(of, os_.detach()) + wc * F.mse_loss(os_, of.detach())) / (2 * beta)
+    (1.3 * L).backward()
+    assert ora.align_fwd(Of, Os, beta, ws, wc, kind="l2") == pytest.approx(L.item(), rel=1e-14)
+    gf, gs = ora.align_bwd(Of, Os, beta, ws, wc, 1.3, kind="l2")
+    np.testing.assert_allclose(gf, of.grad.numpy(), rtol=1e-14, atol=1e-18)
+    np.testing.assert_allclose(gs, os_.grad.numpy(), rtol=1e-14, atol=1e-18)
+
+
+def test_align_l2_equals_smooth_l1_inside_beta(ora):
+    # the two kinds agree where every |o_f - o_s| < beta, and L2 exceeds SmoothL1 beyond it
+    Of = _rand((6, 8), 53) * 0.1
+    Os = Of + _rand((6, 8), 54) * 0.1
+    assert ora.align_fwd(Of, Os, 2.0, 1.0, 1.0, kind="l2") == pytest.approx(ora.align_fwd(Of, Os, 2.0, 1.0, 1.0),
+                                                                            rel=1e-14)
+    far = Os + 5.0
+    assert ora.align_fwd(Of, far, 1.0, 1.0, 1.0, kind="l2") > ora.align_fwd(Of, far, 1.0, 1.0, 1.0)
 
 
 # --------------------------------------------------------------------------- input generator
