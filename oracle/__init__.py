@@ -57,12 +57,13 @@ def _load():
     i64, dbl, p = ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
     lib.ora_num_threads.restype = ctypes.c_int
     lib.ora_block_pool.argtypes = [i64, i64, i64, i64, p, p]
-    lib.ora_block_select.argtypes = [i64, i64, i64, i64, i64, p, p, p, p, p]
-    lib.ora_block_scores.argtypes = [i64, i64, i64, i64, i64, p, p, p, p, p]
+    lib.ora_block_select.argtypes = [i64, i64, i64, i64, i64, i64, p, p, p, p, p]
+    lib.ora_block_scores.argtypes = [i64, i64, i64, i64, i64, i64, p, p, p, p, p]
     lib.ora_check_selection.argtypes = [i64, i64, i64, i64, p]
     lib.ora_check_selection.restype = ctypes.c_int
-    lib.ora_attn_fwd.argtypes = [i64, i64, i64, i64, i64, dbl, p, p, p, p, i64, p, p, p]
-    lib.ora_attn_bwd.argtypes = [i64, i64, i64, i64, i64, dbl, p, p, p, p, p, i64, p, i64, p, p, p, p, ctypes.c_int]
+    lib.ora_attn_fwd.argtypes = [i64, i64, i64, i64, i64, i64, dbl, p, p, p, p, i64, p, p, p]
+    lib.ora_attn_bwd.argtypes = [i64, i64, i64, i64, i64, i64, dbl, p, p, p, p, p, i64, p, i64, p, p, p, p,
+                                 ctypes.c_int]
     lib.ora_align_fwd.argtypes = [i64, p, p, dbl, dbl, dbl, ctypes.c_int]
     lib.ora_align_fwd.restype = dbl
     lib.ora_align_bwd.argtypes = [i64, p, p, dbl, dbl, dbl, dbl, p, p, ctypes.c_int]
@@ -95,26 +96,40 @@ def block_pool(K: np.ndarray, s: int) -> np.ndarray:
     return out
 
 
+def _group(nq: int, nk: int) -> int:
+    """Query heads per key/value head (grouped-query attention); 1 when the counts agree."""
+    if nk <= 0 or nq % nk:
+        raise ValueError("query heads (%d) must be a multiple of key heads (%d)" % (nq, nk))
+    return nq // nk
+
+
 def block_select(Q: np.ndarray, Kbar: np.ndarray, s: int, k: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
-    """Q [BH, T, d], Kbar [BH, nb, d] -> (idx int32 [BH,T,k], r_(k-1) [BH,T], r_(k) [BH,T])."""
+    """Q [BH, T, d], Kbar [BHk, nb, d] -> (idx int32 [BHk,T,k], r_(k-1) [BHk,T], r_(k) [BHk,T]).
+
+    With BH = G * BHk (grouped query heads), key head g's selection scores block j by the sum over its G
+    query heads of q . Kbar_j."""
     Q, Kbar = _f64(Q), _f64(Kbar)
     BH, T, d = Q.shape
-    idx = np.empty((BH, T, k), dtype=np.int32)
-    r1 = np.empty((BH, T), dtype=np.float64)
-    r2 = np.empty((BH, T), dtype=np.float64)
-    _load().ora_block_select(BH, T, d, s, k, _ptr(Q), _ptr(Kbar), _ptr(idx), _ptr(r1), _ptr(r2))
+    BHk = Kbar.shape[0]
+    G = _group(BH, BHk)
+    idx = np.empty((BHk, T, k), dtype=np.int32)
+    r1 = np.empty((BHk, T), dtype=np.float64)
+    r2 = np.empty((BHk, T), dtype=np.float64)
+    _load().ora_block_select(BHk, G, T, d, s, k, _ptr(Q), _ptr(Kbar), _ptr(idx), _ptr(r1), _ptr(r2))
     return idx, r1, r2
 
 
 def block_scores(Q: np.ndarray, Kbar: np.ndarray, s: int, bh, t) -> np.ndarray:
-    """Candidate scores q_t . Kbar_j of the rows (bh[i], t[i]) -> [n, nb] (NaN for j >= b(t))."""
+    """Candidate scores of the rows (key head bh[i], query t[i]) -> [n, nb] (NaN for j >= b(t))."""
     Q, Kbar = _f64(Q), _f64(Kbar)
     BH, T, d = Q.shape
+    BHk = Kbar.shape[0]
+    G = _group(BH, BHk)
     nb = T // s
     bh = np.ascontiguousarray(bh, dtype=np.int64)
     t = np.ascontiguousarray(t, dtype=np.int64)
     out = np.empty((bh.shape[0], nb), dtype=np.float64)
-    _load().ora_block_scores(BH, T, d, s, bh.shape[0], _ptr(bh), _ptr(t), _ptr(Q), _ptr(Kbar), _ptr(out))
+    _load().ora_block_scores(BHk, G, T, d, s, bh.shape[0], _ptr(bh), _ptr(t), _ptr(Q), _ptr(Kbar), _ptr(out))
     return out
 
 
@@ -125,9 +140,12 @@ def check_selection(idx: np.ndarray, s: int) -> bool:
 
 
 def attn_fwd(Q, K, V, s: int, scale: float, idx: Optional[np.ndarray] = None, rows=None):
-    """Full (idx None) or sparse attention forward -> (O [BH, n, d], lse [BH, n])."""
+    """Full (idx None) or sparse attention forward -> (O [BH, n, d], lse [BH, n]).
+
+    K, V (and idx) may have BH / G heads: query head bh then reads key head bh // G."""
     Q, K, V = _f64(Q), _f64(K), _f64(V)
     BH, T, d = Q.shape
+    G = _group(BH, K.shape[0])
     k = 0 if idx is None else idx.shape[-1]
     if idx is not None:
         idx = np.ascontiguousarray(idx, dtype=np.int32)
@@ -135,19 +153,21 @@ def attn_fwd(Q, K, V, s: int, scale: float, idx: Optional[np.ndarray] = None, ro
     n = T if rows is None else rows.shape[0]
     O = np.empty((BH, n, d), dtype=np.float64)
     lse = np.empty((BH, n), dtype=np.float64)
-    _load().ora_attn_fwd(BH, T, d, s, k, float(scale), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
+    _load().ora_attn_fwd(BH, G, T, d, s, k, float(scale), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
                          n, _ptr(rows), _ptr(O), _ptr(lse))
     return O, lse
 
 
 def attn_bwd(Q, K, V, dO, s: int, scale: float, idx: Optional[np.ndarray] = None, qrows=None, krows=None,
              stored_o: str = "exact"):
-    """Gradients of sum(dO * O) -> (dQ [BH, nq, d], dK [BH, nk, d], dV [BH, nk, d]).
+    """Gradients of sum(dO * O) -> (dQ [BH, nq, d], dK [BHk, nk, d], dV [BHk, nk, d]) (BHk = BH with one key
+    head per query head; grouped query heads sum into their key head).
 
     stored_o="bf16": D_t = dO_t . o_t is formed with the oracle's own output rounded to bfloat16, the value
     a backward pass is given when the forward stores its output in bfloat16; "exact" uses o_t itself."""
     Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
     BH, T, d = Q.shape
+    G = _group(BH, K.shape[0])
     k = 0 if idx is None else idx.shape[-1]
     if idx is not None:
         idx = np.ascontiguousarray(idx, dtype=np.int32)
@@ -155,9 +175,9 @@ def attn_bwd(Q, K, V, dO, s: int, scale: float, idx: Optional[np.ndarray] = None
     nq = T if qrows is None else qrows.shape[0]
     nk = T if krows is None else krows.shape[0]
     dQ = np.empty((BH, nq, d), dtype=np.float64)
-    dK = np.empty((BH, nk, d), dtype=np.float64)
-    dV = np.empty((BH, nk, d), dtype=np.float64)
-    _load().ora_attn_bwd(BH, T, d, s, k, float(scale), _ptr(Q), _ptr(K), _ptr(V), _ptr(dO), _ptr(idx),
+    dK = np.empty((BH // G, nk, d), dtype=np.float64)
+    dV = np.empty((BH // G, nk, d), dtype=np.float64)
+    _load().ora_attn_bwd(BH, G, T, d, s, k, float(scale), _ptr(Q), _ptr(K), _ptr(V), _ptr(dO), _ptr(idx),
                          nq, _ptr(qrows), nk, _ptr(krows), _ptr(dQ), _ptr(dK), _ptr(dV),
                          1 if stored_o == "bf16" else 0)
     return dQ, dK, dV

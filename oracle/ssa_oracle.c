@@ -79,8 +79,10 @@ static int ora_int_order(const void *pa, const void *pb) {
     return (a > b) - (a < b);
 }
 
-void ora_block_select(i64 BH, i64 T, i64 d, i64 s, i64 k, const double *Q, const double *Kbar,
+void ora_block_select(i64 BH, i64 G, i64 T, i64 d, i64 s, i64 k, const double *Q, const double *Kbar,
                       int32_t *idx, double *r_km1, double *r_k) {
+    /* BH key/value heads, each shared by the G consecutive query heads of its group (G = 1: one query head
+     * per key head); the group's score of block j is the sum of its query heads' scores. */
     i64 nb = T / s;
 #pragma omp parallel
     {
@@ -89,12 +91,14 @@ void ora_block_select(i64 BH, i64 T, i64 d, i64 s, i64 k, const double *Q, const
 #pragma omp for collapse(2) schedule(dynamic, 64)
         for (i64 bh = 0; bh < BH; ++bh) {
             for (i64 t = 0; t < T; ++t) {
-                const double *q = Q + (bh * T + t) * d;
                 i64 bt = t / s;
                 for (i64 j = 0; j < bt; ++j) {
                     const double *kb = Kbar + (bh * nb + j) * d;
                     double r = 0.0;
-                    for (i64 c = 0; c < d; ++c) r += q[c] * kb[c];
+                    for (i64 g = 0; g < G; ++g) {
+                        const double *q = Q + ((bh * G + g) * T + t) * d;
+                        for (i64 c = 0; c < d; ++c) r += q[c] * kb[c];
+                    }
                     cand[j].score = r;
                     cand[j].j = (int32_t)j;
                 }
@@ -117,16 +121,16 @@ void ora_block_select(i64 BH, i64 T, i64 d, i64 s, i64 k, const double *Q, const
 /* Candidate scores of listed rows -- page section 3: every strictly preceding
  * block j < b(t) is scored r_j = q_t . Kbar_j.  For the n (head, query) pairs
  * (bh_list[i], t_list[i]), out[i * nb + j] = r_j for j < b(t) and NaN for the
- * blocks that are not candidates.  Used to check that a selection which differs
- * from block_select's on a near-tie row is still a valid top set. */
-void ora_block_scores(i64 BH, i64 T, i64 d, i64 s, i64 n, const i64 *bh_list, const i64 *t_list, const double *Q,
-                      const double *Kbar, double *out) {
+ * blocks that are not candidates (bh_list names key/value heads; with G > 1 the
+ * score is the group's sum, as in block_select).  Used to check that a selection
+ * which differs from block_select's on a near-tie row is still a valid top set. */
+void ora_block_scores(i64 BH, i64 G, i64 T, i64 d, i64 s, i64 n, const i64 *bh_list, const i64 *t_list,
+                      const double *Q, const double *Kbar, double *out) {
     i64 nb = T / s;
     (void)BH;
 #pragma omp parallel for schedule(static)
     for (i64 i = 0; i < n; ++i) {
         i64 bh = bh_list[i], t = t_list[i], bt = t / s;
-        const double *q = Q + (bh * T + t) * d;
         for (i64 j = 0; j < nb; ++j) {
             if (j >= bt) {
                 out[i * nb + j] = NAN;
@@ -134,7 +138,10 @@ void ora_block_scores(i64 BH, i64 T, i64 d, i64 s, i64 n, const i64 *bh_list, co
             }
             const double *kb = Kbar + (bh * nb + j) * d;
             double r = 0.0;
-            for (i64 c = 0; c < d; ++c) r += q[c] * kb[c];
+            for (i64 g = 0; g < G; ++g) {
+                const double *q = Q + ((bh * G + g) * T + t) * d;
+                for (i64 c = 0; c < d; ++c) r += q[c] * kb[c];
+            }
             out[i * nb + j] = r;
         }
     }
@@ -212,8 +219,11 @@ static double attend_row(i64 d, i64 s, i64 k, double scale, const double *Qh, co
 
 /* Forward for the query rows listed in rows[0..nrows) of every head (rows == NULL:
  * all T rows).  O is [BH, nrows, d], lse is [BH, nrows].  idx == NULL selects full
- * causal attention, otherwise the sparse stream over the given selection. */
-void ora_attn_fwd(i64 BH, i64 T, i64 d, i64 s, i64 k, double scale, const double *Q, const double *K,
+ * causal attention, otherwise the sparse stream over the given selection.  Query
+ * head bh reads key/value head bh / G (grouped-query attention; G = 1 for one key
+ * head per query head) and, in the sparse stream, that key head's selection:
+ * K, V are [BH / G, T, d], idx is [BH / G, T, k]. */
+void ora_attn_fwd(i64 BH, i64 G, i64 T, i64 d, i64 s, i64 k, double scale, const double *Q, const double *K,
                   const double *V, const int32_t *idx, i64 nrows, const i64 *rows, double *O, double *lse) {
     i64 n = rows ? nrows : T;
 #pragma omp parallel
@@ -223,8 +233,9 @@ void ora_attn_fwd(i64 BH, i64 T, i64 d, i64 s, i64 k, double scale, const double
         for (i64 bh = 0; bh < BH; ++bh) {
             for (i64 r = 0; r < n; ++r) {
                 i64 t = rows ? rows[r] : r;
-                const int32_t *sel_row = idx ? idx + (bh * T + t) * k : NULL;
-                lse[bh * n + r] = attend_row(d, s, k, scale, Q + bh * T * d, K + bh * T * d, V + bh * T * d,
+                const i64 kh = bh / G; /* key/value head (and selection) of query head bh */
+                const int32_t *sel_row = idx ? idx + (kh * T + t) * k : NULL;
+                lse[bh * n + r] = attend_row(d, s, k, scale, Q + bh * T * d, K + kh * T * d, V + kh * T * d,
                                              sel_row, t, O + (bh * n + r) * d, pos);
             }
         }
@@ -242,7 +253,8 @@ void ora_attn_fwd(i64 BH, i64 T, i64 d, i64 s, i64 k, double scale, const double
  *   dK_u = scale * sum_{t : u in S(t)} P_tu (dP_tu - D_t) q_t
  *   dV_u = sum_{t : u in S(t)} P_tu dO_t
  * Computes dQ for query rows qrows[0..nq) and dK, dV for key rows krows[0..nk)
- * (NULL: all rows); outputs are [BH, nq, d] and [BH, nk, d].
+ * (NULL: all rows); outputs are [BH, nq, d] and [BH / G, nk, d]: with grouped
+ * query heads (G > 1) a key head's gradients sum over the G query heads reading it.
  * ------------------------------------------------------------------------- */
 /* x rounded to the nearest bfloat16 value (8 significant bits, ties to even), as a forward output
  * stored in bfloat16 holds it. */
@@ -255,18 +267,18 @@ static double round_bf16(double x) {
 
 /* round_o != 0: D_t = dO_t . o_t uses o_t rounded to bfloat16 -- the value a backward pass receives
  * when the forward stores its output in bfloat16 (the backward takes the stored output as input). */
-void ora_attn_bwd(i64 BH, i64 T, i64 d, i64 s, i64 k, double scale, const double *Q, const double *K,
+void ora_attn_bwd(i64 BH, i64 G, i64 T, i64 d, i64 s, i64 k, double scale, const double *Q, const double *K,
                   const double *V, const double *dO, const int32_t *idx, i64 nq, const i64 *qrows, i64 nk,
                   const i64 *krows, double *dQ, double *dK, double *dV, int round_o) {
-    i64 nQ = qrows ? nq : T, nK = krows ? nk : T;
+    i64 nQ = qrows ? nq : T, nK = krows ? nk : T, BHk = BH / G;
     double *lse = (double *)malloc(sizeof(double) * (size_t)(BH * T));
     double *Dt = (double *)malloc(sizeof(double) * (size_t)(BH * T));
     i64 *kslot = (i64 *)malloc(sizeof(i64) * (size_t)T); /* key position -> output row, or -1 */
     for (i64 u = 0; u < T; ++u) kslot[u] = krows ? -1 : u;
     if (krows)
         for (i64 r = 0; r < nK; ++r) kslot[krows[r]] = r;
-    memset(dK, 0, sizeof(double) * (size_t)(BH * nK * d));
-    memset(dV, 0, sizeof(double) * (size_t)(BH * nK * d));
+    memset(dK, 0, sizeof(double) * (size_t)(BHk * nK * d));
+    memset(dV, 0, sizeof(double) * (size_t)(BHk * nK * d));
 
     /* Forward over every row: LSE_t and D_t = dO_t . o_t. */
 #pragma omp parallel
@@ -276,9 +288,10 @@ void ora_attn_bwd(i64 BH, i64 T, i64 d, i64 s, i64 k, double scale, const double
 #pragma omp for collapse(2) schedule(dynamic, 16)
         for (i64 bh = 0; bh < BH; ++bh) {
             for (i64 t = 0; t < T; ++t) {
-                const int32_t *sel_row = idx ? idx + (bh * T + t) * k : NULL;
+                const i64 kh = bh / G;
+                const int32_t *sel_row = idx ? idx + (kh * T + t) * k : NULL;
                 lse[bh * T + t] =
-                    attend_row(d, s, k, scale, Q + bh * T * d, K + bh * T * d, V + bh * T * d, sel_row, t, o, pos);
+                    attend_row(d, s, k, scale, Q + bh * T * d, K + kh * T * d, V + kh * T * d, sel_row, t, o, pos);
                 double acc = 0.0;
                 for (i64 c = 0; c < d; ++c) acc += dO[(bh * T + t) * d + c] * (round_o ? round_bf16(o[c]) : o[c]);
                 Dt[bh * T + t] = acc;
@@ -295,14 +308,14 @@ void ora_attn_bwd(i64 BH, i64 T, i64 d, i64 s, i64 k, double scale, const double
 #pragma omp for collapse(2) schedule(dynamic, 16)
         for (i64 bh = 0; bh < BH; ++bh) {
             for (i64 r = 0; r < nQ; ++r) {
-                i64 t = qrows ? qrows[r] : r;
+                i64 t = qrows ? qrows[r] : r, kh = bh / G;
                 const double *q = Q + (bh * T + t) * d, *g = dO + (bh * T + t) * d;
-                const int32_t *sel_row = idx ? idx + (bh * T + t) * k : NULL;
+                const int32_t *sel_row = idx ? idx + (kh * T + t) * k : NULL;
                 double *out = dQ + (bh * nQ + r) * d;
                 for (i64 c = 0; c < d; ++c) out[c] = 0.0;
                 i64 n = attended_set(sel_row, k, s, t, pos);
                 for (i64 a = 0; a < n; ++a) {
-                    const double *ku = K + (bh * T + pos[a]) * d, *vu = V + (bh * T + pos[a]) * d;
+                    const double *ku = K + (kh * T + pos[a]) * d, *vu = V + (kh * T + pos[a]) * d;
                     double x = 0.0, dp = 0.0;
                     for (i64 c = 0; c < d; ++c) {
                         x += q[c] * ku[c];
@@ -317,23 +330,24 @@ void ora_attn_bwd(i64 BH, i64 T, i64 d, i64 s, i64 k, double scale, const double
         free(pos);
     }
 
-    /* dK, dV rows: every query scatters into the keys of S(t); each thread keeps
-     * its own accumulators, summed at the end. */
-    for (i64 bh = 0; bh < BH; ++bh) {
+    /* dK, dV rows: every query of every head of a key head's group scatters into the keys of
+     * S(t); each thread keeps its own accumulators, summed at the end. */
+    for (i64 kh = 0; kh < BHk; ++kh) {
 #pragma omp parallel
         {
             i64 *pos = (i64 *)malloc(sizeof(i64) * (size_t)T);
             double *ak = (double *)calloc((size_t)(nK * d), sizeof(double));
             double *av = (double *)calloc((size_t)(nK * d), sizeof(double));
 #pragma omp for schedule(dynamic, 16)
-            for (i64 t = 0; t < T; ++t) {
-                const int32_t *sel_row = idx ? idx + (bh * T + t) * k : NULL;
+            for (i64 gt = 0; gt < G * T; ++gt) {
+                const i64 bh = kh * G + gt / T, t = gt % T;
+                const int32_t *sel_row = idx ? idx + (kh * T + t) * k : NULL;
                 const double *q = Q + (bh * T + t) * d, *g = dO + (bh * T + t) * d;
                 i64 n = attended_set(sel_row, k, s, t, pos);
                 for (i64 a = 0; a < n; ++a) {
                     i64 r = kslot[pos[a]];
                     if (r < 0) continue;
-                    const double *ku = K + (bh * T + pos[a]) * d, *vu = V + (bh * T + pos[a]) * d;
+                    const double *ku = K + (kh * T + pos[a]) * d, *vu = V + (kh * T + pos[a]) * d;
                     double x = 0.0, dp = 0.0;
                     for (i64 c = 0; c < d; ++c) {
                         x += q[c] * ku[c];
@@ -350,8 +364,8 @@ void ora_attn_bwd(i64 BH, i64 T, i64 d, i64 s, i64 k, double scale, const double
 #pragma omp critical
             {
                 for (i64 e = 0; e < nK * d; ++e) {
-                    dK[bh * nK * d + e] += ak[e];
-                    dV[bh * nK * d + e] += av[e];
+                    dK[kh * nK * d + e] += ak[e];
+                    dV[kh * nK * d + e] += av[e];
                 }
             }
             free(pos);

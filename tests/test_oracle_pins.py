@@ -338,6 +338,77 @@ def test_bwd_row_subsets(ora):
     np.testing.assert_allclose(sub[2], full[2][:, kr], rtol=0, atol=1e-14)
 
 
+# --------------------------------------------------------------------------- grouped-query attention
+
+def _grouped_inputs(G, BHk=2, T=64, d=6, seed=60):
+    Q = _rand((BHk * G, T, d), seed)
+    K = _rand((BHk, T, d), seed + 1)
+    V = _rand((BHk, T, d), seed + 2)
+    dO = _rand((BHk * G, T, d), seed + 3)
+    return Q, K, V, dO
+
+
+@pytest.mark.parametrize("G,s,k", [(2, 4, 3), (4, 8, 2), (3, 4, 16)])
+def test_grouped_select_brute_force(ora, G, s, k):
+    # a key head's selection ranks blocks by the sum of its G query heads' scores
+    Q, K, _, _ = _grouped_inputs(G)
+    Kbar = ora.block_pool(K, s)
+    idx, _, _ = ora.block_select(Q, Kbar, s, k)
+    BHk, T = K.shape[0], K.shape[1]
+    means = np.stack([K[:, j * s:(j + 1) * s].mean(axis=1) for j in range(T // s)], axis=1)
+    scores = np.einsum("gitd,gjd->gtj", Q.reshape(BHk, G, T, -1), means)
+    for b in range(BHk):
+        for t in range(T):
+            bt = t // s
+            cand = np.arange(bt)
+            pick = sorted(list(cand[np.lexsort((cand, -scores[b, t, :bt]))][:k - 1]) + [bt])
+            np.testing.assert_array_equal(idx[b, t, :len(pick)], pick)
+    assert ora.check_selection(idx, s)
+
+
+@pytest.mark.parametrize("G", [2, 4])
+def test_grouped_full_attention_matches_sdpa_and_autograd(ora, G):
+    # grouped-query attention is attention with each key/value head repeated for its G query heads
+    Q, K, V, dO = _grouped_inputs(G)
+    T, scale = Q.shape[1], 0.4
+    mask = np.broadcast_to(np.tril(np.ones((T, T), dtype=bool)), (Q.shape[0], T, T))
+    O, lse = ora.attn_fwd(Q, K, V, 4, scale)
+    Kr, Vr = np.repeat(K, G, axis=0), np.repeat(V, G, axis=0)
+    ref = F.scaled_dot_product_attention(torch.tensor(Q), torch.tensor(Kr), torch.tensor(Vr), is_causal=True,
+                                         scale=scale).numpy()
+    np.testing.assert_allclose(O, ref, rtol=0, atol=1e-12)
+    dq, dk, dv = ora.attn_bwd(Q, K, V, dO, 4, scale)
+    q, kk, vv = (torch.tensor(a, requires_grad=True) for a in (Q, K, V))
+    o = F.scaled_dot_product_attention(q, kk.repeat_interleave(G, dim=0), vv.repeat_interleave(G, dim=0),
+                                       is_causal=True, scale=scale)
+    (o * torch.from_numpy(dO)).sum().backward()
+    for got, want in ((dq, q.grad), (dk, kk.grad), (dv, vv.grad)):
+        np.testing.assert_allclose(got, want.numpy(), rtol=0, atol=1e-11)
+    assert dk.shape == K.shape and dv.shape == V.shape
+
+
+@pytest.mark.parametrize("G,s,k", [(2, 4, 2), (4, 8, 3)])
+def test_grouped_sparse_attention_matches_dense_mask(ora, G, s, k):
+    # every query head of a group attends over its key head's selection
+    Q, K, V, dO = _grouped_inputs(G)
+    T, scale = Q.shape[1], 0.7
+    idx, _, _ = ora.block_select(Q, ora.block_pool(K, s), s, k)
+    mask = np.repeat(_dense_mask(idx, T, s), G, axis=0)
+    Kr, Vr = np.repeat(K, G, axis=0), np.repeat(V, G, axis=0)
+    O, lse = ora.attn_fwd(Q, K, V, s, scale, idx)
+    O_ref, lse_ref = _dense_attn(Q, Kr, Vr, mask, scale)
+    np.testing.assert_allclose(O, O_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-12)
+    dq, dk, dv = ora.attn_bwd(Q, K, V, dO, s, scale, idx)
+    q, kk, vv = (torch.tensor(a, requires_grad=True) for a in (Q, K, V))
+    x = torch.einsum("btd,bud->btu", q, kk.repeat_interleave(G, dim=0)) * scale
+    x = x.masked_fill(~torch.from_numpy(mask), -float("inf"))
+    o = torch.einsum("btu,bud->btd", torch.softmax(x, dim=-1), vv.repeat_interleave(G, dim=0))
+    (o * torch.from_numpy(dO)).sum().backward()
+    for got, want in ((dq, q.grad), (dk, kk.grad), (dv, vv.grad)):
+        np.testing.assert_allclose(got, want.numpy(), rtol=0, atol=1e-11)
+
+
 # --------------------------------------------------------------------------- alignment loss
 
 @pytest.mark.parametrize("beta,ws,wc", [(1.0, 1.0, 1.0), (0.5, 0.3, 2.0)])
