@@ -3,11 +3,16 @@
 
 One step = one pass of the whole path over one batch of the 32K-context
 workload (B=1, H=32, T=32768, d=128, s=128, k=16, bf16, sink block):
-  block pooling, causal top-k selection, full causal attention forward,
-  sparse attention forward, alignment loss forward, alignment backward (the
-  main stream -- full on even steps, sparse on odd steps -- also receives its
-  upstream gradient), full attention backward and sparse attention backward
-  accumulating into one set of dQ, dK, dV.
+  block pooling, causal top-k selection, inverse selection index, full causal
+  attention forward, sparse attention forward, alignment loss forward,
+  alignment backward (the main stream -- full on even steps, sparse on odd
+  steps -- also receives its upstream gradient), full attention backward and
+  sparse attention backward accumulating into one set of dQ, dK, dV.
+
+The metric is the sparse attention's forward + backward throughput: `value` is
+tokens/s of the sparse stream's calls (inverse index, forward, backward), timed
+with CUDA events around those calls inside the timed region of whole steps; the
+whole step's time and every call's time come from the same timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -34,6 +39,9 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse-attn fwd+bwd TFLOP/s & tokens/s at 32K ctx; % of bf16 tensor peak"
 WORKLOAD = "long"
 K_SEL = 16
+# DRAM bytes (read + write) of one attn_bwd_kernel launch of the full stream on the 4-head case of the
+# 32K workload, from an ncu capture of the current kernel; None until one exists.
+FULL_BWD_DRAM_BYTES_H4 = None
 
 
 def flops(B, H, T, d, s, k):
@@ -117,10 +125,11 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def oracle_sample(T_sample: int, seed_rows: int = 0):
-    """Run the oracle's whole step on a prefix sample: head (0,0), first T_sample tokens.
+def oracle_sample(T_sample: int):
+    """Run the oracle's sparse path on a prefix sample: head (0,0), first T_sample tokens.
 
-    Returns (seconds, sample FLOPs by the same algorithmic count, description)."""
+    The sparse path is what the metric times: pooling, selection, sparse attention forward and backward.
+    Returns (seconds, sample FLOPs of sparse fwd + bwd by the metric's count, description)."""
     import oracle
     from block_top_sparse_b200 import inputs
     wl = inputs.WORKLOADS[WORKLOAD]
@@ -130,26 +139,24 @@ def oracle_sample(T_sample: int, seed_rows: int = 0):
     t0 = time.perf_counter()
     Kbar = oracle.block_pool(f["K"], s)
     idx, _, _ = oracle.block_select(f["Q"], Kbar, s, k)
-    Of, lf = oracle.attn_fwd(f["Q"], f["K"], f["V"], s, scale)
-    Os, ls = oracle.attn_fwd(f["Q"], f["K"], f["V"], s, scale, idx)
-    oracle.align_fwd(Of, Os)
-    gf, gs = oracle.align_bwd(Of, Os)
-    oracle.attn_bwd(f["Q"], f["K"], f["V"], f["dO"] + gf, s, scale)
-    oracle.attn_bwd(f["Q"], f["K"], f["V"], gs, s, scale, idx)
+    oracle.attn_fwd(f["Q"], f["K"], f["V"], s, scale, idx)
+    oracle.attn_bwd(f["Q"], f["K"], f["V"], f["dO"], s, scale, idx)
     dt = time.perf_counter() - t0
-    fl = sum(flops(1, 1, T_sample, wl.d, s, k))
-    return dt, fl, "head (b=0,h=0), first %d of %d tokens, whole step (pool, select, full+sparse fwd, align fwd/bwd, full+sparse bwd)" % (T_sample, wl.T)
+    sf, sb, _, _ = flops(1, 1, T_sample, wl.d, s, k)
+    return dt, sf + sb, ("head (b=0,h=0), first %d of %d tokens: pool, select, sparse attention fwd + bwd; "
+                         "extrapolated to the full workload by the sparse fwd+bwd FLOP count" % (T_sample, wl.T))
 
 
 def reference_arm(args, rank):
-    """The oracle as it stands on the host cores; throughput scaled to the full workload by FLOPs."""
+    """The oracle as it stands on the host cores, on the metric's quantity (sparse attention fwd + bwd
+    tokens/s), extrapolated from a prefix sample to the full workload by FLOPs."""
     if rank != 0:
         return
     import oracle
     from block_top_sparse_b200 import inputs
     oracle.build()
     wl = inputs.WORKLOADS[WORKLOAD]
-    full_fl = sum(flops(wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL))
+    sf, sb, _, _ = flops(wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL)
     T_sample = args.ref_tokens
     for _ in range(args.warmup):
         oracle_sample(T_sample)
@@ -157,15 +164,15 @@ def reference_arm(args, rank):
     for _ in range(args.steps):
         dt, fl, desc = oracle_sample(T_sample)
         times.append(dt)
-    est = sum(times) / len(times) * full_fl / fl  # seconds for one full step
+    est = sum(times) / len(times) * (sf + sb) / fl  # seconds for the full workload's sparse fwd + bwd
     tok_s = wl.B * wl.T / est
     line = {"metric": METRIC, "value": tok_s, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_block(wl),
             "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-                             "sample": desc + "; time per sample %.2f s, scaled to the full step by algorithmic FLOPs"
-                             % (sum(times) / len(times))},
+                             "sample": desc + "; time per sample %.2f s" % (sum(times) / len(times)),
+                             "extrapolated": True},
             "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -192,7 +199,7 @@ def sweep(args):
     Q, K, V = dev["Q"], dev["K"], dev["V"]
     B, H, T, d, s = wl.B, wl.H, wl.T, wl.d, wl.s
     dims0 = L.make_dims(B, H, T, d, s, 1)
-    Of, lf = ops.attn_fwd(dims0, Q, K, V)
+    Of, lf, _ = ops.attn_fwd(dims0, Q, K, V)
     vmax = torch.linalg.vector_norm(V.float(), dim=-1).amax(dim=-1, keepdim=True)
     for k in (4, 8, 16, 32, 64):
         dims = L.make_dims(B, H, T, d, s, k)
@@ -200,6 +207,7 @@ def sweep(args):
         Os = torch.empty_like(Q)
         lse = torch.empty(B, H, T, dtype=torch.float32, device=Q.device)
         ws = ops._ws(dims, L.SSA_OP_SPARSE_FWD, Q.device)
+        # the call builds its own inverse index: the timed forward includes it
         call = lambda: L.ssa_sparse_attn_fwd(dims, Q, K, V, idx, Os, lse, ws)
         for _ in range(args.warmup):
             call()
@@ -230,7 +238,10 @@ def config_block(wl):
                         % (wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL),
             "B": wl.B, "H": wl.H, "T": wl.T, "d": wl.d, "s": wl.s, "k": K_SEL, "global_batch": wl.B, "seq_len": wl.T,
             "parallelism": "replicas", "main_stream": "alternating full/sparse per step",
-            "l2": "inputs larger than L2 (Q, K, V, dO 268 MB each)"}
+            "l2": "inputs larger than L2 (Q, K, V, dO 268 MB each)",
+            "value_is": "sparse attention fwd+bwd tokens/s (inverse index + forward + backward calls, CUDA events "
+                        "inside the timed region)",
+            "gradients": "fp32 dQ, dK, dV (both streams summed in fp32); bf16 inputs and outputs"}
 
 
 def ours(args, rank, world, local_rank):
@@ -249,45 +260,48 @@ def ours(args, rank, world, local_rank):
         host[key] = t.pin_memory()
     d = {key: host[key].to(dev, non_blocking=False) for key in host}
     dims = L.make_dims(wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL, dtype="bf16")
-    steps = [ops.SSAStep(dims, device=dev, main="full"), ops.SSAStep(dims, device=dev, main="sparse")]
+    # fp32 gradients: the two streams' contributions to dQ, dK, dV are summed without rounding the first
+    steps = [ops.SSAStep(dims, device=dev, main="full", grad_fp32=True),
+             ops.SSAStep(dims, device=dev, main="sparse", grad_fp32=True)]
+    G32 = L.SSA_BWD_GRAD_FP32
     # the two steps share no buffers: allocate once, reuse alternately
     stream = torch.cuda.current_stream(dev)
 
-    ev = {name: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for name in ("pool", "select", "full_fwd", "sparse_fwd", "align_fwd", "align_bwd", "full_bwd", "sparse_bwd")}
-    per_op = {name: [] for name in ev}
+    names = ("pool", "select", "index", "full_fwd", "sparse_fwd", "align_fwd", "align_bwd", "full_bwd", "sparse_bwd")
+    n_ev = max(args.steps, 1)
+    ev = {name: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
+          for name in names}
 
-    def run_step(i, timed_ops=False):
+    def run_step(i, timed=False):
         st = steps[i % 2]
         Q, K, V = d["Q"], d["K"], d["V"]
         dd = st.dims
 
         def rec(name, fn):
-            if timed_ops:
-                ev[name][0].record(stream)
+            if timed:
+                ev[name][i][0].record(stream)
             fn()
-            if timed_ops:
-                ev[name][1].record(stream)
+            if timed:
+                ev[name][i][1].record(stream)
 
         rec("pool", lambda: L.ssa_block_pool(dd, K, st.Kbar))
         rec("select", lambda: L.ssa_block_select(dd, Q, st.Kbar, st.idx))
-        rec("full_fwd", lambda: L.ssa_full_attn_fwd(dd, Q, K, V, st.Of, st.lse_f, st.ws[L.SSA_OP_FULL_FWD]))
+        rec("index", lambda: L.ssa_sparse_index(dd, st.idx, st.index))
+        rec("full_fwd", lambda: L.ssa_full_attn_fwd(dd, Q, K, V, st.Of, st.lse_f, st.ws[L.SSA_OP_FULL_FWD],
+                                                    O_lo=st.Of_lo))
         rec("sparse_fwd", lambda: L.ssa_sparse_attn_fwd(dd, Q, K, V, st.idx, st.Os, st.lse_s,
-                                                        st.ws[L.SSA_OP_SPARSE_FWD]))
+                                                        st.ws[L.SSA_OP_SPARSE_FWD], O_lo=st.Os_lo, index=st.index))
         rec("align_fwd", lambda: L.ssa_align_loss_fwd(dd, st.Of, st.Os, 1.0, 1.0, 1.0, st.loss,
                                                       st.ws[L.SSA_OP_ALIGN_FWD]))
         st.main_grad_buffer().copy_(d["dO"], non_blocking=True)  # upstream gradient of the main stream
         acc = L.SSA_ACC_OF if st.main == "full" else L.SSA_ACC_OS
         rec("align_bwd", lambda: L.ssa_align_loss_bwd(dd, st.Of, st.Os, 1.0, 1.0, 1.0, st.dloss, st.dOf, st.dOs,
                                                       acc))
-        rec("full_bwd", lambda: L.ssa_full_attn_bwd(dd, Q, K, V, st.Of, st.lse_f, st.dOf, st.dQ, st.dK, st.dV, 0,
-                                                    st.ws[L.SSA_OP_FULL_BWD]))
+        rec("full_bwd", lambda: L.ssa_full_attn_bwd(dd, Q, K, V, st.Of, st.lse_f, st.dOf, st.dQ, st.dK, st.dV, G32,
+                                                    st.ws[L.SSA_OP_FULL_BWD], O_lo=st.Of_lo))
         rec("sparse_bwd", lambda: L.ssa_sparse_attn_bwd(dd, Q, K, V, st.Os, st.lse_s, st.dOs, st.idx, st.dQ, st.dK,
-                                                        st.dV, 1, st.ws[L.SSA_OP_SPARSE_BWD]))
-        if timed_ops:
-            torch.cuda.synchronize(dev)
-            for name, (a, b) in ev.items():
-                per_op[name].append(a.elapsed_time(b))
+                                                        st.dV, L.SSA_BWD_ACCUMULATE | G32,
+                                                        st.ws[L.SSA_OP_SPARSE_BWD], O_lo=st.Os_lo, index=st.index))
 
     dist = None
     if world > 1:
@@ -303,35 +317,38 @@ def ours(args, rank, world, local_rank):
     if L.ssa_get_device_error() != L.SSA_OK:
         raise RuntimeError("device error during warm-up")
 
-    # ---- timed region: K whole steps, inputs resident in HBM ----
+    # ---- timed region: K whole steps, inputs resident in HBM; every call bracketed by events ----
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
         barrier()
         torch.cuda.synchronize(dev)
         start.record(stream)
         for i in range(args.steps):
-            run_step(i)
+            run_step(i, timed=True)
         end.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
     ms = start.elapsed_time(end)
     clocks = clk.summary()
+    op_ms_sum = {name: sum(a.elapsed_time(b) for a, b in ev[name][:args.steps]) for name in names}
+    sparse_ms_sum = op_ms_sum["index"] + op_ms_sum["sparse_fwd"] + op_ms_sum["sparse_bwd"]
 
-    # ---- per-op breakdown (separate, untimed-for-value pass) ----
-    for i in range(max(2, min(args.steps, 4))):
-        run_step(i, timed_ops=True)
-    # Pooling bandwidth from back-to-back launches: the events around the first call of a step
-    # also hold the host's launch latency.  K (268 MB) exceeds L2, so every launch streams it from HBM.
+    # Pooling bandwidth from back-to-back launches (also reported from the in-step events above).
+    # K (268 MB) exceeds L2, so every launch streams it from HBM.
     pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     pa.record(stream)
     for _ in range(10):
         L.ssa_block_pool(steps[0].dims, d["K"], steps[0].Kbar)
     pb.record(stream)
     torch.cuda.synchronize(dev)
-    pool_kernel_ms = pa.elapsed_time(pb) / 10
+    pool_b2b_ms = pa.elapsed_time(pb) / 10
 
-    # ---- end to end: pinned host inputs -> device, step, loss back to host ----
-    loss_host = torch.empty((), dtype=torch.float32).pin_memory()
+    # ---- end to end, through the same calls with host buffers: each step copies Q, K, V, dO from pinned
+    # host memory, runs the sparse path (pool, select, index, sparse forward, sparse backward) and copies
+    # its results O, dQ, dK, dV back to pinned host memory ----
+    out_host = {"O": torch.empty_like(host["Q"]).pin_memory()}
+    out_host.update({key: torch.empty(host["Q"].shape, dtype=torch.float32).pin_memory() for key in ("dQ", "dK", "dV")})
+    st0 = steps[1]
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
@@ -339,8 +356,16 @@ def ours(args, rank, world, local_rank):
     for i in range(args.steps):
         for key in ("Q", "K", "V", "dO"):
             d[key].copy_(host[key], non_blocking=True)
-        run_step(i)
-        loss_host.copy_(steps[i % 2].loss, non_blocking=True)
+        dd = st0.dims
+        L.ssa_block_pool(dd, d["K"], st0.Kbar)
+        L.ssa_block_select(dd, d["Q"], st0.Kbar, st0.idx)
+        L.ssa_sparse_index(dd, st0.idx, st0.index)
+        L.ssa_sparse_attn_fwd(dd, d["Q"], d["K"], d["V"], st0.idx, st0.Os, st0.lse_s, st0.ws[L.SSA_OP_SPARSE_FWD],
+                              O_lo=st0.Os_lo, index=st0.index)
+        L.ssa_sparse_attn_bwd(dd, d["Q"], d["K"], d["V"], st0.Os, st0.lse_s, d["dO"], st0.idx, st0.dQ, st0.dK,
+                              st0.dV, G32, st0.ws[L.SSA_OP_SPARSE_BWD], O_lo=st0.Os_lo, index=st0.index)
+        for key, src in (("O", st0.Os), ("dQ", st0.dQ), ("dK", st0.dK), ("dV", st0.dV)):
+            out_host[key].copy_(src, non_blocking=True)
     e_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -348,51 +373,59 @@ def ours(args, rank, world, local_rank):
     if L.ssa_get_device_error() != L.SSA_OK:
         raise RuntimeError("device error during timing")
 
-    ms, e_ms = max_over_ranks([ms, e_ms], dev)
+    ms, e_ms, sparse_ms_sum = max_over_ranks([ms, e_ms, sparse_ms_sum], dev)
     if rank != 0:
         return
 
     hbm, peak_burst, peak_sust, peak_kind = measured_peaks()
     sf, sb, ff, fb = flops(wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL)
     ms_step = ms / args.steps
-    value = whole_job_tokens_per_s(wl.B * wl.T, world, ms_step)
-    op_ms = {name: statistics.median(v) for name, v in per_op.items()}
-    sparse_ms = op_ms["sparse_fwd"] + op_ms["sparse_bwd"]
+    sparse_ms = sparse_ms_sum / args.steps
+    value = whole_job_tokens_per_s(wl.B * wl.T, world, sparse_ms)
+    op_ms = {name: v / args.steps for name, v in op_ms_sum.items()}
     full_ms = op_ms["full_fwd"] + op_ms["full_bwd"]
     op_flops = {"full_fwd": ff, "full_bwd": fb, "sparse_fwd": sf, "sparse_bwd": sb}
-    dominant = max(op_ms, key=op_ms.get)
-    # DRAM bytes per launch of the dominant kernel from one ncu capture of the same build
-    # (profiles/attn_bwd_full_long_H4.md: the 4-head case, read 221.7 MB + write 106.3 MB; heads are
-    # independent units of the grid, so traffic scales by 32/4 to the benchmarked launch).
-    traffic = (221.727488e6 + 106.342656e6) * (wl.H / 4) if dominant == "full_bwd" else None
-    roof = {"kernel": "ssa_%s call" % dominant, "bound": "tensor",
-            "achieved": op_flops.get(dominant, 0.0) / (op_ms[dominant] / 1e3) / 1e12, "peak": peak_sust,
+    # Dominant call of the step: the full-attention backward.  DRAM bytes per launch of its kernel from
+    # one ncu capture of this build on the 4-head case of the same workload (heads are independent units
+    # of the grid, so the traffic scales by 32/4 to the benchmarked launch); None when no capture of the
+    # current kernel exists.
+    traffic = FULL_BWD_DRAM_BYTES_H4 * (wl.H / 4) if FULL_BWD_DRAM_BYTES_H4 else None
+    roof = {"kernel": "ssa_full_attn_bwd call (attn_bwd_kernel, prep, dQ conversion)", "bound": "tensor",
+            "achieved": fb / (op_ms["full_bwd"] / 1e3) / 1e12, "peak": peak_sust,
             "unit": "TFLOP/s", "traffic": traffic, "traffic_unit": "DRAM bytes per launch (ncu)",
             "peak_basis": "%s bf16 dense, sustained (kernel timed inside a long step)" % peak_kind}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    sparse_tflops = (sf + sb) / (sparse_ms / 1e3) / 1e12
+    sel_bytes = wl.B * wl.H * wl.T * (2 * wl.d + 4 * K_SEL)
+    pool_bytes = wl.B * wl.H * wl.T * 2 * wl.d
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_block(wl),
-        "sparse_attn": {"fwd_bwd_ms": sparse_ms, "tflops": (sf + sb) / (sparse_ms / 1e3) / 1e12,
+        "sparse_attn": {"fwd_bwd_ms": sparse_ms, "tflops": sparse_tflops,
                         "tflops_exact_attended": 3.5 * exact_attended_flops(wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL)
                         / (sparse_ms / 1e3) / 1e12,
-                        "frac_of_peak": (sf + sb) / (sparse_ms / 1e3) / 1e12 / peak_sust,
-                        "frac_of_burst_peak": (sf + sb) / (sparse_ms / 1e3) / 1e12 / peak_burst,
-                        "tokens_per_s": wl.B * wl.T / (sparse_ms / 1e3), "flop_per_step": sf + sb},
+                        "frac_of_peak": sparse_tflops / peak_sust, "frac_of_burst_peak": sparse_tflops / peak_burst,
+                        "tokens_per_s": wl.B * wl.T / (sparse_ms / 1e3), "flop_per_step": sf + sb,
+                        "calls": "ssa_sparse_index + ssa_sparse_attn_fwd + ssa_sparse_attn_bwd (accumulating)"},
+        "step_tokens_per_s": whole_job_tokens_per_s(wl.B * wl.T, world, ms_step),
         "full_attn": {"fwd_bwd_ms": full_ms, "tflops": (ff + fb) / (full_ms / 1e3) / 1e12,
                       "frac_of_peak": (ff + fb) / (full_ms / 1e3) / 1e12 / peak_sust},
         "op_ms": op_ms,
-        "select_hbm": {"gbs": (wl.B * wl.H * wl.T * (2 * wl.d + 4 * K_SEL)) / (op_ms["select"] / 1e3) / 1e9,
-                       "frac": (wl.B * wl.H * wl.T * (2 * wl.d + 4 * K_SEL)) / (op_ms["select"] / 1e3) / 1e9 / hbm,
-                       "frac_of_nominal_8tbs": (wl.B * wl.H * wl.T * (2 * wl.d + 4 * K_SEL))
-                       / (op_ms["select"] / 1e3) / 1e9 / 8000.0},
-        "pool_hbm": {"gbs": (wl.B * wl.H * wl.T * 2 * wl.d) / (pool_kernel_ms / 1e3) / 1e9,
-                     "frac": (wl.B * wl.H * wl.T * 2 * wl.d) / (pool_kernel_ms / 1e3) / 1e9 / hbm,
-                     "ms": pool_kernel_ms, "timing": "mean of 10 back-to-back launches"},
+        "select_hbm": {"gbs": sel_bytes / (op_ms["select"] / 1e3) / 1e9,
+                       "frac": sel_bytes / (op_ms["select"] / 1e3) / 1e9 / hbm,
+                       "frac_of_nominal_8tbs": sel_bytes / (op_ms["select"] / 1e3) / 1e9 / 8000.0},
+        "pool_hbm": {"gbs": pool_bytes / (op_ms["pool"] / 1e3) / 1e9,
+                     "frac": pool_bytes / (op_ms["pool"] / 1e3) / 1e9 / hbm, "ms": op_ms["pool"],
+                     "timing": "in-step CUDA events",
+                     "back_to_back": {"ms": pool_b2b_ms, "gbs": pool_bytes / (pool_b2b_ms / 1e3) / 1e9,
+                                      "frac": pool_bytes / (pool_b2b_ms / 1e3) / 1e9 / hbm}},
         "roofline": roof,
         "e2e": {"value": whole_job_tokens_per_s(wl.B * wl.T, world, e_ms / args.steps), "unit": "tokens/s",
-                "h2d_bytes_per_step": sum(host[k].numel() * 2 for k in host), "d2h_bytes_per_step": 4},
+                "h2d_bytes_per_step": sum(host[k].numel() * 2 for k in host),
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in out_host.values()),
+                "path": "pool, select, index, sparse fwd, sparse bwd with Q, K, V, dO copied in and O, dQ, dK, dV "
+                        "copied out every step"},
         "gpu_launches": args.steps * (ops.SSAStep.KERNELS_FWD + ops.SSAStep.KERNELS_BWD),
         "clocks": clocks,
     }
@@ -401,10 +434,9 @@ def ours(args, rank, world, local_rank):
             import oracle
             oracle.build()
             dt, fl, desc = oracle_sample(args.ref_tokens)
-            full_fl = sf + sb + ff + fb
-            line["cpu_baseline"] = {"value": wl.B * wl.T / (dt * full_fl / fl), "unit": "tokens/s",
+            line["cpu_baseline"] = {"value": wl.B * wl.T / (dt * (sf + sb) / fl), "unit": "tokens/s",
                                     "cores": oracle.num_threads(), "kind": "oracle",
-                                    "sample": desc + "; %.2f s, scaled to the full step by algorithmic FLOPs" % dt}
+                                    "sample": desc + "; %.2f s" % dt, "extrapolated": True}
         except Exception as e:  # the baseline never blocks the GPU number
             line["cpu_baseline"] = {"value": None, "unit": "tokens/s", "cores": None, "kind": "oracle",
                                     "sample": "failed: %s" % e}
@@ -426,7 +458,7 @@ def single_op(args):
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     dev = {key: torch.from_numpy(g[key].view(np.int16) if w.dtype == "bf16" else g[key]).view(dt).cuda()
            for key in ("Q", "K", "V", "dO")}
-    st = ops.SSAStep(dims)
+    st = ops.SSAStep(dims, grad_fp32=True)
     st.forward(dev["Q"], dev["K"], dev["V"])
     st.dOf.copy_(dev["dO"])
     st.dOs.copy_(dev["dO"])
@@ -434,13 +466,16 @@ def single_op(args):
     calls = {
         "pool": lambda: L.ssa_block_pool(dims, K, st.Kbar),
         "select": lambda: L.ssa_block_select(dims, Q, st.Kbar, st.idx),
-        "full_fwd": lambda: L.ssa_full_attn_fwd(dims, Q, K, V, st.Of, st.lse_f, st.ws[L.SSA_OP_FULL_FWD]),
+        "index": lambda: L.ssa_sparse_index(dims, st.idx, st.index),
+        "full_fwd": lambda: L.ssa_full_attn_fwd(dims, Q, K, V, st.Of, st.lse_f, st.ws[L.SSA_OP_FULL_FWD],
+                                                O_lo=st.Of_lo),
         "sparse_fwd": lambda: L.ssa_sparse_attn_fwd(dims, Q, K, V, st.idx, st.Os, st.lse_s,
-                                                    st.ws[L.SSA_OP_SPARSE_FWD]),
-        "full_bwd": lambda: L.ssa_full_attn_bwd(dims, Q, K, V, st.Of, st.lse_f, st.dOf, st.dQ, st.dK, st.dV, 0,
-                                                st.ws[L.SSA_OP_FULL_BWD]),
+                                                    st.ws[L.SSA_OP_SPARSE_FWD], O_lo=st.Os_lo, index=st.index),
+        "full_bwd": lambda: L.ssa_full_attn_bwd(dims, Q, K, V, st.Of, st.lse_f, st.dOf, st.dQ, st.dK, st.dV,
+                                                L.SSA_BWD_GRAD_FP32, st.ws[L.SSA_OP_FULL_BWD], O_lo=st.Of_lo),
         "sparse_bwd": lambda: L.ssa_sparse_attn_bwd(dims, Q, K, V, st.Os, st.lse_s, st.dOs, st.idx, st.dQ, st.dK,
-                                                    st.dV, 0, st.ws[L.SSA_OP_SPARSE_BWD]),
+                                                    st.dV, L.SSA_BWD_GRAD_FP32, st.ws[L.SSA_OP_SPARSE_BWD],
+                                                    O_lo=st.Os_lo, index=st.index),
     }
     fn = calls[args.op]
     for _ in range(args.warmup):
@@ -470,7 +505,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="the k sweep at T = 131072 (one JSON line per k)")
     ap.add_argument("--op", default=None,
-                    choices=["pool", "select", "full_fwd", "sparse_fwd", "full_bwd", "sparse_bwd"],
+                    choices=["pool", "select", "index", "full_fwd", "sparse_fwd", "full_bwd", "sparse_bwd"],
                     help="time one library call instead of the whole step (profiling)")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--T", type=int, default=0)

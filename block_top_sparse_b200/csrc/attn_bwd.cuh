@@ -3,14 +3,15 @@
 //
 // Key-block-outer: one CTA per key tile (full: 128 keys; the query tiles from
 // the diagonal on) or per key block j (sparse: s keys; the 128-row tiles of the
-// queries whose selection holds j, gathered by row).  K_j, V_j stay in shared
+// queries whose selection holds j, gathered by row), of one key/value head: with
+// grouped query heads the tiles of all G heads reading it (full: head after
+// head; sparse: 128 / G list entries per tile, each for the G heads).  K_j, V_j stay in shared
 // memory and the transposed accumulators dV_j^T, dK_j^T stay in tensor memory
 // for the whole unit.  Per query tile:
 //   S = Q K^T, dP = dO V^T                      (M = 128 query rows)
 //   P = exp(scale S - lse), dS = P o (dP - D)   -> shared memory, bf16
 //   dV^T += dO^T P, dK^T += Q^T dS              (M = head dim 128)
-//   dQ = dS K, * scale                           -> full: added into an fp32 accumulator;
-//                                                   sparse: a bf16 partial row per (query, slot)
+//   dQ = dS K, * scale                           -> added into an fp32 accumulator
 // Paper: section 4.2 (keys outside S(t) get no gradient; the selection is a
 // constant), FlashAttention-2 style recomputation of P from the saved lse.
 //
@@ -23,10 +24,9 @@
 //                tile's rows are contiguous): columns 0-63 into a 32 KB staging
 //                buffer of its own, 64-127 into the P region (free once dQ is
 //                computed), added by four TMA tensor reduce-adds issued by one
-//                thread.  Sparse stream (gathered rows): the tile is rounded to
-//                bf16 and written by TMA tile stores as partial rows at the list
-//                positions of the block's entries (contiguous there); a merge
-//                kernel later sums each query's k partials;
+//                thread.  Sparse stream (gathered rows): each warp adds its 32 rows
+//                with coalesced fp32 vector reductions through its own region of
+//                the staging buffer;
 //   warp 12      MMA issuer (one thread);
 //   warp 13      TMA producer (K_j, V_j; contiguous Q / dO tiles of the full stream);
 //   warps 14-19  sparse stream: gather the next tile's Q and dO rows with
@@ -58,9 +58,11 @@ struct BwdSmem {
 struct BwdArgs {
     const __nv_bfloat16 *Q, *dO;
     const float *lse, *Dvec;
-    __nv_bfloat16 *dK, *dV;
+    float *dQacc;  // sparse stream: fp32 dQ accumulator [B*H*T, 128] (the full stream adds through tmdQ)
+    void *dK, *dV;  // bf16, or fp32 when grad_fp32
     const int32_t *entries, *lstart, *llen;  // sparse only
-    int BH, T, k, nb, sparse, accumulate;
+    int BH, T, k, nb, sparse, accumulate, grad_fp32;
+    int G;  // query heads per key/value head; BH counts key/value heads
     float scale, scale_log2;
 };
 
@@ -95,10 +97,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // Head-major unit order: the query rows and the dQ accumulator of the head
     // being worked on stay in L2.
     const int units_per_head = a.sparse ? a.nb : (a.T + NKV - 1) / NKV;
-    int bh, kb;
+    int bh, kb;  // key/value head, key tile (block)
     unit_order(blockIdx.x, a.BH, units_per_head, bh, kb);
     const int kv0 = kb * NKV;
-    const size_t head_rows = static_cast<size_t>(bh) * T;
+    const size_t head_rows = static_cast<size_t>(bh) * T;  // key/value rows of this head
     const bool sparse = a.sparse != 0;
     Rows R;
     if (sparse) {
@@ -107,11 +109,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         R.first = 0;
     } else {
         R.list = nullptr;
-        R.first = kv0;  // causal: query tiles from the key tile onward
+        R.first = kv0;  // causal: query tiles from the key tile onward, for each of the G heads
         R.len = T - kv0;
     }
     R.k = a.k;
-    const int ntiles = (R.len + kTileQ - 1) / kTileQ;
+    R.gshift = log2_pow2(a.G);
+    R.T = T;
+    R.qrow0 = static_cast<size_t>(bh) * a.G * T;
+    const int ntiles = R.ntiles();
+    // query-tensor row of tile row 0 of contiguous tile it (full stream)
+    auto tile_row0 = [&](int it) {
+        int t;
+        size_t qrow;
+        tile_row(R, it, 0, t, qrow);
+        return static_cast<int>(qrow);
+    };
 
     const uint32_t sQ = smem_u32(smem + L::kQ), sdO = smem_u32(smem + L::kdO), sK = smem_u32(smem + L::kK),
                    sV = smem_u32(smem + L::kV), sP = smem_u32(smem + L::kP), sdS = smem_u32(smem + L::kdS),
@@ -154,12 +166,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (sparse) {
                 const int gw = warp - 14, u = lane & 15;
                 int tn[kBwdGatherPairs];
-                auto load_rows = [&](int it) {
+                auto load_rows = [&](int it) {  // query-tensor rows, -1 past the list
 #pragma unroll
                     for (int q = 0; q < kBwdGatherPairs; ++q) {
                         const int p = gw + kBwdGatherWarps * q;
-                        const int li = it * kTileQ + 2 * p + (lane >> 4);
-                        tn[q] = (p < 64 && li < R.len) ? (__ldg(R.list + li) >> 8) : -1;
+                        int t = 0;
+                        size_t row = 0;
+                        tn[q] = (p < 64 && tile_row(R, it, 2 * p + (lane >> 4), t, row)) ? static_cast<int>(row) : -1;
                     }
                 };
                 load_rows(0);
@@ -175,7 +188,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                             const int r = 2 * p + (lane >> 4);
                             const uint32_t off = (u >> 3) * kChunkBytes + r * 128 + ((((u & 7) ^ (r & 7)) & 7) << 4);
                             const bool valid = tn[q] >= 0;
-                            const size_t src = (head_rows + (valid ? tn[q] : 0)) * kD + u * 8;
+                            const size_t src = static_cast<size_t>(valid ? tn[q] : 0) * kD + u * 8;
                             cp_async_16(sQ + off, a.Q + src, valid ? 16u : 0u);
                             cp_async_16(sdO + off, a.dO + src, valid ? 16u : 0u);
                         }
@@ -197,7 +210,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (!sparse) {
                     int do_issued = 0, q_issued = 0;
                     for (int it = 0; it < ntiles; ++it) {
-                        const int qrow = static_cast<int>(head_rows) + kv0 + it * kTileQ;
+                        const int qrow = tile_row0(it);
                         // dO of tile it once the dV MMAs of tile it-1 have read dO
                         if (it > 0 && !mbar_wait(bar_do_free, (it - 1) & 1, abort_flag, 0x314)) break;
                         mbar_arrive_expect_tx(bar_do_full, 2 * kChunkBytes);
@@ -304,7 +317,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     if (!mbar_wait(bar_f_staged, it & 1, abort_flag, 0x30a)) break;
                     // rows past T in the last tile hold exact zeros (P = 0 there); rows past the
                     // tensor are clipped by the TMA unit
-                    const int row0 = static_cast<int>(head_rows) + kv0 + it * kTileQ;
+                    const int row0 = tile_row0(it);
                     // the P-region chunks first, in a group of their own, so that P is released early
                     tma_reduce_add_2d(&tmdQ, sP, 64, row0);
                     tma_reduce_add_2d(&tmdQ, sP + kChunkBytes, 96, row0);
@@ -320,50 +333,72 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             if (r == 0) bulk_wait();  // the TMA reduce-adds have completed
         } else {
-            // Sparse stream: the tile's dQ (scaled, rounded to bf16) is one partial row per
-            // (query, slot) at the entry's list position, so nothing is reduced here: each warp
-            // stages its 32 rows in the 128-byte-swizzled layout (columns 0-63 | 64-127 in the two
-            // halves of the staging buffer) and writes them with two TMA tile stores.  The list
-            // region of every block is padded to whole tiles, so the rows of a partial last tile
-            // stay inside this block's region (and are never read).
-            const size_t lbase = static_cast<size_t>(bh) * list_stride(T, a.k, a.nb) + a.lstart[bh * a.nb + kb];
-            const uint32_t wrow = static_cast<uint32_t>((warp & 3) * 32);
+            // Sparse stream (gathered rows): each warp adds its 32 rows of the tile's dQ (scaled,
+            // fp32) into the fp32 accumulator rows of their queries with vector reductions.  One
+            // 64-column half at a time goes through the warp's own 8 KB region of the staging buffer
+            // (row rl: 16-byte unit q at position q ^ (rl & 15), conflict-free for the row-owner
+            // writes and for the reads below), then each half-warp adds one 256-byte row half per
+            // instruction.  Columns 64-127 wait in registers, so the whole tile leaves tensor
+            // memory at once.  No cross-warp barrier: a warp only reuses its own region.
+            const uint32_t stg = sF + static_cast<uint32_t>(warp & 3) * 8192u;
+            auto stage = [&](const uint32_t (&g)[32], int q0) {
+#pragma unroll
+                for (int q8 = 0; q8 < 8; ++q8) {
+                    const int q = q0 + q8;
+                    const uint32_t *x = g + 4 * q8;
+                    st_shared_v4(stg + lane * 256 + (((q ^ lane) & 15) << 4),
+                                 __float_as_uint(__uint_as_float(x[0]) * a.scale),
+                                 __float_as_uint(__uint_as_float(x[1]) * a.scale),
+                                 __float_as_uint(__uint_as_float(x[2]) * a.scale),
+                                 __float_as_uint(__uint_as_float(x[3]) * a.scale));
+                }
+            };
+            auto add_half = [&](int hf, int t_mine) {
+                __syncwarp();
+                const int u = lane & 15;
+#pragma unroll 4
+                for (int i = 0; i < 16; ++i) {
+                    const int rl = 2 * i + (lane >> 4);
+                    const int t_dst = __shfl_sync(0xffffffffu, t_mine, rl);  // query-tensor row
+                    float4 v;
+                    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                                 : "r"(stg + rl * 256 + (((u ^ rl) & 15) << 4)));
+                    if (t_dst >= 0)
+                        atomicAdd(reinterpret_cast<float4 *>(a.dQacc + static_cast<size_t>(t_dst) * kD + 64 * hf) + u, v);
+                }
+                __syncwarp();
+            };
+            // row r's query-tensor row (-1 past the list), loaded one tile ahead
+            auto row_of = [&](int it) {
+                int t;
+                size_t qrow;
+                return (it < ntiles && tile_row(R, it, r, t, qrow)) ? static_cast<int>(qrow) : -1;
+            };
+            int q_n = row_of(0);
             for (int it = 0; it < ntiles; ++it) {
+                const int t_mine = q_n;  // destination row of this thread's dQ row
+                q_n = row_of(it + 1);
                 if (!mbar_wait(bar_dq_full, it & 1, abort_flag, 0x307)) break;
                 tc_fence_after();
-                // the previous tile's stores have read this warp's staging rows
-                if (lane == 0) bulk_wait_read();
-                __syncwarp();
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t g[2][32];
-                    tmem_ld32_async(tdQ + lane_off + 64 * hh, g[0]);
-                    tmem_ld32_async(tdQ + lane_off + 64 * hh + 32, g[1]);
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t g[32];
+                    tmem_ld32_async(tdQ + lane_off + 32 * c, g);
                     tmem_ld_wait();
-                    if (hh == 1) {
-                        tc_fence_before();
-                        mbar_arrive(bar_dq_empty);  // dQ has left tensor memory: the next S may overwrite it
-                    }
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const uint32_t *x = g[u >> 2] + 8 * (u & 3);
-                        st_shared_v4(sF + hh * kChunkBytes + r * 128 + (((u ^ (r & 7)) & 7) << 4),
-                                     pack_bf16x2(__uint_as_float(x[0]) * a.scale, __uint_as_float(x[1]) * a.scale),
-                                     pack_bf16x2(__uint_as_float(x[2]) * a.scale, __uint_as_float(x[3]) * a.scale),
-                                     pack_bf16x2(__uint_as_float(x[4]) * a.scale, __uint_as_float(x[5]) * a.scale),
-                                     pack_bf16x2(__uint_as_float(x[6]) * a.scale, __uint_as_float(x[7]) * a.scale));
-                    }
+                    stage(g, 8 * c);
                 }
-                fence_proxy_async_smem();  // generic-proxy staging writes -> TMA reads
-                __syncwarp();
-                if (lane == 0) {
-                    const int row0 = static_cast<int>(lbase + static_cast<size_t>(it) * kTileQ + wrow);
-                    tma_store_2d(&tmdQ, sF + wrow * 128, 0, row0);
-                    tma_store_2d(&tmdQ, sF + kChunkBytes + wrow * 128, 64, row0);
-                    bulk_commit();
-                }
+                uint32_t hi[2][32];
+                tmem_ld32_async(tdQ + lane_off + 64, hi[0]);
+                tmem_ld32_async(tdQ + lane_off + 96, hi[1]);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(bar_dq_empty);  // dQ has left tensor memory: the next S may overwrite it
+                add_half(0, t_mine);
+                stage(hi[0], 0);
+                stage(hi[1], 8);
+                add_half(1, t_mine);
             }
-            if (lane == 0) bulk_wait();  // the stores have completed
         }
     } else {
         // ---------------- softmax / dS warpgroups ----------------
@@ -375,11 +410,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // Row data is fetched ahead: the query position of tile it+2 and the lse, D of tile it+1
         // are loaded while tile it is processed (the sparse stream's lse / D addresses depend on
         // the position loaded from the list), so no dependent global load sits between two tiles.
-        int e = 0, t_n1 = 0, t_n2 = 0;
-        bool v_n1 = ntiles > 0 && tile_row(R, T, 0, r, t_n1, e);
-        float lse_n = v_n1 ? __ldg(a.lse + head_rows + t_n1) : 0.f;
-        float D_n = v_n1 ? __ldg(a.Dvec + head_rows + t_n1) : 0.f;
-        bool v_n2 = ntiles > 1 && tile_row(R, T, 1, r, t_n2, e);
+        int t_n1 = 0, t_n2 = 0;
+        size_t q_n1 = 0, q_n2 = 0;
+        bool v_n1 = ntiles > 0 && tile_row(R, 0, r, t_n1, q_n1);
+        float lse_n = v_n1 ? __ldg(a.lse + q_n1) : 0.f;
+        float D_n = v_n1 ? __ldg(a.Dvec + q_n1) : 0.f;
+        bool v_n2 = ntiles > 1 && tile_row(R, 1, r, t_n2, q_n2);
         for (int it = 0; it < ntiles; ++it) {
             const bool valid = v_n1;
             const int t = t_n1;
@@ -387,9 +423,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float Dt = D_n;
             v_n1 = v_n2;
             t_n1 = t_n2;
-            lse_n = v_n1 ? __ldg(a.lse + head_rows + t_n1) : 0.f;
-            D_n = v_n1 ? __ldg(a.Dvec + head_rows + t_n1) : 0.f;
-            v_n2 = it + 2 < ntiles && tile_row(R, T, it + 2, r, t_n2, e);
+            q_n1 = q_n2;
+            lse_n = v_n1 ? __ldg(a.lse + q_n1) : 0.f;
+            D_n = v_n1 ? __ldg(a.Dvec + q_n1) : 0.f;
+            v_n2 = it + 2 < ntiles && tile_row(R, it + 2, r, t_n2, q_n2);
             if (!mbar_wait(bar_sdp_full, it & 1, abort_flag, 0x306)) {
                 ok = false;
                 break;
@@ -471,8 +508,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                              : "=f"(k4.x), "=f"(k4.y), "=f"(k4.z), "=f"(k4.w)
                              : "r"(sdk + kr * 512 + lane * 16));
                 const size_t off = (head_rows + kv0 + kr) * kD + 4 * lane;
-                uint2 *dv2 = reinterpret_cast<uint2 *>(a.dV + off);
-                uint2 *dk2 = reinterpret_cast<uint2 *>(a.dK + off);
+                if (a.grad_fp32) {
+                    // fp32 gradients: 16 bytes per lane, added to the existing values when asked
+                    float4 *dv4 = reinterpret_cast<float4 *>(static_cast<float *>(a.dV) + off);
+                    float4 *dk4 = reinterpret_cast<float4 *>(static_cast<float *>(a.dK) + off);
+                    if (a.accumulate) {
+                        const float4 ov = *dv4, ok4 = *dk4;
+                        v4.x += ov.x;
+                        v4.y += ov.y;
+                        v4.z += ov.z;
+                        v4.w += ov.w;
+                        k4.x += ok4.x;
+                        k4.y += ok4.y;
+                        k4.z += ok4.z;
+                        k4.w += ok4.w;
+                    }
+                    *dv4 = v4;
+                    *dk4 = k4;
+                    continue;
+                }
+                uint2 *dv2 = reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.dV) + off);
+                uint2 *dk2 = reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.dK) + off);
                 if (a.accumulate) {
                     const uint2 ov = *dv2, ok2 = *dk2;
                     v4.x += __uint_as_float(ov.x << 16);

@@ -46,14 +46,15 @@ __device__ __forceinline__ void for_each_attended(const int32_t *sel, int k, int
 template <typename T, int DPL>
 __global__ void __launch_bounds__(256) simt_fwd_kernel(const T *__restrict__ Q, const T *__restrict__ K,
                                                        const T *__restrict__ V, const int32_t *__restrict__ idx,
-                                                       T *__restrict__ O, float *__restrict__ lse, size_t rows,
-                                                       int Tl, int s, int k, float scale) {
+                                                       T *__restrict__ O, T *__restrict__ O_lo,
+                                                       float *__restrict__ lse, size_t rows, int Tl, int s, int k,
+                                                       float scale, int G) {
     const size_t row = static_cast<size_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
     constexpr int d = DPL * 32;
-    const size_t head = row - row % Tl;
     const int t = static_cast<int>(row % Tl);
+    const size_t head = (row / Tl / G) * Tl;  // first row of the key/value head (and its selection)
     float q[DPL], o[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) {
@@ -61,7 +62,7 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(const T *__restrict__ Q, 
         o[i] = 0.f;
     }
     float m = -INFINITY, l = 0.f;
-    for_each_attended(idx ? idx + row * k : nullptr, k, s, t, [&](int u) {
+    for_each_attended(idx ? idx + (head + t) * k : nullptr, k, s, t, [&](int u) {
         const T *kr = K + (head + u) * d;
         const T *vr = V + (head + u) * d;
         float part = 0.f;
@@ -76,7 +77,12 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(const T *__restrict__ Q, 
         m = mn;
     });
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) store_as(O + row * d + lane + 32 * i, o[i] / l);
+    for (int i = 0; i < DPL; ++i) {
+        const float v = o[i] / l;
+        store_as(O + row * d + lane + 32 * i, v);
+        // bf16 outputs: the rounding residual o - bf16(o), rounded to bf16 (the caller passes no O_lo for fp32)
+        if (O_lo) store_as(O_lo + row * d + lane + 32 * i, v - to_f32(O[row * d + lane + 32 * i]));
+    }
     if (lane == 0) lse[row] = m + logf(l);
 }
 
@@ -86,13 +92,13 @@ __global__ void __launch_bounds__(256) simt_bwd_kernel(const T *__restrict__ Q, 
                                                        const int32_t *__restrict__ idx, const float *__restrict__ lse,
                                                        const float *__restrict__ Dvec, float *__restrict__ dQacc,
                                                        float *__restrict__ dKacc, float *__restrict__ dVacc,
-                                                       size_t rows, int Tl, int s, int k, float scale) {
+                                                       size_t rows, int Tl, int s, int k, float scale, int G) {
     const size_t row = static_cast<size_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
     constexpr int d = DPL * 32;
-    const size_t head = row - row % Tl;
     const int t = static_cast<int>(row % Tl);
+    const size_t head = (row / Tl / G) * Tl;  // first row of the key/value head (and its selection)
     float q[DPL], g[DPL], dq[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) {
@@ -101,7 +107,7 @@ __global__ void __launch_bounds__(256) simt_bwd_kernel(const T *__restrict__ Q, 
         dq[i] = 0.f;
     }
     const float L = lse[row], Dt = Dvec[row];
-    for_each_attended(idx ? idx + row * k : nullptr, k, s, t, [&](int u) {
+    for_each_attended(idx ? idx + (head + t) * k : nullptr, k, s, t, [&](int u) {
         const T *kr = K + (head + u) * d;
         const T *vr = V + (head + u) * d;
         float kx[DPL], part = 0.f, partv = 0.f;

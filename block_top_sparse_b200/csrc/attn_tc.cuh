@@ -6,7 +6,7 @@
 //                     online softmax (paper section 3, full attention).
 //  sparse_fwd_kernel  block-major sparse forward: one CTA per (head, key block
 //                     j) processes, 128 at a time, the queries whose selection
-//                     holds j (gathered by row), and writes a normalised
+//                     holds j (gathered by row), and writes a normalised fp16
 //                     partial output + log-sum-exp per (query, slot); a merge
 //                     kernel combines the k partials of each query.
 //  (the backward kernel shared by both streams is in attn_bwd.cuh)
@@ -26,26 +26,46 @@ constexpr int kTileQ = 128;     // query rows per tile (MMA M)
 constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16
 
 struct Rows {
-    // Row source of a query tile: contiguous (full attention) or gathered from
-    // the inverse selection index (sparse attention).
-    const int32_t *list;  // entries (t << 8) | slot, or nullptr for contiguous rows
-    int len;              // number of rows in the list / valid rows overall
-    int first;            // contiguous: first query position
+    // Row source of a query tile of one key/value head's unit.  G query heads read the key head
+    // (grouped-query attention; G = 1 for one query head per key head; G is a power of two).
+    //  sparse: gathered from the key block's list of entries (t << 8) | slot; a tile holds
+    //          128 / G entries, each for all G heads, entry-major (tile row r: entry r / G,
+    //          head r % G), so that tile row r of tile it is partial row it * 128 + r of the block;
+    //  full:   contiguous query rows from `first` on, the G heads' tiles one head after another.
+    const int32_t *list;  // entries, or nullptr for contiguous rows
+    int len;              // sparse: entries in the list; full: query rows per head (T - first)
+    int first;            // full: first query position
     int k;
+    int gshift;           // log2(G)
+    int T;
+    size_t qrow0;         // row of the group's first query head in the [B*H*T] query tensors
+    __device__ __forceinline__ int per_tile() const { return list ? kTileQ >> gshift : kTileQ; }
+    __device__ __forceinline__ int tiles_per_head() const { return (len + kTileQ - 1) / kTileQ; }
+    __device__ __forceinline__ int ntiles() const {
+        return list ? (len + per_tile() - 1) / per_tile() : (tiles_per_head() << gshift);
+    }
 };
 
-// Query position and global selection entry of tile row r of tile `it`.
-__device__ __forceinline__ bool tile_row(const Rows &R, int T, int it, int r, int &t, int &entry) {
+__host__ __device__ __forceinline__ int log2_pow2(int g) {
+    int s = 0;
+    while ((1 << s) < g) ++s;
+    return s;
+}
+
+// Query position t and query-tensor row of tile row r of tile `it`; false past the end.
+__device__ __forceinline__ bool tile_row(const Rows &R, int it, int r, int &t, size_t &qrow) {
     if (R.list) {
-        const int li = it * kTileQ + r;
+        const int li = ((it * kTileQ + r) >> R.gshift);  // it * (128 / G) + r / G
         if (li >= R.len) return false;
-        entry = __ldg(R.list + li);
-        t = entry >> 8;
+        t = __ldg(R.list + li) >> 8;
+        qrow = R.qrow0 + static_cast<size_t>(r & ((1 << R.gshift) - 1)) * R.T + t;
         return true;
     }
-    t = R.first + it * kTileQ + r;
-    entry = -1;
-    return t < T;
+    const int tph = R.tiles_per_head();
+    const int hi = R.gshift ? it / tph : 0;
+    t = R.first + (it - hi * tph) * kTileQ + r;
+    qrow = R.qrow0 + static_cast<size_t>(hi) * R.T + t;
+    return t < R.T;
 }
 
 // Write 32 fp32 values as bf16 into row r, columns [c0, c0+32) of a swizzled
@@ -79,7 +99,8 @@ __device__ __forceinline__ void mma_k128_kmajor(uint32_t d_tmem, uint32_t a, uin
 
 // ---------------------------------------------------------------------------
 // Full causal attention forward, two query tiles per CTA in ping-pong.
-// grid = (ceil(T/256), B*H), heaviest query blocks first; block = 384 threads.
+// grid = B*H*ceil(T/256) (query heads; head h reads key/value head h / G), heaviest
+// query blocks first; block = 384 threads.
 //   warpgroup x in {0, 1} owns query tile x (rows 256*qb + 128*x + row): online
 //   softmax over the key tiles 0..diag(x) with lazy rescaling of O (only when the
 //   running maximum grows by more than 2^8), P written as bf16 pairs over S in
@@ -105,8 +126,9 @@ constexpr int kFullFwdThreads = 384;
 
 __global__ void __launch_bounds__(kFullFwdThreads, 1)
     full_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ O, float *__restrict__ lse,
-                    int BH, int T, float scale_log2) {
+                    const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ O,
+                    __nv_bfloat16 *__restrict__ O_lo, float *__restrict__ lse, int BH, int T, int G,
+                    float scale_log2) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + FullFwdSmem::kBar);
@@ -125,7 +147,8 @@ __global__ void __launch_bounds__(kFullFwdThreads, 1)
     int bh, u;
     unit_order(blockIdx.x, BH, nqb, bh, u);
     const int qb = nqb - 1 - u;  // heaviest query blocks first
-    const int row0 = bh * T;              // first tensor-map row of this head
+    const int row0 = bh * T;              // first tensor-map row of this query head
+    const int krow0 = (bh / G) * T;       // first row of its key/value head
     const int q0 = qb * 256;              // first query of tile a; tile b starts at q0 + 128
     // key tiles 0 .. diag: tile a ends at key tile 2qb, tile b at 2qb+1
     const int nkv_a = 2 * qb + 1, nkv_b = 2 * qb + 2;
@@ -168,10 +191,10 @@ __global__ void __launch_bounds__(kFullFwdThreads, 1)
                 mbar_arrive_expect_tx(bar_kv_full + st, 4 * kChunkBytes);
                 uint8_t *k = smem + FullFwdSmem::kK + st * 2 * kChunkBytes;
                 uint8_t *v = smem + FullFwdSmem::kV + st * 2 * kChunkBytes;
-                tma_load_2d(&tmK, bar_kv_full + st, k, 0, row0 + n * kTileQ);
-                tma_load_2d(&tmK, bar_kv_full + st, k + kChunkBytes, 64, row0 + n * kTileQ);
-                tma_load_2d(&tmV, bar_kv_full + st, v, 0, row0 + n * kTileQ);
-                tma_load_2d(&tmV, bar_kv_full + st, v + kChunkBytes, 64, row0 + n * kTileQ);
+                tma_load_2d(&tmK, bar_kv_full + st, k, 0, krow0 + n * kTileQ);
+                tma_load_2d(&tmK, bar_kv_full + st, k + kChunkBytes, 64, krow0 + n * kTileQ);
+                tma_load_2d(&tmV, bar_kv_full + st, v, 0, krow0 + n * kTileQ);
+                tma_load_2d(&tmV, bar_kv_full + st, v + kChunkBytes, 64, krow0 + n * kTileQ);
             }
         }
     } else if (warp == 8) {
@@ -324,22 +347,35 @@ __global__ void __launch_bounds__(kFullFwdThreads, 1)
         if (ok && mbar_wait(bar_o_full + x, (nkv - 1) & 1, abort_flag, 0x10a)) {
             tc_fence_after();
             const float inv_l = 1.f / l;
-            uint4 *d4 = reinterpret_cast<uint4 *>(O + (static_cast<size_t>(row0) + (t < T ? t : 0)) * kD);
+            const size_t orow = (static_cast<size_t>(row0) + (t < T ? t : 0)) * kD;
+            uint4 *d4 = reinterpret_cast<uint4 *>(O + orow);
+            uint4 *l4 = O_lo ? reinterpret_cast<uint4 *>(O_lo + orow) : nullptr;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                uint32_t orow[2][32];
-                tmem_ld32_async(tO + 64 * hh, orow[0]);  // warp-collective: outside the row branch
-                tmem_ld32_async(tO + 64 * hh + 32, orow[1]);
+                uint32_t orow_v[2][32];
+                tmem_ld32_async(tO + 64 * hh, orow_v[0]);  // warp-collective: outside the row branch
+                tmem_ld32_async(tO + 64 * hh + 32, orow_v[1]);
                 tmem_ld_wait();
                 if (t < T) {
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const uint32_t *xo = orow[q >> 2] + 8 * (q & 3);
-                        d4[8 * hh + q] =
-                            make_uint4(pack_bf16x2(__uint_as_float(xo[0]) * inv_l, __uint_as_float(xo[1]) * inv_l),
-                                       pack_bf16x2(__uint_as_float(xo[2]) * inv_l, __uint_as_float(xo[3]) * inv_l),
-                                       pack_bf16x2(__uint_as_float(xo[4]) * inv_l, __uint_as_float(xo[5]) * inv_l),
-                                       pack_bf16x2(__uint_as_float(xo[6]) * inv_l, __uint_as_float(xo[7]) * inv_l));
+                        const uint32_t *xo = orow_v[q >> 2] + 8 * (q & 3);
+                        float v[8];
+                        uint32_t hi[4];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(xo[i]) * inv_l;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) hi[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                        d4[8 * hh + q] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                        if (l4) {
+                            // the rounding residual o - bf16(o), itself rounded to bf16
+                            uint32_t lo[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                lo[i] = pack_bf16x2(v[2 * i] - __uint_as_float(hi[i] << 16),
+                                                    v[2 * i + 1] - __uint_as_float(hi[i] & 0xFFFF0000u));
+                            l4[8 * hh + q] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                        }
                     }
                 }
             }
@@ -354,14 +390,20 @@ __global__ void __launch_bounds__(kFullFwdThreads, 1)
 
 // ---------------------------------------------------------------------------
 // Sparse forward, block-major, two warpgroups in ping-pong.
-// grid = (B*H*nb): unit u -> head bh = u / nb, block j = u % nb (head-major, so
-// the head's query rows stay in L2).  block = 512 threads:
+// grid = (B*Hkv*nb): unit u -> key/value head bh = u / nb, block j = u % nb
+// (head-major, so the head's query rows stay in L2); a tile holds 128 / G list
+// entries for each of the G query heads reading the key head.  block = 512 threads:
 //   warpgroup g (warps 4g .. 4g+3) owns the query tiles it = g, g+2, ... of the
 //   block's list: masked softmax over the block's NKV keys, P written back over
 //   S in tensor memory as bf16 pairs, then the normalised partial output o / l
 //   and the partial log-sum-exp of every (query, slot) at the entry's position
 //   in the block's list (each warp stages its 32 rows in shared memory and
-//   writes them with two TMA tile stores: a tile's rows are contiguous);
+//   writes them with two TMA tile stores: a tile's rows are contiguous).  The
+//   partial is fp16 (11 significant bits: the merged output, and the D of the
+//   backward formed from it, stay far below bf16 rounding) scaled by 2^-e_j,
+//   where e_j >= 0 keeps the block's values below 2^15 (e_j = 0 unless some
+//   |v| of block j reaches 2^15; stored per block for the merge, with a flag
+//   word after the last block that is set when any e_j is not 0);
 //   warps 8-11 and 13-15 gather each tile's query rows with cp.async, a
 //   half-warp per 256-byte row (a gather's cost is set by the number of warp
 //   instructions in flight, so seven warps share it; completion on an mbarrier);
@@ -395,17 +437,19 @@ constexpr int kSparseFwdGatherWarps = 7;
 // unit, into the 2-chunk 128-byte-swizzled tile.  Rows past the list are zero-filled.
 constexpr int kGatherPairs = (64 + kSparseFwdGatherWarps - 1) / kSparseFwdGatherWarps;
 
-__device__ __forceinline__ void gather_rows_load(const Rows &R, int it, int gw, int lane, int (&t)[kGatherPairs]) {
+// Query-tensor rows (-1 past the list) of this lane's rows of tile `it`.
+__device__ __forceinline__ void gather_rows_load(const Rows &R, int it, int gw, int lane, int (&qrow)[kGatherPairs]) {
 #pragma unroll
     for (int q = 0; q < kGatherPairs; ++q) {
         const int p = gw + kSparseFwdGatherWarps * q;
-        const int li = it * kTileQ + 2 * p + (lane >> 4);
-        t[q] = (p < 64 && li < R.len) ? (__ldg(R.list + li) >> 8) : -1;
+        int t = 0;
+        size_t row = 0;
+        qrow[q] = (p < 64 && tile_row(R, it, 2 * p + (lane >> 4), t, row)) ? static_cast<int>(row) : -1;
     }
 }
 
-__device__ __forceinline__ void gather_rows_issue(uint32_t tile, const __nv_bfloat16 *base, size_t head_rows, int gw,
-                                                  int lane, const int (&t)[kGatherPairs]) {
+__device__ __forceinline__ void gather_rows_issue(uint32_t tile, const __nv_bfloat16 *base, int gw, int lane,
+                                                  const int (&qrow)[kGatherPairs]) {
     const int u = lane & 15;
 #pragma unroll
     for (int q = 0; q < kGatherPairs; ++q) {
@@ -413,8 +457,8 @@ __device__ __forceinline__ void gather_rows_issue(uint32_t tile, const __nv_bflo
         if (p < 64) {
             const int r = 2 * p + (lane >> 4);
             const uint32_t dst = tile + (u >> 3) * kChunkBytes + r * 128 + ((((u & 7) ^ (r & 7)) & 7) << 4);
-            const bool valid = t[q] >= 0;
-            cp_async_16(dst, base + (head_rows + (valid ? t[q] : 0)) * kD + u * 8, valid ? 16u : 0u);
+            const bool valid = qrow[q] >= 0;
+            cp_async_16(dst, base + static_cast<size_t>(valid ? qrow[q] : 0) * kD + u * 8, valid ? 16u : 0u);
         }
     }
 }
@@ -424,8 +468,8 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmO, const __nv_bfloat16 *__restrict__ Q,
                       const int32_t *__restrict__ entries, const int32_t *__restrict__ lstart,
-                      const int32_t *__restrict__ llen, float *__restrict__ lsepart, int BH, int T, int k, int nb,
-                      float scale_log2) {
+                      const int32_t *__restrict__ llen, float *__restrict__ lsepart, int32_t *__restrict__ bexp,
+                      int BH, int T, int k, int nb, int G, float scale_log2) {
     using L = SparseFwdSmem<NKV>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -439,20 +483,25 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
     uint64_t *bar_q_free = bars + 20;  // [kSparseFwdQStages] the S MMA reading a stage has completed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 15);
+    uint32_t *vmax_part = reinterpret_cast<uint32_t *>(bars + 24);  // [8] per softmax warp, |v| bits
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int bh, j;
+    int bh, j;  // key/value head, key block
     unit_order(blockIdx.x, BH, nb, bh, j);
     const int kv0 = j * NKV;
-    const size_t head_rows = static_cast<size_t>(bh) * T;
-    // this block's list (and partial-output rows) start at list position obase
+    const size_t head_rows = static_cast<size_t>(bh) * T;  // key/value rows of this head
+    // this block's list starts at list position obase; its partial-output rows at obase * G
     const size_t obase = static_cast<size_t>(bh) * list_stride(T, k, nb) + lstart[bh * nb + j];
     Rows R;
     R.list = entries + obase;
     R.len = llen[bh * nb + j];
     R.first = 0;
     R.k = k;
-    const int ntiles = (R.len + kTileQ - 1) / kTileQ;
+    R.gshift = log2_pow2(G);
+    R.T = T;
+    R.qrow0 = static_cast<size_t>(bh) * G * T;
+    const int ntiles = R.ntiles();
+    const size_t prow0 = obase * G;  // partial row of tile row 0 of tile 0
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
@@ -493,7 +542,7 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
             if (lane == 0 && it >= kSparseFwdQStages)
                 ok = mbar_wait(bar_q_free + qs, (it / kSparseFwdQStages - 1) & 1, abort_flag, 0x208);
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            gather_rows_issue(smem_u32(smem + L::kQ + qs * 2 * kChunkBytes), Q, head_rows, gw, lane, tn);
+            gather_rows_issue(smem_u32(smem + L::kQ + qs * 2 * kChunkBytes), Q, gw, lane, tn);
             cp_async_mbar_arrive_noinc(bar_q_full + qs);
             if (it + 1 < ntiles) gather_rows_load(R, it + 1, gw, lane, tn);  // in flight during the next wait
         }
@@ -559,17 +608,52 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t sO = smem_u32(smem + L::kO + g * L::kOStage);  // this warpgroup's staging tile
         const uint32_t tS = tmem + 128 * g + lane_off, tO = tmem + 256 + 128 * g + lane_off;
-        // this row's list entry (t << 8 | slot, or -1 past the list) is loaded one tile ahead
-        int ent_n = (g < ntiles && g * kTileQ + r < R.len) ? __ldg(R.list + g * kTileQ + r) : -1;
+        // this row's query position (-1 past the list) is loaded one tile ahead
+        auto row_t = [&](int it) {
+            int t = -1;
+            size_t qrow;
+            return (it < ntiles && tile_row(R, it, r, t, qrow)) ? t : -1;
+        };
+        int t_n = row_t(g);
+        // range exponent of the block: max |v| over V_j (bf16 in shared memory; the layout does
+        // not matter for a maximum), reduced over the 256 softmax threads
+        int e_blk = 0;
+        {
+            bool okv = mbar_wait(bar_kv, 0, abort_flag, 0x209);
+            uint32_t m = 0u;
+            if (okv) {
+                constexpr int kBytesPer = 2 * NKV * 128 / 256;  // V_j bytes per softmax thread
+                const uint4 *src = reinterpret_cast<const uint4 *>(smem + L::kV + threadIdx.x * kBytesPer);
+#pragma unroll
+                for (int q = 0; q < kBytesPer / 16; ++q) {
+                    const uint4 v = src[q];
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) m = max(m, max((w[i] << 16) & 0x7FFF0000u, w[i] & 0x7FFF0000u));
+                }
+            }
+            m = __reduce_max_sync(0xffffffffu, m);  // |v| as fp32 bits: integer order = value order
+            if (lane == 0) vmax_part[warp] = m;
+            named_barrier(1, 256);
+            uint32_t mm = 0u;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) mm = max(mm, vmax_part[w]);
+            const int ex = static_cast<int>(mm >> 23) - 127;  // floor(log2 max|v|); NaN / inf give 128
+            e_blk = min(max(ex - 14, 0), 100);
+            if (threadIdx.x == 0) {
+                bexp[bh * nb + j] = e_blk;
+                if (e_blk > 0) atomicOr(bexp + static_cast<size_t>(BH) * nb, 1);  // some block needs its exponent
+            }
+        }
+        const float escale = __uint_as_float(static_cast<uint32_t>(127 - e_blk) << 23);  // 2^-e
         for (int it = g; it < ntiles; it += 2) {
             const int i = it >> 1;
-            const int ent = ent_n;
-            if (it + 2 < ntiles)
-                ent_n = (it + 2) * kTileQ + r < R.len ? __ldg(R.list + (it + 2) * kTileQ + r) : -1;
-            const bool valid = ent >= 0;
+            const int t_row = t_n;
+            if (it + 2 < ntiles) t_n = row_t(it + 2);
+            const bool valid = t_row >= 0;
             if (!mbar_wait(bar_s_full + g, i & 1, abort_flag, 0x206)) break;
             tc_fence_after();
-            const int lim = valid ? (ent >> 8) - kv0 : -1;
+            const int lim = valid ? t_row - kv0 : -1;
             uint32_t sr[NKV / 32][32];
 #pragma unroll
             for (int c = 0; c < NKV / 32; ++c) tmem_ld32_async(tS + 32 * c, sr[c]);
@@ -615,8 +699,8 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
             f2_unpack(l2[0], la, lb);
             f2_unpack(l2[1], lc, ld);
             const float l = (la + lb) + (lc + ld);
-            const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-            const size_t orow = obase + static_cast<size_t>(it) * kTileQ + r;  // list position of this row
+            const float inv_l = (l > 0.f) ? escale / l : 0.f;
+            const size_t orow = prow0 + static_cast<size_t>(it) * kTileQ + r;  // partial row of this tile row
             if (valid) lsepart[orow] = (l > 0.f) ? (mref + __log2f(l)) * kLn2 : -INFINITY;
             // the TMA stores of tile it-2 must have read this warp's staging rows
             if (lane == 0) bulk_wait_read();
@@ -634,17 +718,17 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
                 for (int u = 0; u < 8; ++u) {
                     const uint32_t *xo = ov[u >> 2] + 8 * (u & 3);
                     st_shared_v4(sO + hh * kChunkBytes + r * 128 + (((u ^ (r & 7)) & 7) << 4),
-                                 pack_bf16x2(__uint_as_float(xo[0]) * inv_l, __uint_as_float(xo[1]) * inv_l),
-                                 pack_bf16x2(__uint_as_float(xo[2]) * inv_l, __uint_as_float(xo[3]) * inv_l),
-                                 pack_bf16x2(__uint_as_float(xo[4]) * inv_l, __uint_as_float(xo[5]) * inv_l),
-                                 pack_bf16x2(__uint_as_float(xo[6]) * inv_l, __uint_as_float(xo[7]) * inv_l));
+                                 pack_half2(__uint_as_float(xo[0]) * inv_l, __uint_as_float(xo[1]) * inv_l),
+                                 pack_half2(__uint_as_float(xo[2]) * inv_l, __uint_as_float(xo[3]) * inv_l),
+                                 pack_half2(__uint_as_float(xo[4]) * inv_l, __uint_as_float(xo[5]) * inv_l),
+                                 pack_half2(__uint_as_float(xo[6]) * inv_l, __uint_as_float(xo[7]) * inv_l));
                 }
             }
             fence_proxy_async_smem();  // generic-proxy staging writes -> TMA reads
             __syncwarp();
             if (lane == 0) {
                 // rows 32w .. 32w+31 of the tile: the padded list region keeps them inside this block's rows
-                const int row0 = static_cast<int>(obase + static_cast<size_t>(it) * kTileQ + (r - lane));
+                const int row0 = static_cast<int>(prow0 + static_cast<size_t>(it) * kTileQ + (r - lane));
                 tma_store_2d(&tmO, sO + (r - lane) * 128, 0, row0);
                 tma_store_2d(&tmO, sO + kChunkBytes + (r - lane) * 128, 64, row0);
                 bulk_commit();

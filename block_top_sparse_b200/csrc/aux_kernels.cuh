@@ -2,7 +2,7 @@
 //   * inverse selection index (key block -> list of (query, slot) entries,
 //     ascending in query position), built deterministically in three passes;
 //   * merge of the block-major sparse forward's per-slot partial outputs;
-//   * backward pre/post-processing (D = rowsum(dO o O), dQ accumulator -> dQ);
+//   * backward pre/post-processing (D = rowsum(dO o (O + O_lo)), dQ accumulator -> dQ);
 //   * bidirectional SmoothL1 alignment loss forward/backward (paper section 5);
 //   * dropped attention mass delta = 1 - exp(lse_s - lse_f) (section 4.2).
 #pragma once
@@ -166,30 +166,58 @@ __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t *__restri
 // Merge of the per-slot partials: one warp per query row, 4 columns per lane.
 //   lse = log sum_i exp(lse_i),  o = sum_i exp(lse_i - lse) o_i
 // The partial of (query, slot i) sits at list position pos[query * k + i] of its
-// head's region (-1: slot not attended).  Lane i holds slot i's position and
-// weight (32 slots at a time), so the slots' row loads are all in flight at once.
-template <typename TO>
+// key head's region (-1: slot not attended), in partial row position * G + (query
+// head within the group).  Partials are fp16 (11 significant bits)
+// holding o_i * 2^-e_j, where e_j >= 0 is the range exponent of key block
+// j = idx[query * k + i] (0 unless |V| in that block reaches 2^15); the word after
+// the last block's exponent is non-zero when any exponent is, and only then are
+// idx and the exponents read.  Lane i holds
+// slot i's position and weight (32 slots at a time), so the slots' row loads are
+// all in flight at once.  The merged fp32 row is stored as O = bf16(o) and, when
+// O_lo is given, O_lo = bf16(o - O).
+__device__ __forceinline__ void half4_to_f32(uint2 u, float (&f)[4]) {
+    const __half2 a = *reinterpret_cast<const __half2 *>(&u.x), b = *reinterpret_cast<const __half2 *>(&u.y);
+    const float2 fa = __half22float2(a), fb = __half22float2(b);
+    f[0] = fa.x;
+    f[1] = fa.y;
+    f[2] = fb.x;
+    f[3] = fb.y;
+}
+
 __global__ void __launch_bounds__(256) sparse_merge_kernel(const int32_t *__restrict__ pos,
-                                                           const __nv_bfloat16 *__restrict__ Opart,
-                                                           const float *__restrict__ lsepart, TO *__restrict__ O,
-                                                           float *__restrict__ lse, size_t rows, int T, int k,
-                                                           int nb) {
+                                                           const int32_t *__restrict__ idx,
+                                                           const int32_t *__restrict__ bexp,
+                                                           const __half *__restrict__ Opart,
+                                                           const float *__restrict__ lsepart,
+                                                           __nv_bfloat16 *__restrict__ O,
+                                                           __nv_bfloat16 *__restrict__ O_lo, float *__restrict__ lse,
+                                                           size_t rows, int T, int k, int nb, int G) {
     const size_t row = static_cast<size_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
-    const size_t region = (row / T) * list_stride(T, k, nb);
-    const int32_t *ps = pos + row * k;
+    // query row -> key/value head bh (whose selection, positions and partials it uses), head in group hi
+    const size_t qh = row / T, t = row % T;
+    const size_t bh = qh / G, hi = qh % G;
+    const size_t region = bh * list_stride(T, k, nb);
+    const int32_t *ps = pos + (bh * T + t) * k;
+    const int32_t *js = idx + (bh * T + t) * k;
+    const bool scaled = __ldg(bexp + (rows / T / G) * nb) != 0;
     float mx = -INFINITY;
     for (int i0 = 0; i0 < k; i0 += 32) {
         const int p = (i0 + lane < k) ? __ldg(ps + i0 + lane) : -1;
-        if (p >= 0) mx = fmaxf(mx, __ldg(lsepart + region + p));
+        if (p >= 0) mx = fmaxf(mx, __ldg(lsepart + (region + p) * G + hi));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float wsum = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int i0 = 0; i0 < k; i0 += 32) {
         const int p = (i0 + lane < k) ? __ldg(ps + i0 + lane) : -1;
-        const float w = (p >= 0) ? __expf(__ldg(lsepart + region + p) - mx) : 0.f;
+        float w = 0.f, wo = 0.f;
+        if (p >= 0) {
+            w = __expf(__ldg(lsepart + (region + p) * G + hi) - mx);
+            // the partial's weight with its range exponent restored
+            wo = scaled ? ldexpf(w, __ldg(bexp + bh * nb + __ldg(js + i0 + lane))) : w;
+        }
         wsum += w;
         const int n = min(32, k - i0);
         for (int s0 = 0; s0 < n; s0 += 8) {
@@ -198,93 +226,50 @@ __global__ void __launch_bounds__(256) sparse_merge_kernel(const int32_t *__rest
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const int pq = __shfl_sync(0xffffffffu, p, (s0 + q) & 31);
-                wu[q] = __shfl_sync(0xffffffffu, w, (s0 + q) & 31);
+                wu[q] = __shfl_sync(0xffffffffu, wo, (s0 + q) & 31);
                 u[q] = (s0 + q < n && pq >= 0)
-                           ? __ldg(reinterpret_cast<const uint2 *>(Opart + (region + pq) * 128) + lane)
+                           ? __ldg(reinterpret_cast<const uint2 *>(Opart + ((region + pq) * G + hi) * 128) + lane)
                            : make_uint2(0u, 0u);
             }
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                acc[0] += wu[q] * __uint_as_float(u[q].x << 16);
-                acc[1] += wu[q] * __uint_as_float(u[q].x & 0xFFFF0000u);
-                acc[2] += wu[q] * __uint_as_float(u[q].y << 16);
-                acc[3] += wu[q] * __uint_as_float(u[q].y & 0xFFFF0000u);
+                float f[4];
+                half4_to_f32(u[q], f);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[c] = fmaf(wu[q], f[c], acc[c]);
             }
         }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
     const float inv = 1.f / wsum;
-    TO *dst = O + row * 128 + lane * 4;
-    if constexpr (sizeof(TO) == 2) {
-        *reinterpret_cast<uint2 *>(dst) =
-            make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
-    } else {
-        *reinterpret_cast<float4 *>(dst) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    float o4[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) o4[c] = acc[c] * inv;
+    const uint32_t h01 = pack_bf16x2(o4[0], o4[1]), h23 = pack_bf16x2(o4[2], o4[3]);
+    reinterpret_cast<uint2 *>(O + row * 128)[lane] = make_uint2(h01, h23);
+    if (O_lo) {
+        const uint32_t l01 = pack_bf16x2(o4[0] - __uint_as_float(h01 << 16), o4[1] - __uint_as_float(h01 & 0xFFFF0000u));
+        const uint32_t l23 = pack_bf16x2(o4[2] - __uint_as_float(h23 << 16), o4[3] - __uint_as_float(h23 & 0xFFFF0000u));
+        reinterpret_cast<uint2 *>(O_lo + row * 128)[lane] = make_uint2(l01, l23);
     }
     if (lane == 0) lse[row] = mx + __logf(wsum);
 }
 
-// Sparse-stream dQ from its partials (head dimension 128):
-//   dQ[row] = (accumulate ? dQ[row] : 0) + sum_i dQpart[pos[row * k + i]]
-// summed in fp32 and rounded once.  The partial of (query, slot i) sits at list
-// position pos[row * k + i] of its head's region (-1: slot not attended).  Lane i
-// holds slot i's position, so the slots' row loads are all in flight at once; lane
-// l then owns columns 4l .. 4l+3.
-__global__ void __launch_bounds__(256) dq_merge_kernel(const int32_t *__restrict__ pos,
-                                                       const __nv_bfloat16 *__restrict__ dQpart,
-                                                       __nv_bfloat16 *__restrict__ dQ, size_t rows, int T, int k,
-                                                       int nb, int accumulate) {
-    const size_t row = static_cast<size_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    const size_t region = (row / T) * list_stride(T, k, nb);
-    const int32_t *ps = pos + row * k;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    uint2 *dst = reinterpret_cast<uint2 *>(dQ + row * 128) + lane;
-    if (accumulate) {
-        const uint2 o = *dst;
-        acc[0] = __uint_as_float(o.x << 16);
-        acc[1] = __uint_as_float(o.x & 0xFFFF0000u);
-        acc[2] = __uint_as_float(o.y << 16);
-        acc[3] = __uint_as_float(o.y & 0xFFFF0000u);
-    }
-    for (int i0 = 0; i0 < k; i0 += 32) {
-        const int p = (i0 + lane < k) ? __ldg(ps + i0 + lane) : -1;
-        const int n = min(32, k - i0);
-        for (int s0 = 0; s0 < n; s0 += 8) {
-            uint2 u[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int pq = __shfl_sync(0xffffffffu, p, (s0 + q) & 31);
-                u[q] = (s0 + q < n && pq >= 0)
-                           ? __ldg(reinterpret_cast<const uint2 *>(dQpart + (region + pq) * 128) + lane)
-                           : make_uint2(0u, 0u);
-            }
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                acc[0] += __uint_as_float(u[q].x << 16);
-                acc[1] += __uint_as_float(u[q].x & 0xFFFF0000u);
-                acc[2] += __uint_as_float(u[q].y << 16);
-                acc[3] += __uint_as_float(u[q].y & 0xFFFF0000u);
-            }
-        }
-    }
-    *dst = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
-}
-
-// D[row] = sum_c dO[row,c] * O[row,c] (one warp per row); zero the fp32 dQ
-// accumulator row when there is one (the sparse tensor-core stream has partials instead).
+// D[row] = sum_c dO[row,c] * (O[row,c] + O_lo[row,c]) (one warp per row; O_lo may be
+// NULL); zero the fp32 dQ accumulator row.
 template <typename T>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const T *__restrict__ dO, const T *__restrict__ O,
-                                                       float *__restrict__ Dvec, float *__restrict__ dQacc,
-                                                       size_t rows, int d) {
+                                                       const T *__restrict__ O_lo, float *__restrict__ Dvec,
+                                                       float *__restrict__ dQacc, size_t rows, int d) {
     const size_t row = static_cast<size_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
     float acc = 0.f;
     for (int c = lane; c < d; c += 32) {
-        acc += to_f32(dO[row * d + c]) * to_f32(O[row * d + c]);
+        float o = to_f32(O[row * d + c]);
+        if (O_lo) o += to_f32(O_lo[row * d + c]);
+        acc += to_f32(dO[row * d + c]) * o;
         if (dQacc) dQacc[row * d + c] = 0.f;
     }
 #pragma unroll
@@ -308,8 +293,8 @@ __global__ void __launch_bounds__(256) acc_to_out_kernel(const float *__restrict
 }
 
 // ---------------------------------------------------------------------------
-// Alignment loss (paper section 5).  huber_beta is symmetric, so both
-// directions share sum_i huber(Of_i - Os_i):
+// Alignment loss (paper section 5).  Both per-element losses are symmetric, so
+// both directions share sum_i l(Of_i - Os_i):
 //   loss = (w_sparsity + w_commit) * sum / n
 // Pass 1: fixed grid of kAlignBlocks CTAs, per-CTA partial sums (fp32);
 // pass 2: one warp adds the partials in fixed order (fp64) -> deterministic.
@@ -326,9 +311,20 @@ __device__ __forceinline__ float huber_slope(float x, float beta) {
     return x > 0.f ? 1.f : -1.f;
 }
 
+// Per-element alignment loss and slope: kind 0 SmoothL1, kind 1 adjusted L2 (0.5 x^2 / beta
+// everywhere, the section 7.5 ablation variant).
+__device__ __forceinline__ float align_elem(int kind, float x, float beta) {
+    return kind ? 0.5f * x * x / beta : huber(x, beta);
+}
+
+__device__ __forceinline__ float align_slope(int kind, float x, float beta) {
+    return kind ? x / beta : huber_slope(x, beta);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) align_fwd_partial_kernel(const T *__restrict__ Of, const T *__restrict__ Os,
-                                                                float *__restrict__ partial, size_t n, float beta) {
+                                                                float *__restrict__ partial, size_t n, int kind,
+                                                                float beta) {
     constexpr int V = Vec16<T>::N;
     __shared__ float red[8];
     float acc = 0.f;
@@ -339,10 +335,11 @@ __global__ void __launch_bounds__(256) align_fwd_partial_kernel(const T *__restr
         Vec16<T>::load(Of + i * V, a);
         Vec16<T>::load(Os + i * V, b);
 #pragma unroll
-        for (int q = 0; q < V; ++q) acc += huber(a[q] - b[q], beta);
+        for (int q = 0; q < V; ++q) acc += align_elem(kind, a[q] - b[q], beta);
     }
     if (blockIdx.x == 0)
-        for (size_t i = nv * V + threadIdx.x; i < n; i += blockDim.x) acc += huber(to_f32(Of[i]) - to_f32(Os[i]), beta);
+        for (size_t i = nv * V + threadIdx.x; i < n; i += blockDim.x)
+            acc += align_elem(kind, to_f32(Of[i]) - to_f32(Os[i]), beta);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
@@ -367,15 +364,15 @@ __global__ void align_fwd_final_kernel(const float *__restrict__ partial, int np
 template <typename T>
 __global__ void __launch_bounds__(256) align_bwd_kernel(const T *__restrict__ Of, const T *__restrict__ Os,
                                                         const float *__restrict__ dloss, T *__restrict__ dOf,
-                                                        T *__restrict__ dOs, size_t n, float beta, float w_s,
-                                                        float w_c, int accumulate) {
+                                                        T *__restrict__ dOs, size_t n, int kind, float beta,
+                                                        float w_s, float w_c, int accumulate) {
     const float g = __ldg(dloss) / static_cast<float>(n);
     const float cf = g * w_s, cs = g * w_c;
     for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<size_t>(gridDim.x) * blockDim.x) {
         const float x = to_f32(Of[i]) - to_f32(Os[i]);
-        const float h = huber_slope(x, beta);
-        float gf = cf * h, gs = -cs * h;  // huber' is odd: huber'(Os - Of) = -huber'(Of - Os)
+        const float h = align_slope(kind, x, beta);
+        float gf = cf * h, gs = -cs * h;  // both slopes are odd: l'(Os - Of) = -l'(Of - Os)
         if (accumulate & 1) gf += to_f32(dOf[i]);
         if (accumulate & 2) gs += to_f32(dOs[i]);
         if constexpr (sizeof(T) == 2) {

@@ -7,6 +7,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace ssa {
@@ -69,21 +70,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Bounded wait on phase `parity`.  Returns false (and records the site) when the
-// phase did not complete within kWaitLimitNs or when another thread of the CTA
+// phase did not complete within limit_ns or when another thread of the CTA
 // already aborted (abort flag in shared memory).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          unsigned site) {
+                                          unsigned site, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             *abort_flag = 1;
             record_error(ERR_TIMEOUT, site);
             return false;
         }
     }
+}
+
+// Self-test of the bounded wait: one warp waits on an mbarrier that nothing
+// arrives on, with a short limit; the wait gives up, records the timeout in the
+// device error word and the kernel returns (no fault, no trap).
+__global__ void wait_probe_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);  // expects one arrival that never comes
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, 0x7F0, limit_ns);
+    __syncwarp();
 }
 
 // Bounded wait used on exit paths to let this CTA's own copies in flight land
@@ -382,6 +399,17 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
+}
+
+// Pack two floats into an fp16x2 word, `lo` in the low half (round to nearest even).
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Named barrier over `count` threads (ids other than 0, which __syncthreads uses).
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Pack two floats into a bf16x2 word, `lo` in the low half (round to nearest even).

@@ -53,44 +53,75 @@ __device__ __forceinline__ float to_f32<float>(float x) {
 }
 
 // ---------------------------------------------------------------------------
-// Pooling: one CTA (256 threads) per (head, block).  Thread (row group g,
-// column vector c) sums rows g, g+G, ... in order; the G partial sums are then
-// added in fixed order and divided by s.
+// Pooling: one warp per (head, block), no shared memory and no CTA barrier.
+// A warp instruction reads 512 contiguous bytes: lane l takes the 16-byte unit
+// l % U of row l / U (U = units per row, R = 32 / U rows per instruction), so
+// every load of the block is a full coalesced line set.  Each lane keeps
+// kPoolInFlight loads in flight, sums its unit's columns in fp32 over the rows
+// it visits (in row order), and the R lanes that hold the same columns are
+// combined by shuffles; lanes of row slot 0 write Kbar = sum / s.
 // ---------------------------------------------------------------------------
-template <typename T>
-__global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ K, float *__restrict__ Kbar, int T_len, int d,
-                                                   int s, int nb) {
-    constexpr int V = Vec16<T>::N;
-    __shared__ float part[256 * V];
-    const int tpr = d / V;                  // threads per row
-    const int G = blockDim.x / tpr;         // rows in flight
-    const int g = threadIdx.x / tpr, cv = threadIdx.x % tpr;
-    const int bh = blockIdx.x / nb, j = blockIdx.x % nb;
-    const T *base = K + (static_cast<size_t>(bh) * T_len + static_cast<size_t>(j) * s) * d + cv * V;
+constexpr int kPoolWarps = 8;     // warps (blocks) per CTA
+constexpr int kPoolInFlight = 16;  // 16-byte loads in flight per lane (one pass covers R * 16 <= 64 rows)
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kPoolWarps * 32) pool_kernel(const T *__restrict__ K, float *__restrict__ Kbar,
+                                                             int T_len, int s, int nb, size_t units) {
+    constexpr int V = Vec16<T>::N;      // elements per 16-byte unit
+    constexpr int U = D / V;            // units per row
+    constexpr int R = 32 / U;           // rows per warp instruction
+    const int lane = threadIdx.x & 31;
+    const size_t u = static_cast<size_t>(blockIdx.x) * kPoolWarps + (threadIdx.x >> 5);
+    if (u >= units) return;
+    const size_t bh = u / nb;
+    const int j = static_cast<int>(u % nb);
+    const int cu = lane % U, ro = lane / U;
+    const T *base = K + (bh * T_len + static_cast<size_t>(j) * s) * D + cu * V;
     float acc[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) acc[i] = 0.f;
-#pragma unroll 8
-    for (int r = g; r < s; r += G) {
-        float f[V];
-        Vec16<T>::load(base + static_cast<size_t>(r) * d, f);
+    for (int r0 = 0; r0 < s; r0 += R * kPoolInFlight) {
+        // all the raw 16-byte units first (kPoolInFlight loads in flight), then the fp32 sums
+        // (s in {64, 128} is a multiple of the R * kPoolInFlight <= 64 rows of one pass)
+        uint4 raw[kPoolInFlight];
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] += f[i];
+        for (int q = 0; q < kPoolInFlight; ++q)
+            raw[q] = __ldg(reinterpret_cast<const uint4 *>(base + static_cast<size_t>(r0 + q * R + ro) * D));
+#pragma unroll
+        for (int q = 0; q < kPoolInFlight; ++q) {
+            const uint32_t w[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
+            if constexpr (sizeof(T) == 2) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    acc[2 * i] += __uint_as_float(w[i] << 16);
+                    acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i] += __uint_as_float(w[i]);
+            }
+        }
     }
+    // lanes ro = 0 .. R-1 of the same unit hold partial sums of the same columns
 #pragma unroll
-    for (int i = 0; i < V; ++i) part[g * d + cv * V + i] = acc[i];
-    __syncthreads();
-    for (int c = threadIdx.x; c < d; c += blockDim.x) {
-        float sum = 0.f;
-        for (int q = 0; q < G; ++q) sum += part[q * d + c];
-        Kbar[(static_cast<size_t>(bh) * nb + j) * d + c] = sum / static_cast<float>(s);
+    for (int o = U; o < 32; o <<= 1)
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    if (ro == 0) {
+        const float inv = 1.f / static_cast<float>(s);
+        float4 *dst = reinterpret_cast<float4 *>(Kbar + u * D + cu * V);
+#pragma unroll
+        for (int i = 0; i < V; i += 4)
+            dst[i / 4] = make_float4(acc[i] * inv, acc[i + 1] * inv, acc[i + 2] * inv, acc[i + 3] * inv);
     }
 }
 
 // ---------------------------------------------------------------------------
-// Selection.  One CTA (256 threads) per 32 consecutive queries of one head
-// (all in the same block, since s is a multiple of 32); warp w owns queries
-// 4w .. 4w+3 from scoring to output.
+// Selection.  One CTA (256 threads) per 32 consecutive queries of one key/value
+// head (all in the same block, since s is a multiple of 32); warp w owns queries
+// 4w .. 4w+3 from scoring to output.  With G query heads per key head the query
+// row scored is the fp32 sum of the group's rows (the sum of the heads' scores up
+// to fp32 rounding).
 //   scores: r[q][j] = q . Kbar_j for j < b(t), fp32 FMA in column order; Kbar
 //           staged 64 blocks at a time; lane l of warp w scores blocks l and
 //           l + 32 of the chunk for the warp's 4 queries;
@@ -209,34 +240,10 @@ __device__ __forceinline__ void select_row(const float *row, int n, int want, in
     select_emit<KPL>(key, st, n, want, bt, k, out, lane);
 }
 
-// Two rows' searches interleaved in one warp: their chains of dependent warp reductions overlap.
-template <int KPL>
-__device__ __forceinline__ void select_row2(const float *rowA, int nA, int wantA, int btA, int32_t *outA,
-                                            const float *rowB, int nB, int wantB, int btB, int32_t *outB, int k,
-                                            int lane) {
-    uint32_t ka[KPL], kb[KPL];
-    select_load<KPL>(rowA, nA, ka, lane);
-    select_load<KPL>(rowB, nB, kb, lane);
-    SelSearch sa, sb;
-    sa.done = !(wantA > 0 && wantA < nA);
-    sb.done = !(wantB > 0 && wantB < nB);
-#pragma unroll 1
-    for (int b = 31; b >= 0 && !(sa.done && sb.done); --b) {
-        const unsigned ta = select_count<KPL>(ka, sa.tau | (1u << b));
-        const unsigned tb = select_count<KPL>(kb, sb.tau | (1u << b));
-        select_step(sa, wantA, b, ta);
-        select_step(sb, wantB, b, tb);
-    }
-    select_finish<KPL>(ka, sa, wantA, nA);
-    select_finish<KPL>(kb, sb, wantB, nB);
-    if (outA) select_emit<KPL>(ka, sa, nA, wantA, btA, k, outA, lane);
-    if (outB) select_emit<KPL>(kb, sb, nB, wantB, btB, k, outB, lane);
-}
-
 template <typename T, int KPL>
 __global__ void __launch_bounds__(256) select_kernel(const T *__restrict__ Q, const float *__restrict__ Kbar,
                                                      int32_t *__restrict__ idx, int T_len, int d, int s, int k,
-                                                     int nb) {
+                                                     int nb, int G) {
     extern __shared__ __align__(16) float sm[];
     const int dp = d + 4;
     float *sQ = sm;                       // [32][dp]
@@ -247,9 +254,13 @@ __global__ void __launch_bounds__(256) select_kernel(const T *__restrict__ Q, co
     const int bt = t0 / s;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+    // the query row of the group: the fp32 sum of its G heads' rows (G = 1: the row itself)
     for (int e = tid; e < kSelQ * d; e += blockDim.x) {
         const int qi = e / d, c = e % d;
-        sQ[qi * dp + c] = to_f32(Q[(static_cast<size_t>(bh) * T_len + t0 + qi) * d + c]);
+        float v = 0.f;
+        for (int hi = 0; hi < G; ++hi)
+            v += to_f32(Q[((static_cast<size_t>(bh) * G + hi) * T_len + t0 + qi) * d + c]);
+        sQ[qi * dp + c] = v;
     }
     for (int jc = 0; jc < bt; jc += kSelJ) {
         const int nj = min(kSelJ, bt - jc);
@@ -300,25 +311,36 @@ __global__ void __launch_bounds__(256) select_kernel(const T *__restrict__ Q, co
 // Selection with the block scores on the tensor cores (bf16 Q, d = 128, nb <= 256).
 // One CTA (512 threads) per 128 consecutive queries of one head:
 //   scores: r[q][j] = q . Kbar_j as one dense contraction S = Q Kbar^T (M = 128 queries,
-//           N = 64 blocks per group, K = d) in tensor memory.  Kbar (fp32) is split into
+//           N = 64 blocks per group, K = d) in tensor memory; with G query heads per key
+//           head, the G heads' contractions accumulate into the same scores (the group's
+//           selection ranks by the sum of its heads' scores).  Kbar (fp32) is split into
 //           three bf16 terms, hi = bf16(x), mid = bf16(x - hi), lo = bf16(x - hi - mid),
 //           which carry its 24 significant bits; the products with the bf16 query are
 //           exact and the three contractions accumulate in fp32;
-//   top-(k-1): the scores are staged row-major in shared memory and each of the 16 warps runs
-//           the threshold search of select_row on 8 of the 128 rows (a search is a chain of
-//           dependent warp reductions, so many rows are kept in flight).
+//   top-(k-1): thread <-> query row (tensor-memory lane).  Warp w reads rows
+//           32 (w & 3) .. +31 and the 32-column chunks c = w >> 2, (w >> 2) + 4 of the
+//           scores straight from tensor memory into registers (64 per thread at most), so
+//           the four warps of a row group share each row's candidates.  The (k-1)-th
+//           largest order key tau is built bit by bit from the most significant end: each
+//           step counts, per row, the scores at or above the candidate threshold (compared
+//           as floats against the threshold's value), and the four partial counts meet in
+//           shared memory behind one named barrier of the row group; the search stops at a
+//           threshold with exactly k-1 scores at or above it.  Otherwise the scores above
+//           tau are kept and those equal to it in ascending block order until k-1 are
+//           chosen (lowest index wins ties).  Each warp then leaves the chosen columns of
+//           its chunks as 32-bit masks, and one warp per row group writes the row:
+//           chosen blocks ascending, b(t), -1 padding.
 // ---------------------------------------------------------------------------
 constexpr int kSelTcRows = 128;
 constexpr int kSelTcThreads = 512;
-constexpr int kSelTcWarps = kSelTcThreads / 32;
 constexpr int kSelTcMaxBlocks = 256;
-constexpr int kSelTcPitch = kSelTcMaxBlocks + 4;  // fp32 score row pitch: conflict-free staging
 
 struct SelTcSmem {
     static constexpr int kQ = 0;                      // 128 rows x 128 bf16: 2 swizzled 16 KB chunks
     static constexpr int kB = 2 * 16384;              // hi / mid / lo: 3 x (64 blocks x 128 bf16), 16 KB each
-    static constexpr int kS = kB + 3 * 16384;         // 128 x kSelTcPitch fp32 scores
-    static constexpr int kBar = kS + kSelTcRows * kSelTcPitch * 4;
+    static constexpr int kCnt = kB + 3 * 16384;       // [2 steps][4 column groups][128 rows] partial counts
+    static constexpr int kMask = kCnt + 2 * 4 * 128 * 4;  // [8 chunks][128 rows] x {above, equal} masks
+    static constexpr int kBar = kMask + 2 * 8 * 128 * 4;
     static constexpr int kTotal = kBar + 64;
 };
 
@@ -326,15 +348,27 @@ __device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t
     asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
 
+// The float whose order key is `key` (inverse of order_key): key(x) >= key <=> x >= value, for every
+// non-NaN x.  Keys above that of +inf map to NaN (nothing compares at or above them); keys at or below
+// that of -inf map to -inf (everything does).
+__device__ __forceinline__ float key_value(uint32_t key) {
+    if (key & 0x80000000u) return __uint_as_float(key & 0x7FFFFFFFu);
+    if (key >= 0x00800000u) return __uint_as_float(~key);
+    return -INFINITY;
+}
+
 __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_bfloat16 *__restrict__ Q,
                                                            const float *__restrict__ Kbar, int32_t *__restrict__ idx,
-                                                           int T_len, int s, int k, int nb) {
+                                                           int T_len, int s, int k, int nb, int G) {
     using L = SelTcSmem;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bar_mma = reinterpret_cast<uint64_t *>(smem + L::kBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kBar + 8);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kBar + 16);
+    int *cnt_sm = reinterpret_cast<int *>(smem + L::kCnt);          // [2][4][128]
+    uint32_t *gt_sm = reinterpret_cast<uint32_t *>(smem + L::kMask);  // [8][128]
+    uint32_t *eq_sm = gt_sm + 8 * 128;                                // [8][128]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.y, t0 = blockIdx.x * kSelTcRows;
     const size_t head_rows = static_cast<size_t>(bh) * T_len;
@@ -342,7 +376,6 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
     const int nbc = min(last / s, nb);  // blocks scored by some row of the tile (j < b(t))
     const int ngroups = (nbc + 63) / 64;
     const uint32_t sQ = smem_u32(smem + L::kQ), sB = smem_u32(smem + L::kB);
-    float *sS = reinterpret_cast<float *>(smem + L::kS);
 
     if (tid == 0) {
         mbar_init(bar_mma, 1);
@@ -353,28 +386,31 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
         tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
     }
-    {
-        // query rows -> K-major 128-byte-swizzled tile; rows past T are zero-filled
+    // query rows of head (bh * G + hi) -> K-major 128-byte-swizzled tile; rows past T are zero-filled
+    auto load_q = [&](int hi) {
         const int u = tid & 15;
+        const size_t qrows = (static_cast<size_t>(bh) * G + hi) * T_len;
         for (int row = tid >> 4; row < kSelTcRows; row += kSelTcThreads / 16) {
             const int t = t0 + row;
             const bool valid = t < T_len;
             const uint32_t dst = sQ + (u >> 3) * 16384 + row * 128 + ((((u & 7) ^ (row & 7)) & 7) << 4);
-            cp_async_16(dst, Q + (head_rows + (valid ? t : 0)) * 128 + u * 8, valid ? 16u : 0u);
+            cp_async_16(dst, Q + (qrows + (valid ? t : 0)) * 128 + u * 8, valid ? 16u : 0u);
         }
         cp_async_wait_all();
-    }
-    fence_proxy_async_smem();
+        fence_proxy_async_smem();
+    };
+    if (G == 1) load_q(0);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
-    for (int gi = 0; gi < ngroups; ++gi) {
+    int phase = 0;  // completed MMA batches (bar_mma phases)
+    for (int gi = 0; gi < ngroups && ok; ++gi) {
         // Kbar rows 64gi .. 64gi+63 -> hi / mid / lo tiles (K-major, swizzled); rows >= nbc are zero.
         // Lane c4 of a warp takes dims 4c4 .. 4c4+3 of one row: two 128-byte row halves per store.
         const int c4 = lane;
-        for (int jj = warp; jj < 64; jj += kSelTcWarps) {
+        for (int jj = warp; jj < 64; jj += kSelTcThreads / 32) {
             const int j = 64 * gi + jj;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
             if (j < nbc) v = __ldg(reinterpret_cast<const float4 *>(Kbar + (static_cast<size_t>(bh) * nb + j) * 128) + c4);
@@ -390,52 +426,137 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
             st_shared_v2(sB + 2 * 16384 + off, l01, l23);
         }
         fence_proxy_async_smem();  // generic-proxy tile writes -> tensor-core reads
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, false, false);
+        // with grouped query heads the group's tiles are added one after another into the same scores
+        for (int hi = 0; hi < G && ok; ++hi) {
+            if (G > 1) load_q(hi);  // the previous batch's MMAs have read the tile (waited below)
+            __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
-            for (int sp = 0; sp < 3; ++sp)
+                for (int sp = 0; sp < 3; ++sp)
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ss(tmem + 64 * gi, smem_desc_sw128(sQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
-                                smem_desc_sw128(sB + sp * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32, 16), id,
-                                (sp > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(bar_mma);
-        }
-        // the next group rewrites the split tiles only after these MMAs have read them
-        if (!mbar_wait(bar_mma, gi & 1, abort_flag, 0x501)) {
-            ok = false;
-            break;
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ss(tmem + 64 * gi, smem_desc_sw128(sQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
+                                    smem_desc_sw128(sB + sp * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32, 16), id,
+                                    (hi > 0 || sp > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar_mma);
+            }
+            // the split tiles and the query tile are rewritten only after these MMAs have read them
+            if (!mbar_wait(bar_mma, phase & 1, abort_flag, 0x501)) ok = false;
+            ++phase;
         }
     }
+    // one verdict for the whole CTA: the loads below are warp-collective and the row groups meet on
+    // named barriers, so every thread must take the same branch
+    ok = __syncthreads_and(ok ? 1 : 0) != 0;
     tc_fence_after();
-    // scores -> shared memory: warps 0-3, thread <-> row (tensor-memory lane)
-    if (ok && warp < 4) {
-        const int row = warp * 32 + lane;
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        const uint32_t dst = smem_u32(sS + row * kSelTcPitch);
-        for (int c = 0; c < 2 * ngroups; ++c) {
+
+    // ---- top-(k-1) per row: thread <-> row, four warps (column groups) per row group ----
+    const int rg = warp & 3, cg = warp >> 2;  // row group, column group
+    const int r = rg * 32 + lane;
+    const int t = t0 + r;
+    const bool valid_row = t < T_len;
+    const int bt = t / s;
+    const int n = valid_row ? min(bt, nb) : 0;  // candidates j < b(t)  (uniform over a warp: s >= 64)
+    const int want = min(k - 1, n);
+    const int nch = (nbc + 31) / 32;           // score chunks of the tile (<= 8)
+    const uint32_t lane_off = static_cast<uint32_t>(rg * 32) << 16;
+    float x[2][32];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int c = cg + 4 * i;
+        if (ok && c < nch) {  // warp-uniform
             uint32_t v[32];
             tmem_ld32_async(tmem + lane_off + 32 * c, v);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 8; ++q) st_shared_v4(dst + (32 * c + 4 * q) * 4, v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            for (int e = 0; e < 32; ++e) x[i][e] = (32 * c + e < n) ? __uint_as_float(v[e]) : __int_as_float(0x7FC00000);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[i][e] = __int_as_float(0x7FC00000);  // NaN: never counted
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, 256);
-    // top-(k-1) per row: warp w takes rows w, w + 16, ..., two at a time (rows past T write nothing)
-    for (int row = warp; row < kSelTcRows; row += 2 * kSelTcWarps) {
-        const int ta = t0 + row, tb = t0 + row + kSelTcWarps;
-        const int bta = ta / s, btb = tb / s;
-        const bool va = ta < T_len, vb = tb < T_len;
-        select_row2<8>(sS + row * kSelTcPitch, va ? bta : 0, va ? min(k - 1, bta) : 0, bta,
-                       va ? idx + (head_rows + ta) * k : nullptr, sS + (row + kSelTcWarps) * kSelTcPitch,
-                       vb ? btb : 0, vb ? min(k - 1, btb) : 0, btb, vb ? idx + (head_rows + tb) * k : nullptr, k,
-                       lane);
+
+    // chunks of this warp that hold candidates of its rows (n is uniform over the warp)
+    const int mych = (cg < (n + 31) / 32 ? 1 : 0) + (cg + 4 < (n + 31) / 32 ? 1 : 0);
+    auto count_ge = [&](float f) {
+        int c = 0;
+        if (mych > 0) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) c += (x[0][e] >= f) ? 1 : 0;
+        }
+        if (mych > 1) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) c += (x[1][e] >= f) ? 1 : 0;
+        }
+        return c;
+    };
+    // the row group's four warps meet on named barrier 1 + rg (128 threads)
+    const bool search = ok && want > 0 && want < n;  // uniform over the row group
+    uint32_t tau = 0u;
+    bool exact = false;
+    if (search) {
+        bool done = false;
+        int step = 0;
+        for (int b = 31; b >= 0; --b, ++step) {
+            const uint32_t cand = tau | (1u << b);
+            const int part = count_ge(key_value(cand));
+            int *cs = cnt_sm + (step & 1) * 512;
+            cs[cg * 128 + r] = part;
+            named_barrier(1 + rg, 128);
+            const int tot = cs[r] + cs[128 + r] + cs[256 + r] + cs[384 + r];
+            if (!done && tot >= want) {
+                tau = cand;
+                if (tot == want) exact = done = true;
+            }
+            if (__all_sync(0xffffffffu, done)) break;  // the same rows and counts in all four warps
+        }
+    }
+    // chosen columns of this warp's chunks: above tau (at or above when exact), and the ties
+    const float ft = key_value(tau);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int c = cg + 4 * i;
+        if (c < nch) {
+            uint32_t gm = 0u, em = 0u;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const float v = x[i][e];
+                const bool above = search ? (exact ? v >= ft : v > ft) : (v == v);  // no search: every candidate
+                gm |= (above ? 1u : 0u) << e;
+                em |= ((search && !exact && v == ft) ? 1u : 0u) << e;
+            }
+            gt_sm[c * 128 + r] = gm;
+            eq_sm[c * 128 + r] = em;
+        }
+    }
+    __syncthreads();
+    if (cg == 0 && valid_row && ok) {
+        // need_eq: keys equal to tau taken in ascending block order until want are chosen
+        int above = 0;
+        for (int c = 0; c < nch; ++c) above += __popc(gt_sm[c * 128 + r]);
+        int need = search ? want - above : 0;
+        int32_t *out = idx + (head_rows + t) * k;
+        int pos = 0;
+        for (int c = 0; c < nch && pos < want; ++c) {
+            uint32_t m = gt_sm[c * 128 + r], e = eq_sm[c * 128 + r];
+            while (e != 0u && need > 0) {
+                m |= e & (~e + 1u);  // lowest equal column
+                e &= e - 1u;
+                --need;
+            }
+            while (m != 0u && pos < want) {
+                out[pos++] = 32 * c + __ffs(m) - 1;
+                m &= m - 1u;
+            }
+        }
+        out[pos++] = bt;
+        for (; pos < k; ++pos) out[pos] = -1;
     }
 }
 

@@ -8,7 +8,6 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
-#include <mutex>
 
 #include "ssa.h"
 
@@ -18,6 +17,8 @@
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "attn_bwd.cuh"
+#include "decode.cuh"
+#include "rope.cuh"
 
 using namespace ssa;
 
@@ -26,7 +27,9 @@ namespace {
 struct Shape {
     int B, H, T, d, s, k, dtype;
     float scale;
-    size_t BH, rows;  // rows = B*H*T
+    int Hk, G;         // key/value heads, query heads per key/value head
+    size_t BH, rows;   // query heads B*H, query rows B*H*T
+    size_t BHk, krows; // key/value heads B*Hk, key rows B*Hk*T
     int nb;
     size_t esz;       // element size in bytes
     bool tc;          // tensor-core path (bf16, d == 128)
@@ -48,8 +51,13 @@ ssa_status_t check_dims(const ssa_dims_t *dims, Shape &S, bool need_k) {
     if (S.d != 64 && S.d != 128) return SSA_ERR_UNSUPPORTED;
     if (S.s != 64 && S.s != 128) return SSA_ERR_UNSUPPORTED;
     if (S.T % S.s != 0) return SSA_ERR_UNSUPPORTED;
+    S.Hk = dims->Hkv ? dims->Hkv : S.H;
+    if (S.Hk < 1 || S.H % S.Hk != 0) return SSA_ERR_INVALID_ARG;
+    S.G = S.H / S.Hk;
     S.BH = static_cast<size_t>(S.B) * S.H;
     S.rows = S.BH * S.T;
+    S.BHk = static_cast<size_t>(S.B) * S.Hk;
+    S.krows = S.BHk * S.T;
     if (S.rows > 0x7FFFFFFFull) return SSA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
     S.nb = S.T / S.s;
     if (need_k) {
@@ -58,10 +66,12 @@ ssa_status_t check_dims(const ssa_dims_t *dims, Shape &S, bool need_k) {
     }
     S.esz = S.dtype == SSA_DT_BF16 ? 2 : 4;
     S.tc = S.dtype == SSA_DT_BF16 && S.d == 128;
+    // a tensor-core tile holds 128 / G list entries for each of the G heads of a group
+    if (S.tc && 128 % S.G != 0) return SSA_ERR_UNSUPPORTED;
     // the sparse index packs (t << 8) | slot into an int32
     if (need_k && S.tc && (S.k > 256 || S.T >= (1 << 23))) return SSA_ERR_UNSUPPORTED;
-    // list positions of the whole index (and TMA row coordinates of the partials) fit an int32
-    if (need_k && S.tc && S.BH * list_stride(S.T, S.k, S.nb) >= (size_t(1) << 31)) return SSA_ERR_UNSUPPORTED;
+    // list positions of the whole index (and TMA row coordinates of the G partial rows per entry) fit an int32
+    if (need_k && S.tc && S.BHk * list_stride(S.T, S.k, S.nb) * S.G >= (size_t(1) << 31)) return SSA_ERR_UNSUPPORTED;
     // one warp's staging of the index fill must fit in shared memory
     if (need_k && S.tc && index_fill_warp_ints(S.nb, S.k) * 4 > 227 * 1024) return SSA_ERR_UNSUPPORTED;
     return SSA_OK;
@@ -69,54 +79,64 @@ ssa_status_t check_dims(const ssa_dims_t *dims, Shape &S, bool need_k) {
 
 inline size_t align_up(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Workspace layout of the sparse index.
+// Layout of the inverse selection index (the `index` buffer of ssa_sparse_index, or
+// the head of a sparse call's workspace when the caller passes none).
 struct IndexWs {
     int *cnt, *lstart, *llen;
     int32_t *entries;  // per head: list_stride(T, k, nb) entries, block lists on 128-entry boundaries
+    int32_t *pos;      // [B*H*T, k] list position of every (query, slot), -1 when unused
     int nch;
 };
 
 size_t index_bytes(const Shape &S) {
+    if (!S.tc) return 0;
     const size_t nch = (S.T + kIdxChunk - 1) / kIdxChunk;
-    return align_up(S.BH * nch * S.nb * 4) + 2 * align_up(S.BH * S.nb * 4) +
-           align_up(S.BH * list_stride(S.T, S.k, S.nb) * 4);
+    return align_up(S.BHk * nch * S.nb * 4) + 2 * align_up(S.BHk * S.nb * 4) +
+           align_up(S.BHk * list_stride(S.T, S.k, S.nb) * 4) + align_up(S.krows * S.k * 4);
 }
 
-uint8_t *carve_index(const Shape &S, uint8_t *p, IndexWs &W) {
+IndexWs carve_index(const Shape &S, const void *base) {
+    IndexWs W;
+    uint8_t *p = static_cast<uint8_t *>(const_cast<void *>(base));
     W.nch = (S.T + kIdxChunk - 1) / kIdxChunk;
     W.cnt = reinterpret_cast<int *>(p);
-    p += align_up(S.BH * W.nch * S.nb * 4);
+    p += align_up(S.BHk * W.nch * S.nb * 4);
     W.lstart = reinterpret_cast<int *>(p);
-    p += align_up(S.BH * S.nb * 4);
+    p += align_up(S.BHk * S.nb * 4);
     W.llen = reinterpret_cast<int *>(p);
-    p += align_up(S.BH * S.nb * 4);
+    p += align_up(S.BHk * S.nb * 4);
     W.entries = reinterpret_cast<int32_t *>(p);
-    p += align_up(S.BH * list_stride(S.T, S.k, S.nb) * 4);
-    return p;
+    p += align_up(S.BHk * list_stride(S.T, S.k, S.nb) * 4);
+    W.pos = reinterpret_cast<int32_t *>(p);
+    return W;
 }
 
 size_t ws_bytes_for(const Shape &S, int op) {
     switch (op) {
+        case SSA_OP_SPARSE_INDEX:
+            return index_bytes(S);
         case SSA_OP_SPARSE_FWD:
             if (!S.tc) return 0;
-            // index | partial outputs and lse by list position | list position of every (query, slot)
-            return index_bytes(S) + align_up(S.BH * list_stride(S.T, S.k, S.nb) * (128 * 2 + 4)) +
-                   align_up(S.rows * S.k * 4);
+            // index (used when the caller passes none) | fp16 partial outputs and fp32 partial lse,
+            // G rows per list position | range exponent of every key block, then a flag word
+            return index_bytes(S) + align_up(S.BHk * list_stride(S.T, S.k, S.nb) * S.G * (128 * 2 + 4)) +
+                   align_up(S.BHk * S.nb * 4 + 4);
         case SSA_OP_SPARSE_BWD:
-            // D | index | list position of every (query, slot) | bf16 dQ partials by list position
-            if (S.tc)
-                return align_up(S.rows * 4) + index_bytes(S) + align_up(S.rows * S.k * 4) +
-                       align_up(S.BH * list_stride(S.T, S.k, S.nb) * 128 * 2);
+            // D | index (used when the caller passes none) | fp32 dQ accumulator
+            if (S.tc) return align_up(S.rows * 4) + index_bytes(S) + align_up(S.rows * S.d * 4);
             [[fallthrough]];
         case SSA_OP_FULL_BWD: {
             size_t b = align_up(S.rows * 4) + align_up(S.rows * S.d * 4);  // D, dQacc
-            if (!S.tc) b += 2 * align_up(S.rows * S.d * 4);                // dKacc, dVacc
+            if (!S.tc) b += 2 * align_up(S.krows * S.d * 4);               // dKacc, dVacc
             return b;
         }
         case SSA_OP_FULL_FWD:
             return 0;
         case SSA_OP_ALIGN_FWD:
             return align_up(kAlignBlocks * 4);
+        case SSA_OP_DECODE:
+            // per (sequence, query head, slot): fp32 partial output and log-sum-exp
+            return align_up(S.BH * S.k * S.d * 4) + align_up(S.BH * S.k * 4);
         default:
             return 0;
     }
@@ -126,6 +146,16 @@ ssa_status_t check_ws(const Shape &S, int op, const void *ws, size_t ws_bytes) {
     const size_t need = ws_bytes_for(S, op);
     if (need == 0) return SSA_OK;
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u)) return SSA_ERR_WORKSPACE;
+    return SSA_OK;
+}
+
+// Bits of a backward call's `accumulate`; fp32 gradients are written with 16-byte accesses and
+// reduced into by the TMA unit, so their base addresses must be 16-byte aligned.
+ssa_status_t check_grads(int accumulate, const void *dQ, const void *dK, const void *dV) {
+    if (accumulate & ~static_cast<int>(SSA_BWD_ACCUMULATE | SSA_BWD_GRAD_FP32)) return SSA_ERR_INVALID_ARG;
+    if ((accumulate & SSA_BWD_GRAD_FP32) &&
+        ((reinterpret_cast<uintptr_t>(dQ) | reinterpret_cast<uintptr_t>(dK) | reinterpret_cast<uintptr_t>(dV)) & 15u))
+        return SSA_ERR_INVALID_ARG;
     return SSA_OK;
 }
 
@@ -193,120 +223,132 @@ unsigned grid_for(size_t n, unsigned per_block) {
 template <typename T, int KPL>
 ssa_status_t launch_select(const Shape &S, const void *Q, const float *Kbar, int32_t *idx, size_t sm, cudaStream_t st) {
     if (!set_smem(select_kernel<T, KPL>, sm)) return SSA_ERR_CUDA;
-    select_kernel<T, KPL><<<dim3(S.T / kSelQ, S.BH), 256, sm, st>>>((const T *)Q, Kbar, idx, S.T, S.d, S.s, S.k, S.nb);
+    select_kernel<T, KPL><<<dim3(S.T / kSelQ, S.BHk), 256, sm, st>>>((const T *)Q, Kbar, idx, S.T, S.d, S.s, S.k, S.nb,
+                                                                      S.G);
     return SSA_OK;
 }
 
-// Inverse selection index: entries of block j of head bh (query order).
-ssa_status_t build_index(const Shape &S, const int32_t *idx, IndexWs &W, cudaStream_t st, int32_t *pos = nullptr) {
+// Inverse selection index: entries of block j of head bh (query order) and the list
+// position of every (query, slot).
+ssa_status_t build_index(const Shape &S, const int32_t *idx, const IndexWs &W, cudaStream_t st) {
     const size_t hbytes = static_cast<size_t>(S.nb) * 4;
     if (!set_smem(index_count_kernel, hbytes)) return SSA_ERR_CUDA;
-    index_count_kernel<<<dim3(W.nch, S.BH), 256, hbytes, st>>>(idx, W.cnt, S.T, S.k, S.nb, W.nch);
-    index_scan_kernel<<<S.BH, 1024, 0, st>>>(W.cnt, W.lstart, W.llen, S.nb, W.nch);
+    index_count_kernel<<<dim3(W.nch, S.BHk), 256, hbytes, st>>>(idx, W.cnt, S.T, S.k, S.nb, W.nch);
+    index_scan_kernel<<<S.BHk, 1024, 0, st>>>(W.cnt, W.lstart, W.llen, S.nb, W.nch);
     // four warps (chunks) per CTA while their staging fits comfortably, else one
     const size_t wbytes = index_fill_warp_ints(S.nb, S.k) * 4;
     const int wpc = wbytes * 4 <= 160 * 1024 ? 4 : 1;
     if (!set_smem(index_fill_kernel, wbytes * wpc)) return SSA_ERR_CUDA;
-    index_fill_kernel<<<dim3((W.nch + wpc - 1) / wpc, S.BH), 32 * wpc, wbytes * wpc, st>>>(
-        idx, W.cnt, W.entries, pos, S.T, S.k, S.nb, W.nch);
+    index_fill_kernel<<<dim3((W.nch + wpc - 1) / wpc, S.BHk), 32 * wpc, wbytes * wpc, st>>>(
+        idx, W.cnt, W.entries, W.pos, S.T, S.k, S.nb, W.nch);
     return launch_status();
 }
 
 template <typename T>
 void launch_simt_fwd(const Shape &S, const void *Q, const void *K, const void *V, const int32_t *idx, void *O,
-                     float *lse, cudaStream_t st) {
+                     void *O_lo, float *lse, cudaStream_t st) {
     const unsigned g = static_cast<unsigned>((S.rows + 7) / 8);
+    T *lo = sizeof(T) == 2 ? (T *)O_lo : nullptr;  // the residual is only kept for bf16 outputs
     if (S.d == 64)
-        simt_fwd_kernel<T, 2><<<g, 256, 0, st>>>((const T *)Q, (const T *)K, (const T *)V, idx, (T *)O, lse, S.rows,
-                                                 S.T, S.s, S.k, S.scale);
+        simt_fwd_kernel<T, 2><<<g, 256, 0, st>>>((const T *)Q, (const T *)K, (const T *)V, idx, (T *)O, lo, lse,
+                                                 S.rows, S.T, S.s, S.k, S.scale, S.G);
     else
-        simt_fwd_kernel<T, 4><<<g, 256, 0, st>>>((const T *)Q, (const T *)K, (const T *)V, idx, (T *)O, lse, S.rows,
-                                                 S.T, S.s, S.k, S.scale);
+        simt_fwd_kernel<T, 4><<<g, 256, 0, st>>>((const T *)Q, (const T *)K, (const T *)V, idx, (T *)O, lo, lse,
+                                                 S.rows, S.T, S.s, S.k, S.scale, S.G);
 }
 
 template <typename T>
-ssa_status_t simt_bwd(const Shape &S, const void *Q, const void *K, const void *V, const void *O, const float *lse,
-                      const void *dO, const int32_t *idx, void *dQ, void *dK, void *dV, int accumulate, void *ws,
-                      cudaStream_t st) {
+ssa_status_t simt_bwd(const Shape &S, const void *Q, const void *K, const void *V, const void *O, const void *O_lo,
+                      const float *lse, const void *dO, const int32_t *idx, void *dQ, void *dK, void *dV,
+                      int accumulate, void *ws, cudaStream_t st) {
     uint8_t *p = static_cast<uint8_t *>(ws);
     float *Dvec = reinterpret_cast<float *>(p);
     p += align_up(S.rows * 4);
     float *dQacc = reinterpret_cast<float *>(p);
     p += align_up(S.rows * S.d * 4);
     float *dKacc = reinterpret_cast<float *>(p);
-    p += align_up(S.rows * S.d * 4);
+    p += align_up(S.krows * S.d * 4);
     float *dVacc = reinterpret_cast<float *>(p);
-    const size_t n = S.rows * S.d;
-    if (cudaMemsetAsync(dKacc, 0, n * 4, st) != cudaSuccess || cudaMemsetAsync(dVacc, 0, n * 4, st) != cudaSuccess)
+    const size_t n = S.rows * S.d, nk = S.krows * S.d;
+    if (cudaMemsetAsync(dKacc, 0, nk * 4, st) != cudaSuccess || cudaMemsetAsync(dVacc, 0, nk * 4, st) != cudaSuccess)
         return SSA_ERR_CUDA;
     const unsigned g = static_cast<unsigned>((S.rows + 7) / 8);
-    bwd_prep_kernel<T><<<g, 256, 0, st>>>((const T *)dO, (const T *)O, Dvec, dQacc, S.rows, S.d);
+    bwd_prep_kernel<T><<<g, 256, 0, st>>>((const T *)dO, (const T *)O, sizeof(T) == 2 ? (const T *)O_lo : nullptr,
+                                          Dvec, dQacc, S.rows, S.d);
     if (S.d == 64)
         simt_bwd_kernel<T, 2><<<g, 256, 0, st>>>((const T *)Q, (const T *)K, (const T *)V, (const T *)dO, idx, lse,
-                                                 Dvec, dQacc, dKacc, dVacc, S.rows, S.T, S.s, S.k, S.scale);
+                                                 Dvec, dQacc, dKacc, dVacc, S.rows, S.T, S.s, S.k, S.scale, S.G);
     else
         simt_bwd_kernel<T, 4><<<g, 256, 0, st>>>((const T *)Q, (const T *)K, (const T *)V, (const T *)dO, idx, lse,
-                                                 Dvec, dQacc, dKacc, dVacc, S.rows, S.T, S.s, S.k, S.scale);
-    const unsigned ge = grid_for(n, 256);
-    acc_to_out_kernel<T><<<ge, 256, 0, st>>>(dQacc, (T *)dQ, n, accumulate);
-    acc_to_out_kernel<T><<<ge, 256, 0, st>>>(dKacc, (T *)dK, n, accumulate);
-    acc_to_out_kernel<T><<<ge, 256, 0, st>>>(dVacc, (T *)dV, n, accumulate);
+                                                 Dvec, dQacc, dKacc, dVacc, S.rows, S.T, S.s, S.k, S.scale, S.G);
+    const unsigned ge = grid_for(n, 256), gk = grid_for(nk, 256);
+    const int acc = accumulate & SSA_BWD_ACCUMULATE;
+    if ((accumulate & SSA_BWD_GRAD_FP32) || sizeof(T) == 4) {
+        acc_to_out_kernel<float><<<ge, 256, 0, st>>>(dQacc, (float *)dQ, n, acc);
+        acc_to_out_kernel<float><<<gk, 256, 0, st>>>(dKacc, (float *)dK, nk, acc);
+        acc_to_out_kernel<float><<<gk, 256, 0, st>>>(dVacc, (float *)dV, nk, acc);
+    } else {
+        acc_to_out_kernel<T><<<ge, 256, 0, st>>>(dQacc, (T *)dQ, n, acc);
+        acc_to_out_kernel<T><<<gk, 256, 0, st>>>(dKacc, (T *)dK, nk, acc);
+        acc_to_out_kernel<T><<<gk, 256, 0, st>>>(dVacc, (T *)dV, nk, acc);
+    }
     return launch_status();
 }
 
 // Tensor-core backward shared by both streams.
-ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V, const void *O, const float *lse,
-                    const void *dO, const int32_t *idx, void *dQ, void *dK, void *dV, int accumulate, void *ws,
-                    cudaStream_t st) {
+ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V, const void *O, const void *O_lo,
+                    const float *lse, const void *dO, const int32_t *idx, const void *index, void *dQ, void *dK,
+                    void *dV, int accumulate, void *ws, cudaStream_t st) {
     uint8_t *p = static_cast<uint8_t *>(ws);
     float *Dvec = reinterpret_cast<float *>(p);
     p += align_up(S.rows * 4);
     const bool sparse = idx != nullptr;
-    // full stream: an fp32 dQ accumulator (TMA reduce-adds); sparse stream: one bf16 dQ
-    // partial per (query, slot) at its list position, summed by dq_merge_kernel
-    float *dQacc = nullptr;
-    __nv_bfloat16 *dQpart = nullptr;
-    int32_t *pos = nullptr;
-    const size_t nlist = sparse ? S.BH * list_stride(S.T, S.k, S.nb) : 0;
     IndexWs W{};
     if (sparse) {
-        p = carve_index(S, p, W);
-        pos = reinterpret_cast<int32_t *>(p);
-        p += align_up(S.rows * S.k * 4);
-        dQpart = reinterpret_cast<__nv_bfloat16 *>(p);
-        const ssa_status_t e = build_index(S, idx, W, st, pos);
-        if (e != SSA_OK) return e;
-    } else {
-        dQacc = reinterpret_cast<float *>(p);
+        // the caller's index, or one built here in the workspace
+        W = carve_index(S, index ? index : p);
+        p += index_bytes(S);
+        if (!index) {
+            const ssa_status_t e = build_index(S, idx, W, st);
+            if (e != SSA_OK) return e;
+        }
     }
+    // fp32 dQ accumulator: TMA reduce-adds of whole tiles (full) or vector reductions of gathered
+    // rows (sparse); zeroed by the prep kernel, converted (and added to dQ when accumulating) after.
+    // With fp32 gradients the caller's dQ is the accumulator itself (zeroed unless accumulating).
+    const bool acc = (accumulate & SSA_BWD_ACCUMULATE) != 0, g32 = (accumulate & SSA_BWD_GRAD_FP32) != 0;
+    float *dQacc = g32 ? static_cast<float *>(dQ) : reinterpret_cast<float *>(p);
     const unsigned g = static_cast<unsigned>((S.rows + 7) / 8);
-    bwd_prep_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16 *)dO, (const __nv_bfloat16 *)O, Dvec,
-                                                       dQacc, S.rows, S.d);
+    bwd_prep_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16 *)dO, (const __nv_bfloat16 *)O,
+                                                       (const __nv_bfloat16 *)O_lo, Dvec,
+                                                       (g32 && acc) ? nullptr : dQacc, S.rows, S.d);
     const int nkv = sparse ? S.s : 128;
     CUtensorMap tmK, tmV, tmQ, tmdO, tmdQ;
-    if (!make_tmap(&tmK, K, S.rows, nkv) || !make_tmap(&tmV, V, S.rows, nkv) || !make_tmap(&tmQ, Q, S.rows, 128) ||
-        !make_tmap(&tmdO, dO, S.rows, 128) ||
-        !(sparse ? make_tmap(&tmdQ, dQpart, nlist, 32) : make_tmap_f32(&tmdQ, dQacc, S.rows)))
+    if (!make_tmap(&tmK, K, S.krows, nkv) || !make_tmap(&tmV, V, S.krows, nkv) || !make_tmap(&tmQ, Q, S.rows, 128) ||
+        !make_tmap(&tmdO, dO, S.rows, 128) || !make_tmap_f32(&tmdQ, dQacc, S.rows))
         return SSA_ERR_CUDA;
     BwdArgs a{};
     a.Q = (const __nv_bfloat16 *)Q;
     a.dO = (const __nv_bfloat16 *)dO;
     a.lse = lse;
     a.Dvec = Dvec;
-    a.dK = (__nv_bfloat16 *)dK;
-    a.dV = (__nv_bfloat16 *)dV;
+    a.dQacc = dQacc;
+    a.dK = dK;
+    a.dV = dV;
     a.entries = W.entries;
     a.lstart = W.lstart;
     a.llen = W.llen;
-    a.BH = static_cast<int>(S.BH);
+    a.BH = static_cast<int>(S.BHk);
+    a.G = S.G;
     a.T = S.T;
     a.k = S.k;
     a.nb = S.nb;
     a.sparse = sparse ? 1 : 0;
-    a.accumulate = accumulate;
+    a.accumulate = acc ? 1 : 0;
+    a.grad_fp32 = g32 ? 1 : 0;
     a.scale = S.scale;
     a.scale_log2 = S.scale * kLog2e;
-    const unsigned units = static_cast<unsigned>(S.BH * (sparse ? S.nb : (S.T + 127) / 128));
+    const unsigned units = static_cast<unsigned>(S.BHk * (sparse ? S.nb : (S.T + 127) / 128));
     if (nkv == 128) {
         const size_t sm = BwdSmem<128>::kTotal + 1024;
         if (!set_smem(attn_bwd_kernel<128>, sm)) return SSA_ERR_CUDA;
@@ -316,12 +358,9 @@ ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V,
         if (!set_smem(attn_bwd_kernel<64>, sm)) return SSA_ERR_CUDA;
         attn_bwd_kernel<64><<<units, kBwdThreads, sm, st>>>(tmK, tmV, tmQ, tmdO, tmdQ, a);
     }
-    if (sparse) {
-        dq_merge_kernel<<<g, 256, 0, st>>>(pos, dQpart, (__nv_bfloat16 *)dQ, S.rows, S.T, S.k, S.nb, accumulate);
-    } else {
+    if (!g32) {
         const size_t n = S.rows * S.d;
-        acc_to_out_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, st>>>(dQacc, (__nv_bfloat16 *)dQ, n,
-                                                                           accumulate);
+        acc_to_out_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, st>>>(dQacc, (__nv_bfloat16 *)dQ, n, acc);
     }
     return launch_status();
 }
@@ -343,11 +382,20 @@ ssa_status_t ssa_block_pool(const ssa_dims_t *dims, const void *K, float *Kbar, 
     if (e != SSA_OK) return e;
     if (!K || !Kbar) return SSA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const unsigned g = static_cast<unsigned>(S.BH * S.nb);
-    if (S.dtype == SSA_DT_BF16)
-        pool_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16 *)K, Kbar, S.T, S.d, S.s, S.nb);
-    else
-        pool_kernel<float><<<g, 256, 0, st>>>((const float *)K, Kbar, S.T, S.d, S.s, S.nb);
+    const size_t units = S.BHk * S.nb;  // one warp per (key/value head, block)
+    const unsigned g = static_cast<unsigned>((units + kPoolWarps - 1) / kPoolWarps);
+    const int blk = kPoolWarps * 32;
+    if (S.dtype == SSA_DT_BF16) {
+        if (S.d == 128)
+            pool_kernel<__nv_bfloat16, 128><<<g, blk, 0, st>>>((const __nv_bfloat16 *)K, Kbar, S.T, S.s, S.nb, units);
+        else
+            pool_kernel<__nv_bfloat16, 64><<<g, blk, 0, st>>>((const __nv_bfloat16 *)K, Kbar, S.T, S.s, S.nb, units);
+    } else {
+        if (S.d == 128)
+            pool_kernel<float, 128><<<g, blk, 0, st>>>((const float *)K, Kbar, S.T, S.s, S.nb, units);
+        else
+            pool_kernel<float, 64><<<g, blk, 0, st>>>((const float *)K, Kbar, S.T, S.s, S.nb, units);
+    }
     return launch_status();
 }
 
@@ -366,8 +414,8 @@ ssa_status_t ssa_block_select(const ssa_dims_t *dims, const void *Q, const float
         // scores on the tensor cores
         const size_t smt = SelTcSmem::kTotal + 1024;
         if (!set_smem(select_tc_kernel, smt)) return SSA_ERR_CUDA;
-        select_tc_kernel<<<dim3((S.T + kSelTcRows - 1) / kSelTcRows, S.BH), kSelTcThreads, smt, st>>>(
-            (const __nv_bfloat16 *)Q, Kbar, idx, S.T, S.s, S.k, S.nb);
+        select_tc_kernel<<<dim3((S.T + kSelTcRows - 1) / kSelTcRows, S.BHk), kSelTcThreads, smt, st>>>(
+            (const __nv_bfloat16 *)Q, Kbar, idx, S.T, S.s, S.k, S.nb, S.G);
         return launch_status();
     }
     if (S.dtype == SSA_DT_BF16) {
@@ -389,71 +437,92 @@ ssa_status_t ssa_block_select(const ssa_dims_t *dims, const void *Q, const float
     return launch_status();
 }
 
+ssa_status_t ssa_sparse_index(const ssa_dims_t *dims, const int32_t *idx, void *index, size_t index_bytes_,
+                              ssa_stream_t stream) {
+    Shape S;
+    ssa_status_t e = check_dims(dims, S, true);
+    if (e != SSA_OK) return e;
+    if (!idx) return SSA_ERR_INVALID_ARG;
+    if (!S.tc) return SSA_OK;  // the CUDA-core kernels read idx directly
+    if ((e = check_ws(S, SSA_OP_SPARSE_INDEX, index, index_bytes_)) != SSA_OK) return e;
+    return build_index(S, idx, carve_index(S, index), reinterpret_cast<cudaStream_t>(stream));
+}
+
 ssa_status_t ssa_sparse_attn_fwd(const ssa_dims_t *dims, const void *Q, const void *K, const void *V,
-                                 const int32_t *idx, void *O, float *lse, void *ws, size_t ws_bytes,
-                                 ssa_stream_t stream) {
+                                 const int32_t *idx, const void *index, void *O, void *O_lo, float *lse, void *ws,
+                                 size_t ws_bytes, ssa_stream_t stream) {
     Shape S;
     ssa_status_t e = check_dims(dims, S, true);
     if (e != SSA_OK) return e;
     if (!Q || !K || !V || !idx || !O || !lse) return SSA_ERR_INVALID_ARG;
     if ((e = check_ws(S, SSA_OP_SPARSE_FWD, ws, ws_bytes)) != SSA_OK) return e;
+    if (index && (reinterpret_cast<uintptr_t>(index) & 15u)) return SSA_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (!S.tc) {
         if (S.dtype == SSA_DT_BF16)
-            launch_simt_fwd<__nv_bfloat16>(S, Q, K, V, idx, O, lse, st);
+            launch_simt_fwd<__nv_bfloat16>(S, Q, K, V, idx, O, O_lo, lse, st);
         else
-            launch_simt_fwd<float>(S, Q, K, V, idx, O, lse, st);
+            launch_simt_fwd<float>(S, Q, K, V, idx, O, O_lo, lse, st);
         return launch_status();
     }
-    IndexWs W{};
-    uint8_t *p = carve_index(S, static_cast<uint8_t *>(ws), W);
-    const size_t nlist = S.BH * list_stride(S.T, S.k, S.nb);
-    __nv_bfloat16 *Opart = reinterpret_cast<__nv_bfloat16 *>(p);
-    float *lsepart = reinterpret_cast<float *>(p + nlist * 128 * 2);
-    p += align_up(nlist * (128 * 2 + 4));
-    int32_t *pos = reinterpret_cast<int32_t *>(p);
-    if ((e = build_index(S, idx, W, st, pos)) != SSA_OK) return e;
+    uint8_t *p = static_cast<uint8_t *>(ws);
+    const IndexWs W = carve_index(S, index ? index : p);
+    p += index_bytes(S);
+    if (!index && (e = build_index(S, idx, W, st)) != SSA_OK) return e;
+    const size_t nprow = S.BHk * list_stride(S.T, S.k, S.nb) * S.G;  // partial rows: G per list position
+    __half *Opart = reinterpret_cast<__half *>(p);
+    float *lsepart = reinterpret_cast<float *>(p + nprow * 128 * 2);
+    p += align_up(nprow * (128 * 2 + 4));
+    int32_t *bexp = reinterpret_cast<int32_t *>(p);  // [BHk * nb] exponents, then the "any set" flag
+    if (cudaMemsetAsync(bexp + S.BHk * S.nb, 0, 4, st) != cudaSuccess) return SSA_ERR_CUDA;
     CUtensorMap tmK, tmV, tmO;
-    if (!make_tmap(&tmK, K, S.rows, S.s) || !make_tmap(&tmV, V, S.rows, S.s) || !make_tmap(&tmO, Opart, nlist, 32))
+    // the fp16 partials are stored through a 16-bit tensor map (no conversion happens in a store)
+    if (!make_tmap(&tmK, K, S.krows, S.s) || !make_tmap(&tmV, V, S.krows, S.s) ||
+        !make_tmap(&tmO, Opart, nprow, 32))
         return SSA_ERR_CUDA;
-    const unsigned units = static_cast<unsigned>(S.BH * S.nb);
+    const unsigned units = static_cast<unsigned>(S.BHk * S.nb);
     const float sl2 = S.scale * kLog2e;
     if (S.s == 128) {
         const size_t sm = SparseFwdSmem<128>::kTotal + 1024;
         if (!set_smem(sparse_fwd_kernel<128>, sm)) return SSA_ERR_CUDA;
         sparse_fwd_kernel<128><<<units, kSparseFwdThreads, sm, st>>>(tmK, tmV, tmO, (const __nv_bfloat16 *)Q,
-                                                                      W.entries, W.lstart, W.llen, lsepart,
-                                                                      static_cast<int>(S.BH), S.T, S.k, S.nb, sl2);
+                                                                      W.entries, W.lstart, W.llen, lsepart, bexp,
+                                                                      static_cast<int>(S.BHk), S.T, S.k, S.nb, S.G,
+                                                                      sl2);
     } else {
         const size_t sm = SparseFwdSmem<64>::kTotal + 1024;
         if (!set_smem(sparse_fwd_kernel<64>, sm)) return SSA_ERR_CUDA;
         sparse_fwd_kernel<64><<<units, kSparseFwdThreads, sm, st>>>(tmK, tmV, tmO, (const __nv_bfloat16 *)Q,
-                                                                     W.entries, W.lstart, W.llen, lsepart,
-                                                                     static_cast<int>(S.BH), S.T, S.k, S.nb, sl2);
+                                                                     W.entries, W.lstart, W.llen, lsepart, bexp,
+                                                                     static_cast<int>(S.BHk), S.T, S.k, S.nb, S.G,
+                                                                     sl2);
     }
-    sparse_merge_kernel<__nv_bfloat16><<<static_cast<unsigned>((S.rows + 7) / 8), 256, 0, st>>>(
-        pos, Opart, lsepart, (__nv_bfloat16 *)O, lse, S.rows, S.T, S.k, S.nb);
+    sparse_merge_kernel<<<static_cast<unsigned>((S.rows + 7) / 8), 256, 0, st>>>(
+        W.pos, idx, bexp, Opart, lsepart, (__nv_bfloat16 *)O, (__nv_bfloat16 *)O_lo, lse, S.rows, S.T, S.k, S.nb,
+        S.G);
     return launch_status();
 }
 
 ssa_status_t ssa_sparse_attn_bwd(const ssa_dims_t *dims, const void *Q, const void *K, const void *V,
-                                 const void *O, const float *lse, const void *dO, const int32_t *idx, void *dQ,
-                                 void *dK, void *dV, int accumulate, void *ws, size_t ws_bytes,
-                                 ssa_stream_t stream) {
+                                 const void *O, const void *O_lo, const float *lse, const void *dO,
+                                 const int32_t *idx, const void *index, void *dQ, void *dK, void *dV, int accumulate,
+                                 void *ws, size_t ws_bytes, ssa_stream_t stream) {
     Shape S;
     ssa_status_t e = check_dims(dims, S, true);
     if (e != SSA_OK) return e;
     if (!Q || !K || !V || !O || !lse || !dO || !idx || !dQ || !dK || !dV) return SSA_ERR_INVALID_ARG;
+    if ((e = check_grads(accumulate, dQ, dK, dV)) != SSA_OK) return e;
     if ((e = check_ws(S, SSA_OP_SPARSE_BWD, ws, ws_bytes)) != SSA_OK) return e;
+    if (index && (reinterpret_cast<uintptr_t>(index) & 15u)) return SSA_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (S.tc) return tc_bwd(S, Q, K, V, O, lse, dO, idx, dQ, dK, dV, accumulate, ws, st);
+    if (S.tc) return tc_bwd(S, Q, K, V, O, O_lo, lse, dO, idx, index, dQ, dK, dV, accumulate, ws, st);
     if (S.dtype == SSA_DT_BF16)
-        return simt_bwd<__nv_bfloat16>(S, Q, K, V, O, lse, dO, idx, dQ, dK, dV, accumulate, ws, st);
-    return simt_bwd<float>(S, Q, K, V, O, lse, dO, idx, dQ, dK, dV, accumulate, ws, st);
+        return simt_bwd<__nv_bfloat16>(S, Q, K, V, O, O_lo, lse, dO, idx, dQ, dK, dV, accumulate, ws, st);
+    return simt_bwd<float>(S, Q, K, V, O, O_lo, lse, dO, idx, dQ, dK, dV, accumulate, ws, st);
 }
 
 ssa_status_t ssa_full_attn_fwd(const ssa_dims_t *dims, const void *Q, const void *K, const void *V, void *O,
-                               float *lse, void *ws, size_t ws_bytes, ssa_stream_t stream) {
+                               void *O_lo, float *lse, void *ws, size_t ws_bytes, ssa_stream_t stream) {
     Shape S;
     ssa_status_t e = check_dims(dims, S, false);
     if (e != SSA_OK) return e;
@@ -463,44 +532,46 @@ ssa_status_t ssa_full_attn_fwd(const ssa_dims_t *dims, const void *Q, const void
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (!S.tc) {
         if (S.dtype == SSA_DT_BF16)
-            launch_simt_fwd<__nv_bfloat16>(S, Q, K, V, nullptr, O, lse, st);
+            launch_simt_fwd<__nv_bfloat16>(S, Q, K, V, nullptr, O, O_lo, lse, st);
         else
-            launch_simt_fwd<float>(S, Q, K, V, nullptr, O, lse, st);
+            launch_simt_fwd<float>(S, Q, K, V, nullptr, O, O_lo, lse, st);
         return launch_status();
     }
     CUtensorMap tmQ, tmK, tmV;
-    if (!make_tmap(&tmQ, Q, S.rows, 128) || !make_tmap(&tmK, K, S.rows, 128) || !make_tmap(&tmV, V, S.rows, 128))
+    if (!make_tmap(&tmQ, Q, S.rows, 128) || !make_tmap(&tmK, K, S.krows, 128) || !make_tmap(&tmV, V, S.krows, 128))
         return SSA_ERR_CUDA;
     const size_t sm = FullFwdSmem::kTotal + 1024;
     if (!set_smem(full_fwd_kernel, sm)) return SSA_ERR_CUDA;
     const unsigned grid = static_cast<unsigned>(S.BH * ((S.T + 255) / 256));
-    full_fwd_kernel<<<grid, kFullFwdThreads, sm, st>>>(tmQ, tmK, tmV, (__nv_bfloat16 *)O, lse,
-                                                      static_cast<int>(S.BH), S.T, S.scale * kLog2e);
+    full_fwd_kernel<<<grid, kFullFwdThreads, sm, st>>>(tmQ, tmK, tmV, (__nv_bfloat16 *)O, (__nv_bfloat16 *)O_lo, lse,
+                                                      static_cast<int>(S.BH), S.T, S.G, S.scale * kLog2e);
     return launch_status();
 }
 
 ssa_status_t ssa_full_attn_bwd(const ssa_dims_t *dims, const void *Q, const void *K, const void *V,
-                               const void *O, const float *lse, const void *dO, void *dQ, void *dK, void *dV,
-                               int accumulate, void *ws, size_t ws_bytes, ssa_stream_t stream) {
+                               const void *O, const void *O_lo, const float *lse, const void *dO, void *dQ, void *dK,
+                               void *dV, int accumulate, void *ws, size_t ws_bytes, ssa_stream_t stream) {
     Shape S;
     ssa_status_t e = check_dims(dims, S, false);
     if (e != SSA_OK) return e;
     if (!Q || !K || !V || !O || !lse || !dO || !dQ || !dK || !dV) return SSA_ERR_INVALID_ARG;
+    if ((e = check_grads(accumulate, dQ, dK, dV)) != SSA_OK) return e;
     if ((e = check_ws(S, SSA_OP_FULL_BWD, ws, ws_bytes)) != SSA_OK) return e;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (S.tc) return tc_bwd(S, Q, K, V, O, lse, dO, nullptr, dQ, dK, dV, accumulate, ws, st);
+    if (S.tc) return tc_bwd(S, Q, K, V, O, O_lo, lse, dO, nullptr, nullptr, dQ, dK, dV, accumulate, ws, st);
     if (S.dtype == SSA_DT_BF16)
-        return simt_bwd<__nv_bfloat16>(S, Q, K, V, O, lse, dO, nullptr, dQ, dK, dV, accumulate, ws, st);
-    return simt_bwd<float>(S, Q, K, V, O, lse, dO, nullptr, dQ, dK, dV, accumulate, ws, st);
+        return simt_bwd<__nv_bfloat16>(S, Q, K, V, O, O_lo, lse, dO, nullptr, dQ, dK, dV, accumulate, ws, st);
+    return simt_bwd<float>(S, Q, K, V, O, O_lo, lse, dO, nullptr, dQ, dK, dV, accumulate, ws, st);
 }
 
-ssa_status_t ssa_align_loss_fwd(const ssa_dims_t *dims, const void *Of, const void *Os, float beta,
+ssa_status_t ssa_align_loss_fwd(const ssa_dims_t *dims, const void *Of, const void *Os, int kind, float beta,
                                 float w_sparsity, float w_commit, float *loss_dev, void *ws, size_t ws_bytes,
                                 ssa_stream_t stream) {
     Shape S;
     ssa_status_t e = check_dims(dims, S, false);
     if (e != SSA_OK) return e;
     if (!Of || !Os || !loss_dev) return SSA_ERR_INVALID_ARG;
+    if (kind != SSA_ALIGN_SMOOTH_L1 && kind != SSA_ALIGN_L2) return SSA_ERR_INVALID_ARG;
     if (!(beta > 0.f) || !std::isfinite(beta) || !std::isfinite(w_sparsity) || !std::isfinite(w_commit))
         return SSA_ERR_INVALID_ARG;
     if ((e = check_ws(S, SSA_OP_ALIGN_FWD, ws, ws_bytes)) != SSA_OK) return e;
@@ -509,22 +580,23 @@ ssa_status_t ssa_align_loss_fwd(const ssa_dims_t *dims, const void *Of, const vo
     const size_t n = S.rows * S.d;
     if (S.dtype == SSA_DT_BF16)
         align_fwd_partial_kernel<__nv_bfloat16><<<kAlignBlocks, 256, 0, st>>>(
-            (const __nv_bfloat16 *)Of, (const __nv_bfloat16 *)Os, partial, n, beta);
+            (const __nv_bfloat16 *)Of, (const __nv_bfloat16 *)Os, partial, n, kind, beta);
     else
         align_fwd_partial_kernel<float><<<kAlignBlocks, 256, 0, st>>>((const float *)Of, (const float *)Os, partial,
-                                                                      n, beta);
+                                                                      n, kind, beta);
     align_fwd_final_kernel<<<1, 32, 0, st>>>(partial, kAlignBlocks, loss_dev,
                                              (static_cast<double>(w_sparsity) + w_commit) / static_cast<double>(n));
     return launch_status();
 }
 
-ssa_status_t ssa_align_loss_bwd(const ssa_dims_t *dims, const void *Of, const void *Os, float beta,
+ssa_status_t ssa_align_loss_bwd(const ssa_dims_t *dims, const void *Of, const void *Os, int kind, float beta,
                                 float w_sparsity, float w_commit, const float *dloss_dev, void *dOf, void *dOs,
                                 int accumulate, ssa_stream_t stream) {
     Shape S;
     ssa_status_t e = check_dims(dims, S, false);
     if (e != SSA_OK) return e;
     if (!Of || !Os || !dloss_dev || !dOf || !dOs) return SSA_ERR_INVALID_ARG;
+    if (kind != SSA_ALIGN_SMOOTH_L1 && kind != SSA_ALIGN_L2) return SSA_ERR_INVALID_ARG;
     if (!(beta > 0.f) || !std::isfinite(beta) || !std::isfinite(w_sparsity) || !std::isfinite(w_commit))
         return SSA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -532,11 +604,11 @@ ssa_status_t ssa_align_loss_bwd(const ssa_dims_t *dims, const void *Of, const vo
     if (S.dtype == SSA_DT_BF16)
         align_bwd_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, st>>>(
             (const __nv_bfloat16 *)Of, (const __nv_bfloat16 *)Os, dloss_dev, (__nv_bfloat16 *)dOf,
-            (__nv_bfloat16 *)dOs, n, beta, w_sparsity, w_commit, accumulate);
+            (__nv_bfloat16 *)dOs, n, kind, beta, w_sparsity, w_commit, accumulate);
     else
         align_bwd_kernel<float><<<grid_for(n, 256), 256, 0, st>>>((const float *)Of, (const float *)Os, dloss_dev,
-                                                                  (float *)dOf, (float *)dOs, n, beta, w_sparsity,
-                                                                  w_commit, accumulate);
+                                                                  (float *)dOf, (float *)dOs, n, kind, beta,
+                                                                  w_sparsity, w_commit, accumulate);
     return launch_status();
 }
 
@@ -556,25 +628,18 @@ ssa_status_t ssa_dropped_mass(const ssa_dims_t *dims, const float *lse_sparse, c
 // ---------------------------------------------------------------------------
 // Allocation-free full attention backward: scratch in a static device array.
 // In host code the array's name is only a stand-in; its device address comes
-// from cudaGetSymbolAddress, looked up once per device with that device current.
+// from cudaGetSymbolAddress, looked up with the caller's device current.
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) unsigned char g_noalloc_scratch[SSA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 64;
-void *g_noalloc_ptr[kMaxDevices];
-std::mutex g_noalloc_mutex;
-
+// Device address of the scratch array in the current device's context.  Looked up on
+// every call (the lookup allocates nothing): an address cached across calls would be
+// stale after the context is torn down and the module loaded again.
 ssa_status_t noalloc_scratch(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SSA_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SSA_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
-    }
-    *out = g_noalloc_ptr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SSA_ERR_CUDA;
+    *out = p;
     return SSA_OK;
 }
 }  // namespace
@@ -582,8 +647,8 @@ ssa_status_t noalloc_scratch(void **out) {
 extern "C" {
 
 ssa_status_t ssa_full_attn_bwd_noalloc(const ssa_dims_t *dims, const void *Q, const void *K, const void *V,
-                                       const void *O, const float *lse, const void *dO, void *dQ, void *dK,
-                                       void *dV, int accumulate, ssa_stream_t stream) {
+                                       const void *O, const void *O_lo, const float *lse, const void *dO, void *dQ,
+                                       void *dK, void *dV, int accumulate, ssa_stream_t stream) {
     Shape S;
     ssa_status_t e = check_dims(dims, S, false);
     if (e != SSA_OK) return e;
@@ -592,8 +657,61 @@ ssa_status_t ssa_full_attn_bwd_noalloc(const ssa_dims_t *dims, const void *Q, co
     if (need > SSA_NOALLOC_SCRATCH_BYTES) return SSA_ERR_WORKSPACE;
     void *ws = nullptr;
     if ((e = noalloc_scratch(&ws)) != SSA_OK) return e;
-    return ssa_full_attn_bwd(dims, Q, K, V, O, lse, dO, dQ, dK, dV, accumulate, ws, SSA_NOALLOC_SCRATCH_BYTES,
+    return ssa_full_attn_bwd(dims, Q, K, V, O, O_lo, lse, dO, dQ, dK, dV, accumulate, ws, SSA_NOALLOC_SCRATCH_BYTES,
                              stream);
+}
+
+ssa_status_t ssa_sparse_decode(const ssa_dims_t *dims, const int32_t *cache_len, const void *q, const void *Kcache,
+                               const void *Vcache, float *Kbar_cache, int32_t *idx, void *o, float *lse, void *ws,
+                               size_t ws_bytes, ssa_stream_t stream) {
+    Shape S;
+    ssa_status_t e = check_dims(dims, S, true);
+    if (e != SSA_OK) return e;
+    if (!cache_len || !q || !Kcache || !Vcache || !Kbar_cache || !idx || !o || !lse) return SSA_ERR_INVALID_ARG;
+    if (S.dtype != SSA_DT_BF16 || S.d != 128 || S.nb > kDecMaxBlocks || S.G > kDecMaxGroup) return SSA_ERR_UNSUPPORTED;
+    if ((e = check_ws(S, SSA_OP_DECODE, ws, ws_bytes)) != SSA_OK) return e;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    float *opart = static_cast<float *>(ws);
+    float *lsepart = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + align_up(S.BH * S.k * S.d * 4));
+    const unsigned bhk = static_cast<unsigned>(S.BHk);
+    const size_t sm = (128 + (S.nb > 256 ? S.nb : 256)) * sizeof(float);
+    decode_select_kernel<<<bhk, kDecThreads, sm, st>>>(cache_len, (const __nv_bfloat16 *)q,
+                                                       (const __nv_bfloat16 *)Kcache, Kbar_cache, idx, S.Hk, S.G, S.T,
+                                                       S.s, S.k, S.nb);
+    decode_attend_kernel<<<dim3(bhk, S.k), kDecThreads, 0, st>>>(cache_len, (const __nv_bfloat16 *)q,
+                                                                (const __nv_bfloat16 *)Kcache,
+                                                                (const __nv_bfloat16 *)Vcache, idx, opart, lsepart,
+                                                                S.Hk, S.G, S.T, S.s, S.k, S.scale);
+    const unsigned rows = static_cast<unsigned>(S.BH);
+    decode_combine_kernel<<<(rows + kDecThreads / 32 - 1) / (kDecThreads / 32), kDecThreads, 0, st>>>(
+        opart, lsepart, (__nv_bfloat16 *)o, lse, static_cast<int>(rows), S.k);
+    return launch_status();
+}
+
+ssa_status_t ssa_rope(const ssa_dims_t *dims, void *X, int heads, int pos0, float base, float factor, int transpose,
+                      ssa_stream_t stream) {
+    Shape S;
+    ssa_status_t e = check_dims(dims, S, false);
+    if (e != SSA_OK) return e;
+    if (!X || heads < 1 || pos0 < 0 || !(base > 1.f) || !std::isfinite(base) || !(factor > 0.f) ||
+        !std::isfinite(factor))
+        return SSA_ERR_INVALID_ARG;
+    if (static_cast<size_t>(S.B) * heads * S.T > 0x7FFFFFFFull) return SSA_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid((S.T + kRopeRows - 1) / kRopeRows, S.B);
+    const double l2b = std::log2(static_cast<double>(base)), inv = 1.0 / static_cast<double>(factor);
+    if (S.dtype == SSA_DT_BF16)
+        rope_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((__nv_bfloat16 *)X, heads, S.T, S.d, pos0, l2b, inv,
+                                                         transpose ? 1 : 0);
+    else
+        rope_kernel<float><<<grid, 256, 0, st>>>((float *)X, heads, S.T, S.d, pos0, l2b, inv, transpose ? 1 : 0);
+    return launch_status();
+}
+
+ssa_status_t ssa_wait_probe(uint64_t limit_ns, ssa_stream_t stream) {
+    if (limit_ns < 1000u || limit_ns > 1000000000u) return SSA_ERR_INVALID_ARG;
+    wait_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
+    return launch_status();
 }
 
 ssa_status_t ssa_get_device_error(ssa_stream_t stream) {
@@ -604,7 +722,7 @@ ssa_status_t ssa_get_device_error(ssa_stream_t stream) {
     if (w == 0) return SSA_OK;
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return SSA_ERR_CUDA;
-    return SSA_ERR_TIMEOUT;
+    return (w >> 24) == ERR_BAD_INPUT ? SSA_ERR_BAD_INPUT : SSA_ERR_TIMEOUT;
 }
 
 const char *ssa_status_string(ssa_status_t s) {
@@ -615,6 +733,7 @@ const char *ssa_status_string(ssa_status_t s) {
         case SSA_ERR_WORKSPACE: return "SSA_ERR_WORKSPACE";
         case SSA_ERR_CUDA: return "SSA_ERR_CUDA";
         case SSA_ERR_TIMEOUT: return "SSA_ERR_TIMEOUT";
+        case SSA_ERR_BAD_INPUT: return "SSA_ERR_BAD_INPUT";
     }
     return "SSA_ERR_UNKNOWN";
 }

@@ -201,6 +201,19 @@ def generate(wl: Workload, *, T: Optional[int] = None, H: Optional[int] = None, 
     return out
 
 
+def group_kv(g: Dict[str, np.ndarray], Hkv: int) -> Dict[str, np.ndarray]:
+    """Grouped-query inputs from a draw of H heads: the key/value heads are the K, V of heads 0, G, 2G, ...
+    (G = H / Hkv), so every query head keeps the per-element distribution of its workload."""
+    H = g["Q"].shape[1]
+    if Hkv < 1 or H % Hkv:
+        raise ValueError("H must be a multiple of Hkv")
+    G = H // Hkv
+    out = dict(g)
+    for key in ("K", "V"):
+        out[key] = np.ascontiguousarray(g[key][:, ::G])
+    return out
+
+
 def random_tensor(shape, dtype: str, seed: int, std: float = 1.0) -> np.ndarray:
     """A plain N(0, std^2) tensor in the requested encoding (for edge-case tests)."""
     rng = np.random.default_rng(seed)

@@ -19,6 +19,7 @@ summary of v4):
   align_fwd/bwd section 5  bidirectional SmoothL1 output alignment; section 7.5
                            the adjusted L2 variant (kind="l2")
   dropped_mass  section 4.2 / Appendix B  delta = 1 - exp(lse_s - lse_f)
+  rope          section 6 / Appendix K  rotary positions with a frequency scaling factor
 
 Parity pins: see tests/test_oracle_pins.py.  Every function there is pinned
 (brute force, library special cases, closed forms, invariants, finite
@@ -64,6 +65,7 @@ def _load():
     lib.ora_attn_fwd.argtypes = [i64, i64, i64, i64, i64, i64, dbl, p, p, p, p, i64, p, p, p]
     lib.ora_attn_bwd.argtypes = [i64, i64, i64, i64, i64, i64, dbl, p, p, p, p, p, i64, p, i64, p, p, p, p,
                                  ctypes.c_int]
+    lib.ora_rope.argtypes = [i64, i64, i64, p, i64, dbl, dbl, ctypes.c_int, p]
     lib.ora_align_fwd.argtypes = [i64, p, p, dbl, dbl, dbl, ctypes.c_int]
     lib.ora_align_fwd.restype = dbl
     lib.ora_align_bwd.argtypes = [i64, p, p, dbl, dbl, dbl, dbl, p, p, ctypes.c_int]
@@ -181,6 +183,16 @@ def attn_bwd(Q, K, V, dO, s: int, scale: float, idx: Optional[np.ndarray] = None
                          nq, _ptr(qrows), nk, _ptr(krows), _ptr(dQ), _ptr(dK), _ptr(dV),
                          1 if stored_o == "bf16" else 0)
     return dQ, dK, dV
+
+
+def rope(X: np.ndarray, pos0: int = 0, base: float = 10000.0, factor: float = 1.0, inverse: bool = False):
+    """Rotary position embedding of X [heads, T, d] (rotate-half pairs, angle (pos0+t) base^(-2i/d) / factor)."""
+    X = _f64(X)
+    heads, T, d = X.shape
+    out = np.empty_like(X)
+    _load().ora_rope(heads * T, T, d, _ptr(X), int(pos0), float(base), float(factor), 1 if inverse else 0,
+                     _ptr(out))
+    return out
 
 
 ALIGN_KINDS = {"smooth_l1": 0, "l2": 1}

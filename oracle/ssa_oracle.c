@@ -379,6 +379,34 @@ void ora_attn_bwd(i64 BH, i64 G, i64 T, i64 d, i64 s, i64 k, double scale, const
 }
 
 /* ---------------------------------------------------------------------------
+ * Rotary position embedding -- page section 6 and Appendix K: the model's
+ * queries and keys carry rotary positions, and continued training at 32k uses
+ * "RoPE scaling factor 4", which stretches the rotation periods.  The pages
+ * print neither the rotation nor the base.  Reading: the rotate-half form, pairs
+ * (x_i, x_{i+d/2}) for i < d/2 turned by the angle
+ *   a(t, i) = (pos0 + t) * base^(-2i/d) / factor
+ * (factor 4 divides every frequency by 4, i.e. positions are interpolated);
+ * inverse != 0 turns by -a (the transpose, which carries gradients back).
+ * X is [rows, d] with rows = heads * T (row r is position r % T); out may be X.
+ * ------------------------------------------------------------------------- */
+void ora_rope(i64 rows, i64 T, i64 d, const double *X, i64 pos0, double base, double factor, int inverse,
+              double *out) {
+    i64 h = d / 2;
+#pragma omp parallel for schedule(static)
+    for (i64 r = 0; r < rows; ++r) {
+        double t = (double)(pos0 + r % T);
+        for (i64 i = 0; i < h; ++i) {
+            double a = t * pow(base, -2.0 * (double)i / (double)d) / factor;
+            if (inverse) a = -a;
+            double c = cos(a), sn = sin(a);
+            double x0 = X[r * d + i], x1 = X[r * d + i + h];
+            out[r * d + i] = x0 * c - x1 * sn;
+            out[r * d + i + h] = x0 * sn + x1 * c;
+        }
+    }
+}
+
+/* ---------------------------------------------------------------------------
  * Bidirectional alignment -- page section 5: full-attention outputs are pulled
  * toward the sparse ones (sparsity term, stop-gradient on o_s), a commitment
  * term keeps the sparse outputs near the full ones (stop-gradient on o_f), both

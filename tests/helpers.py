@@ -1,5 +1,12 @@
-"""Shared helpers for the parity tests (tolerances, conversions, oracle runs)."""
+"""Shared helpers for the parity tests (tolerances, conversions, oracle runs).
+
+Every comparison made through check_close is also appended, as one JSON line,
+to the file named by the environment variable SSA_PARITY_LOG when it is set
+(the errors of a run, for the record, whether or not they pass)."""
 from __future__ import annotations
+
+import json
+import os
 
 import numpy as np
 
@@ -38,9 +45,23 @@ def check_close(name: str, got: np.ndarray, ref: np.ndarray, bf16: bool) -> dict
     allow = MAX_ABS + (bf16_half_ulp(ref) if bf16 else 0.0)
     worst = float((diff - allow).max()) if diff.size else 0.0
     rel = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
+    res = {"max_abs": float(diff.max()) if diff.size else 0.0, "rel_l2": rel}
+    log_result(name, res)
     assert worst <= 0, "%s: max-abs excess %.3g (max diff %.3g)" % (name, worst, diff.max())
     assert rel <= REL_L2, "%s: rel-L2 %.3g > %.3g" % (name, rel, REL_L2)
-    return {"max_abs": float(diff.max()), "rel_l2": rel}
+    return res
+
+
+def rel_l2(got: np.ndarray, ref: np.ndarray) -> float:
+    got, ref = np.asarray(got, dtype=np.float64), np.asarray(ref, dtype=np.float64)
+    return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30))
+
+
+def log_result(name: str, res: dict) -> None:
+    path = os.environ.get("SSA_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(dict(name=name, **res)) + "\n")
 
 
 def selection_report(got: np.ndarray, ref: np.ndarray, r1: np.ndarray, r2: np.ndarray) -> dict:
@@ -51,6 +72,36 @@ def selection_report(got: np.ndarray, ref: np.ndarray, r1: np.ndarray, r2: np.nd
     exempt = np.where(np.isnan(r1) | np.isnan(r2), False, exempt)
     return {"rows": int(differ.size), "differ": int(differ.sum()), "exempt_rows": int(exempt.sum()),
             "mismatch": int((differ & ~exempt).sum()), "exempt_and_differ": int((differ & exempt).sum())}
+
+
+def check_gpu_selection(ora, name: str, got: np.ndarray, Q: np.ndarray, Kbar: np.ndarray, s: int, k: int) -> dict:
+    """Selection parity of got [BH, T, k] against the oracle on Q [BH, T, d], Kbar [BH, nb, d] (fp64):
+
+    * every row is structurally valid (ascending, distinct, holds b(t), -1 padding at the end);
+    * rows are bit-exact, except rows whose (k-1)-th and k-th oracle candidate scores lie within
+      TIE_REL of each other;
+    * on such an exempt row that differs, the chosen set is still a valid top-(k-1): the lowest
+      oracle score among the chosen blocks is at least the highest among the blocks left out,
+      less the same tolerance."""
+    assert ora.check_selection(got, s), name + ": structurally invalid selection rows"
+    ref, r1, r2 = ora.block_select(Q, Kbar, s, k)
+    rep = selection_report(got, ref, r1, r2)
+    assert rep["mismatch"] == 0, (name, rep)
+    differ = np.argwhere(np.any(got != ref, axis=-1))
+    if differ.size:
+        sc = ora.block_scores(Q, Kbar, s, differ[:, 0], differ[:, 1])
+        for i, (b, t) in enumerate(differ):
+            bt = t // s
+            chosen = [j for j in got[b, t] if 0 <= j < bt]
+            left = [j for j in range(bt) if j not in chosen]
+            assert len(chosen) == min(k - 1, bt), (name, b, t, chosen)
+            if left:
+                tol = TIE_REL * max(abs(r1[b, t]), abs(r2[b, t]))
+                lo = min(sc[i, j] for j in chosen)
+                hi = max(sc[i, j] for j in left)
+                assert lo >= hi - tol, (name, int(b), int(t), lo, hi, tol)
+    log_result(name + ".selection", rep)
+    return rep
 
 
 def workload_arrays(wl, **over):

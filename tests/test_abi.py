@@ -44,21 +44,30 @@ def test_no_torch_in_boundary():
 
 
 def test_status_strings(lib):
-    for code in range(6):
+    for code in range(7):
         assert L.status_string(code).startswith("SSA_")
     assert L.status_string(99) == "SSA_ERR_UNKNOWN"
 
 
 def test_workspace_sizes(lib):
     d = L.make_dims(1, 32, 32768, 128, 128, 16)
-    # sparse forward: index (counts, starts, lengths, entries) + bf16 partials + partial lse
+    # inverse index: entries and the list position of every (query, slot)
+    ix = L.ssa_workspace_size(d, L.SSA_OP_SPARSE_INDEX)
+    assert ix >= 32 * 32768 * 16 * (4 + 4)
+    # sparse forward: index + fp16 partials + partial lse by list position
     sf = L.ssa_workspace_size(d, L.SSA_OP_SPARSE_FWD)
-    assert sf >= 32 * 32768 * 16 * (128 * 2 + 4 + 4)
+    assert sf >= ix + 32 * 32768 * 16 * (128 * 2 + 4)
     fb = L.ssa_workspace_size(d, L.SSA_OP_FULL_BWD)
     assert fb >= 32 * 32768 * (128 * 4 + 4)
-    # sparse backward: index + one bf16 dQ partial per (query, slot) + the slot positions
+    # sparse backward: D + index + the fp32 dQ accumulator
     sb = L.ssa_workspace_size(d, L.SSA_OP_SPARSE_BWD)
-    assert sb >= 32 * 32768 * 16 * (128 * 2 + 4 + 4) and sb > fb
+    assert sb >= fb + ix
+    # shapes on the CUDA-core path read idx directly: no index
+    assert L.ssa_workspace_size(L.make_dims(1, 2, 1024, 64, 64, 4, dtype="fp32"), L.SSA_OP_SPARSE_INDEX) == 0
+    # grouped-query heads: the index is per key/value head, the partials per query head
+    g = L.make_dims(1, 32, 32768, 128, 128, 16, Hkv=8)
+    assert L.ssa_workspace_size(g, L.SSA_OP_SPARSE_INDEX) * 4 == pytest.approx(ix, rel=0.01)
+    assert L.ssa_workspace_size(g, L.SSA_OP_SPARSE_FWD) == pytest.approx(sf - 3 * ix / 4, rel=0.01)
     assert L.ssa_workspace_size(d, L.SSA_OP_FULL_FWD) == 0
     assert L.ssa_workspace_size(d, L.SSA_OP_ALIGN_FWD) > 0
     # invalid dims -> 0
@@ -89,14 +98,23 @@ BAD_DIMS = [
 ]
 
 
+BAD_DIMS += [
+    (dict(H=6, Hkv=4), L.SSA_ERR_INVALID_ARG),                       # H not a multiple of Hkv
+    (dict(H=6, Hkv=-1), L.SSA_ERR_INVALID_ARG),
+    (dict(H=3, Hkv=1), L.SSA_ERR_UNSUPPORTED),                       # group of 3 does not divide a 128-row tile
+]
+
+
 @pytest.mark.parametrize("over,code", BAD_DIMS)
 def test_dims_validation(lib, over, code):
-    base = dict(B=1, H=2, T=1024, d=128, s=64, k=4, dtype=0, scale=0.088)
+    base = dict(B=1, H=2, T=1024, d=128, s=64, k=4, dtype=0, scale=0.088, Hkv=0)
     base.update(over)
-    d = L.Dims(base["B"], base["H"], base["T"], base["d"], base["s"], base["k"], base["dtype"], base["scale"])
+    d = L.Dims(base["B"], base["H"], base["T"], base["d"], base["s"], base["k"], base["dtype"], base["scale"],
+               base["Hkv"])
     p = ctypes.c_void_p(16)  # never dereferenced: validation fails first
-    st = _call("ssa_sparse_attn_fwd", d, p, p, p, p, p, p, p, 1 << 40, None)
+    st = _call("ssa_sparse_attn_fwd", d, p, p, p, p, None, p, p, p, p, 1 << 40, None)
     assert st == code
+    assert _call("ssa_sparse_index", d, p, p, 1 << 40, None) == code
 
 
 def test_null_pointers_and_workspace(lib):
@@ -109,17 +127,29 @@ def test_null_pointers_and_workspace(lib):
     assert _call("ssa_block_select", d, p, p, p, 3, None) == L.SSA_ERR_UNSUPPORTED
     big = L.make_dims(1, 1, 2048 * 64, 128, 64, 4)     # nb = 2048 > 1024
     assert _call("ssa_block_select", big, p, p, p, 1, None) == L.SSA_ERR_UNSUPPORTED
-    # short / missing / misaligned workspace
+    # short / missing / misaligned workspace or index
     need = L.ssa_workspace_size(d, L.SSA_OP_SPARSE_FWD)
-    assert _call("ssa_sparse_attn_fwd", d, p, p, p, p, p, p, None, need, None) == L.SSA_ERR_WORKSPACE
-    assert _call("ssa_sparse_attn_fwd", d, p, p, p, p, p, p, p, need - 1, None) == L.SSA_ERR_WORKSPACE
-    assert _call("ssa_sparse_attn_fwd", d, p, p, p, p, p, p, ctypes.c_void_p(24), need, None) == L.SSA_ERR_WORKSPACE
+    assert _call("ssa_sparse_attn_fwd", d, p, p, p, p, None, p, None, p, None, need, None) == L.SSA_ERR_WORKSPACE
+    assert _call("ssa_sparse_attn_fwd", d, p, p, p, p, None, p, None, p, p, need - 1, None) == L.SSA_ERR_WORKSPACE
+    assert _call("ssa_sparse_attn_fwd", d, p, p, p, p, None, p, None, p, ctypes.c_void_p(24), need,
+                 None) == L.SSA_ERR_WORKSPACE
+    assert _call("ssa_sparse_attn_fwd", d, p, p, p, p, ctypes.c_void_p(24), p, None, p, p, need,
+                 None) == L.SSA_ERR_WORKSPACE
+    need_i = L.ssa_workspace_size(d, L.SSA_OP_SPARSE_INDEX)
+    assert _call("ssa_sparse_index", d, p, p, need_i - 1, None) == L.SSA_ERR_WORKSPACE
+    assert _call("ssa_sparse_index", d, None, p, need_i, None) == L.SSA_ERR_INVALID_ARG
+    need_s = L.ssa_workspace_size(d, L.SSA_OP_SPARSE_BWD)
+    assert _call("ssa_sparse_attn_bwd", d, p, p, p, p, None, p, p, p, None, p, p, p, 0, p, need_s - 16,
+                 None) == L.SSA_ERR_WORKSPACE
     need_b = L.ssa_workspace_size(d, L.SSA_OP_FULL_BWD)
-    assert _call("ssa_full_attn_bwd", d, p, p, p, p, p, p, p, p, p, 0, p, need_b - 16, None) == L.SSA_ERR_WORKSPACE
-    assert _call("ssa_align_loss_fwd", d, p, p, ctypes.c_float(0.0), ctypes.c_float(1), ctypes.c_float(1), p, p,
+    assert _call("ssa_full_attn_bwd", d, p, p, p, p, None, p, p, p, p, p, 0, p, need_b - 16,
+                 None) == L.SSA_ERR_WORKSPACE
+    assert _call("ssa_align_loss_fwd", d, p, p, 0, ctypes.c_float(0.0), ctypes.c_float(1), ctypes.c_float(1), p, p,
                  1 << 20, None) == L.SSA_ERR_INVALID_ARG
-    assert _call("ssa_align_loss_bwd", d, p, p, ctypes.c_float(1.0), ctypes.c_float(1), ctypes.c_float(1), None, p,
-                 p, 0, None) == L.SSA_ERR_INVALID_ARG
+    assert _call("ssa_align_loss_fwd", d, p, p, 2, ctypes.c_float(1.0), ctypes.c_float(1), ctypes.c_float(1), p, p,
+                 1 << 20, None) == L.SSA_ERR_INVALID_ARG          # unknown kind
+    assert _call("ssa_align_loss_bwd", d, p, p, 0, ctypes.c_float(1.0), ctypes.c_float(1), ctypes.c_float(1), None,
+                 p, p, 0, None) == L.SSA_ERR_INVALID_ARG
     assert _call("ssa_dropped_mass", d, p, None, p, None) == L.SSA_ERR_INVALID_ARG
 
 

@@ -409,6 +409,38 @@ def test_grouped_sparse_attention_matches_dense_mask(ora, G, s, k):
         np.testing.assert_allclose(got, want.numpy(), rtol=0, atol=1e-11)
 
 
+# --------------------------------------------------------------------------- rotary positions
+
+def test_rope_two_dims_closed_form(ora):
+    # d = 2: one pair turned by the position itself (base^0 = 1)
+    X = np.array([[[1.0, 0.0], [0.6, -0.8], [2.0, 3.0]]])
+    out = ora.rope(X, pos0=5)
+    for t in range(3):
+        a = 5.0 + t
+        x0, x1 = X[0, t]
+        np.testing.assert_allclose(out[0, t], [x0 * np.cos(a) - x1 * np.sin(a), x0 * np.sin(a) + x1 * np.cos(a)],
+                                   rtol=0, atol=1e-15)
+
+
+def test_rope_scores_depend_on_relative_position_only(ora):
+    q = _rand((1, 1, 16), 70)
+    k = _rand((1, 1, 16), 71)
+    def score(tq, tk, factor=1.0):
+        return float(ora.rope(q, pos0=tq, factor=factor).ravel() @ ora.rope(k, pos0=tk, factor=factor).ravel())
+    for factor in (1.0, 4.0):
+        assert score(100, 37, factor) == pytest.approx(score(1163, 1100, factor), rel=1e-9, abs=1e-12)
+
+
+def test_rope_inverse_norm_and_scaling(ora):
+    X = _rand((2, 32, 8), 72)
+    Y = ora.rope(X, pos0=3, base=500000.0, factor=4.0)
+    np.testing.assert_allclose(np.linalg.norm(Y, axis=-1), np.linalg.norm(X, axis=-1), rtol=1e-13)
+    np.testing.assert_allclose(ora.rope(Y, pos0=3, base=500000.0, factor=4.0, inverse=True), X, rtol=0, atol=1e-13)
+    # factor 4 at position 4m is the plain rotation at position m
+    Z = ora.rope(X[:, ::4], pos0=0, base=500000.0)
+    np.testing.assert_allclose(ora.rope(X, pos0=0, base=500000.0, factor=4.0)[:, ::4], Z, rtol=0, atol=1e-12)
+
+
 # --------------------------------------------------------------------------- alignment loss
 
 @pytest.mark.parametrize("beta,ws,wc", [(1.0, 1.0, 1.0), (0.5, 0.3, 2.0)])

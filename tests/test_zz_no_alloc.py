@@ -6,7 +6,9 @@ latency-critical path where cudaMalloc (which can synchronise the device) is
 not allowed.  This entry point keeps its scratch in an array inside libssa
 instead of taking a workspace.  The test calls it twice in a row through the C
 ABI and compares each result with the workspace entry point's result, using the
-tolerances of the other parity tests; it also checks the size limit.
+tolerances of the other parity tests, then a third time adding into the second
+call's gradients (the scratch keeps the previous call's contents, so this checks
+that the call clears what must start at zero); it also checks the size limit.
 
 Kept in its own file, collected last, so that a run stopping at the first
 failure has already run every other test.
@@ -34,15 +36,20 @@ def test_noalloc_matches_workspace_entry_point(wlname, over):
     w = g["wl"]
     dims = L.make_dims(w.B, w.H, w.T, w.d, w.s, 1, dtype=w.dtype)
     Q, K, V, dO = (to_device(g[key], w.dtype) for key in ("Q", "K", "V", "dO"))
-    O, lse = ops.attn_fwd(dims, Q, K, V)
-    ref = [to_np(x) for x in ops.attn_bwd(dims, Q, K, V, O, lse, dO)]
+    O, lse, O_lo = ops.attn_fwd(dims, Q, K, V)
+    ref = [to_np(x) for x in ops.attn_bwd(dims, Q, K, V, O, lse, dO, O_lo=O_lo)]
     bf16 = w.dtype == "bf16"
     for call in range(2):
         dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
-        L.ssa_full_attn_bwd_noalloc(dims, Q, K, V, O, lse, dO, dQ, dK, dV, 0)
+        L.ssa_full_attn_bwd_noalloc(dims, Q, K, V, O, lse, dO, dQ, dK, dV, 0, O_lo=O_lo)
         torch.cuda.synchronize()
         for name, got, r in zip(("dQ", "dK", "dV"), (dQ, dK, dV), ref):
             check_close("noalloc call %d %s" % (call, name), to_np(got), r, bf16)
+    # third call: accumulate into the second call's results -> twice the gradients
+    L.ssa_full_attn_bwd_noalloc(dims, Q, K, V, O, lse, dO, dQ, dK, dV, 1, O_lo=O_lo)
+    torch.cuda.synchronize()
+    for name, got, r in zip(("dQ", "dK", "dV"), (dQ, dK, dV), ref):
+        check_close("noalloc accumulate %s" % name, to_np(got), 2 * r, bf16)
     assert L.ssa_get_device_error() == L.SSA_OK
 
 
@@ -53,5 +60,5 @@ def test_noalloc_rejects_problems_beyond_the_scratch():
     dims = L.make_dims(1, 1, T, 128, 128, 1)
     p = torch.empty(16, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(L.SSAError) as e:
-        L.ssa_full_attn_bwd_noalloc(dims, p, p, p, p, p, p, p, p, p, 0)
+        L.ssa_full_attn_bwd_noalloc(dims, p, p, p, p, p, p, p, p, p, 0, O_lo=p)
     assert e.value.status == L.SSA_ERR_WORKSPACE
