@@ -233,6 +233,122 @@ def sweep(args):
         torch.cuda.empty_cache()
 
 
+def union(args):
+    """Union of the selected blocks of a 128-query tile, per workload, from the GPU's own selections: the blocks a
+    query-tile kernel with row masks would have to load, against the causal blocks it covers (full attention) and
+    the blocks any one query attends (k).  One JSON line per workload."""
+    import torch
+    from block_top_sparse_b200 import _lib as L
+    from block_top_sparse_b200 import build, inputs, ops
+    build.build()
+    for name in ("prefill", "train", "long", "sweep"):
+        wl = inputs.WORKLOADS[name]
+        H = min(wl.H, 4)  # heads are independent: four are enough for the distribution
+        g = inputs.generate(wl, H=H)
+        Q = torch.from_numpy(g["Q"].view(np.int16)).view(torch.bfloat16).cuda()
+        K = torch.from_numpy(g["K"].view(np.int16)).view(torch.bfloat16).cuda()
+        for k in wl.k:
+            dims = L.make_dims(wl.B, H, wl.T, wl.d, wl.s, k)
+            idx = ops.block_select(dims, Q, ops.block_pool(dims, K)).cpu().numpy().reshape(wl.B * H, wl.T, k)
+            sizes, causal = [], []
+            for bh in range(wl.B * H):
+                for t0 in range(0, wl.T, 128):
+                    sel = idx[bh, t0:t0 + 128].ravel()
+                    sizes.append(len(np.unique(sel[sel >= 0])))
+                    causal.append((min(t0 + 128, wl.T) - 1) // wl.s + 1)
+            sizes, causal = np.array(sizes), np.array(causal)
+            keep = causal > k  # tiles whose queries have more blocks to choose from than k
+            print(json.dumps({"union": name, "k": k, "s": wl.s, "tile": 128,
+                              "mean_union_blocks": float(sizes.mean()), "p50": float(np.median(sizes)),
+                              "max": int(sizes.max()),
+                              "mean_union_over_causal": float((sizes[keep] / causal[keep]).mean()) if keep.any() else None,
+                              "mean_union_over_k": float((sizes[keep] / k).mean()) if keep.any() else None}),
+                  flush=True)
+        del Q, K
+        torch.cuda.empty_cache()
+
+
+def _time(fn, steps, warmup):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def extras(args):
+    """The rows beside the training path, one JSON line each: grouped-query sparse attention fwd+bwd at 32K
+    (H = 32 query heads on Hkv = 8 key/value heads), sparse decoding over a 32K cache (64 sequences), and the
+    rotary-position pass."""
+    import torch
+    from block_top_sparse_b200 import _lib as L
+    from block_top_sparse_b200 import build, inputs, ops
+    build.build()
+    hbm, _, peak_sust, _ = measured_peaks()
+    wl = inputs.WORKLOADS[WORKLOAD]
+    B, H, T, d, s, k = wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL
+    # ---- grouped-query sparse attention: same FLOPs as 32 heads, 8 key/value heads
+    Hkv = 8
+    g = inputs.group_kv(inputs.generate(wl), Hkv)
+    dev = {key: torch.from_numpy(g[key].view(np.int16)).view(torch.bfloat16).cuda() for key in ("Q", "K", "V", "dO")}
+    dims = L.make_dims(B, H, T, d, s, k, Hkv=Hkv)
+    st = ops.SSAStep(dims, main="sparse", grad_fp32=True)
+    st.forward(dev["Q"], dev["K"], dev["V"])
+    Q, K, V = dev["Q"], dev["K"], dev["V"]
+
+    def sparse_call():
+        L.ssa_sparse_index(dims, st.idx, st.index)
+        L.ssa_sparse_attn_fwd(dims, Q, K, V, st.idx, st.Os, st.lse_s, st.ws[L.SSA_OP_SPARSE_FWD], O_lo=st.Os_lo,
+                              index=st.index)
+        L.ssa_sparse_attn_bwd(dims, Q, K, V, st.Os, st.lse_s, dev["dO"], st.idx, st.dQ, st.dK, st.dV,
+                              L.SSA_BWD_GRAD_FP32, st.ws[L.SSA_OP_SPARSE_BWD], O_lo=st.Os_lo, index=st.index)
+    ms = _time(sparse_call, args.steps, args.warmup)
+    sf, sb, _, _ = flops(B, H, T, d, s, k)
+    print(json.dumps({"extra": "gqa sparse attention fwd+bwd", "B": B, "H": H, "Hkv": Hkv, "T": T, "k": k,
+                      "ms": ms, "tokens_per_s": B * T / (ms / 1e3), "tflops": (sf + sb) / (ms / 1e3) / 1e12,
+                      "frac_of_peak": (sf + sb) / (ms / 1e3) / 1e12 / peak_sust,
+                      "device_error": L.ssa_get_device_error()}), flush=True)
+    del st, dev, Q, K, V
+    torch.cuda.empty_cache()
+    # ---- sparse decoding: 64 sequences, caches of 32768 tokens, new tokens at random lengths
+    Bd, Hd, Hk, Td = 64, 32, 8, 32768
+    ddims = L.make_dims(Bd, Hd, Td, d, s, k, Hkv=Hk)
+    rng = np.random.default_rng(5)
+    lens = torch.from_numpy(rng.integers(Td // 2, Td, size=Bd).astype(np.int32)).cuda()
+    Kc = torch.randn((Bd, Hk, Td, d), device="cuda").mul_(d ** -0.25).to(torch.bfloat16)
+    Vc = torch.randn((Bd, Hk, Td, d), device="cuda").mul_(d ** -0.25).to(torch.bfloat16)
+    q = torch.randn((Bd, Hd, d), device="cuda").mul_(d ** -0.25).to(torch.bfloat16)
+    Kbar = ops.block_pool(ddims, Kc)
+    idx = torch.empty((Bd, Hk, k), dtype=torch.int32, device="cuda")
+    o = torch.empty((Bd, Hd, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((Bd, Hd), dtype=torch.float32, device="cuda")
+    ws = ops._ws(ddims, L.SSA_OP_DECODE, "cuda")
+    ms = _time(lambda: L.ssa_sparse_decode(ddims, lens, q, Kc, Vc, Kbar, idx, o, lse, ws), args.steps, args.warmup)
+    Ls = lens.cpu().numpy().astype(np.int64)
+    # bytes a decode step must read: pooled keys of the complete blocks and the selected blocks' keys and values
+    nbytes = float(sum(Hk * ((L_ // s) * d * 4 + min(k * s, L_ + 1) * d * 2 * 2) for L_ in Ls))
+    print(json.dumps({"extra": "sparse decode", "sequences": Bd, "H": Hd, "Hkv": Hk, "cache": Td, "k": k,
+                      "ms": ms, "tokens_per_s": Bd / (ms / 1e3), "gbs": nbytes / (ms / 1e3) / 1e9,
+                      "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / hbm, "device_error": L.ssa_get_device_error()}),
+          flush=True)
+    del Kc, Vc, Kbar
+    torch.cuda.empty_cache()
+    # ---- rotary positions on Q of the 32K workload (one read and one write)
+    X = torch.randn((B, H, T, d), device="cuda").to(torch.bfloat16)
+    rdims = L.make_dims(B, H, T, d, s, k)
+    ms = _time(lambda: L.ssa_rope(rdims, X, H, 0, 500000.0, 4.0, 0), args.steps, args.warmup)
+    print(json.dumps({"extra": "rope", "B": B, "H": H, "T": T, "ms": ms,
+                      "gbs": 2 * X.numel() * 2 / (ms / 1e3) / 1e9,
+                      "frac_of_hbm": 2 * X.numel() * 2 / (ms / 1e3) / 1e9 / hbm,
+                      "device_error": L.ssa_get_device_error()}), flush=True)
+
+
 def config_block(wl):
     return {"workload": "long-context fwd+bwd, both streams + alignment: B=%d H=%d T=%d d=%d s=%d k=%d, sink block"
                         % (wl.B, wl.H, wl.T, wl.d, wl.s, K_SEL),
@@ -504,6 +620,10 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=16384, help="prefix length of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep", action="store_true", help="the k sweep at T = 131072 (one JSON line per k)")
+    ap.add_argument("--extras", action="store_true",
+                    help="grouped-query sparse attention, sparse decoding and rotary positions (one line each)")
+    ap.add_argument("--union", action="store_true",
+                    help="size of the union of a 128-query tile's selected blocks, per workload (one line each)")
     ap.add_argument("--op", default=None,
                     choices=["pool", "select", "index", "full_fwd", "sparse_fwd", "full_bwd", "sparse_bwd"],
                     help="time one library call instead of the whole step (profiling)")
@@ -514,6 +634,12 @@ def main():
     args = ap.parse_args()
     if args.sweep:
         sweep(args)
+        return
+    if args.union:
+        union(args)
+        return
+    if args.extras:
+        extras(args)
         return
     if args.op:
         single_op(args)

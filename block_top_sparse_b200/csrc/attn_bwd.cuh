@@ -72,7 +72,7 @@ constexpr int kBwdThreads = 640;
 constexpr int kBwdGatherWarps = 6;
 constexpr int kBwdGatherPairs = (64 + kBwdGatherWarps - 1) / kBwdGatherWarps;
 
-template <int NKV>
+template <int NKV, bool GQ>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto tile_row0 = [&](int it) {
         int t;
         size_t qrow;
-        tile_row(R, it, 0, t, qrow);
+        tile_row<GQ>(R, it, 0, t, qrow);
         return static_cast<int>(qrow);
     };
 
@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         const int p = gw + kBwdGatherWarps * q;
                         int t = 0;
                         size_t row = 0;
-                        tn[q] = (p < 64 && tile_row(R, it, 2 * p + (lane >> 4), t, row)) ? static_cast<int>(row) : -1;
+                        tn[q] = (p < 64 && tile_row<GQ>(R, it, 2 * p + (lane >> 4), t, row)) ? static_cast<int>(row) : -1;
                     }
                 };
                 load_rows(0);
@@ -373,7 +373,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             auto row_of = [&](int it) {
                 int t;
                 size_t qrow;
-                return (it < ntiles && tile_row(R, it, r, t, qrow)) ? static_cast<int>(qrow) : -1;
+                return (it < ntiles && tile_row<GQ>(R, it, r, t, qrow)) ? static_cast<int>(qrow) : -1;
             };
             int q_n = row_of(0);
             for (int it = 0; it < ntiles; ++it) {
@@ -412,10 +412,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // the position loaded from the list), so no dependent global load sits between two tiles.
         int t_n1 = 0, t_n2 = 0;
         size_t q_n1 = 0, q_n2 = 0;
-        bool v_n1 = ntiles > 0 && tile_row(R, 0, r, t_n1, q_n1);
+        bool v_n1 = ntiles > 0 && tile_row<GQ>(R, 0, r, t_n1, q_n1);
         float lse_n = v_n1 ? __ldg(a.lse + q_n1) : 0.f;
         float D_n = v_n1 ? __ldg(a.Dvec + q_n1) : 0.f;
-        bool v_n2 = ntiles > 1 && tile_row(R, 1, r, t_n2, q_n2);
+        bool v_n2 = ntiles > 1 && tile_row<GQ>(R, 1, r, t_n2, q_n2);
         for (int it = 0; it < ntiles; ++it) {
             const bool valid = v_n1;
             const int t = t_n1;
@@ -426,7 +426,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             q_n1 = q_n2;
             lse_n = v_n1 ? __ldg(a.lse + q_n1) : 0.f;
             D_n = v_n1 ? __ldg(a.Dvec + q_n1) : 0.f;
-            v_n2 = it + 2 < ntiles && tile_row(R, it + 2, r, t_n2, q_n2);
+            v_n2 = it + 2 < ntiles && tile_row<GQ>(R, it + 2, r, t_n2, q_n2);
             if (!mbar_wait(bar_sdp_full, it & 1, abort_flag, 0x306)) {
                 ok = false;
                 break;

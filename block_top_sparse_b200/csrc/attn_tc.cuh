@@ -52,17 +52,21 @@ __host__ __device__ __forceinline__ int log2_pow2(int g) {
     return s;
 }
 
-// Query position t and query-tensor row of tile row r of tile `it`; false past the end.
+// Query position t and query-tensor row of tile row r of tile `it`; false past the end.  GQ: the
+// kernel was instantiated for grouped heads (G > 1); without it the group arithmetic compiles away.
+template <bool GQ>
 __device__ __forceinline__ bool tile_row(const Rows &R, int it, int r, int &t, size_t &qrow) {
+    const int gs = GQ ? R.gshift : 0;
     if (R.list) {
-        const int li = ((it * kTileQ + r) >> R.gshift);  // it * (128 / G) + r / G
+        const int li = (it * kTileQ + r) >> gs;  // it * (128 / G) + r / G
         if (li >= R.len) return false;
         t = __ldg(R.list + li) >> 8;
-        qrow = R.qrow0 + static_cast<size_t>(r & ((1 << R.gshift) - 1)) * R.T + t;
+        qrow = R.qrow0 + t;
+        if (GQ) qrow += static_cast<size_t>(r & ((1 << gs) - 1)) * R.T;
         return true;
     }
     const int tph = R.tiles_per_head();
-    const int hi = R.gshift ? it / tph : 0;
+    const int hi = GQ ? it / tph : 0;
     t = R.first + (it - hi * tph) * kTileQ + r;
     qrow = R.qrow0 + static_cast<size_t>(hi) * R.T + t;
     return t < R.T;
@@ -438,13 +442,14 @@ constexpr int kSparseFwdGatherWarps = 7;
 constexpr int kGatherPairs = (64 + kSparseFwdGatherWarps - 1) / kSparseFwdGatherWarps;
 
 // Query-tensor rows (-1 past the list) of this lane's rows of tile `it`.
+template <bool GQ>
 __device__ __forceinline__ void gather_rows_load(const Rows &R, int it, int gw, int lane, int (&qrow)[kGatherPairs]) {
 #pragma unroll
     for (int q = 0; q < kGatherPairs; ++q) {
         const int p = gw + kSparseFwdGatherWarps * q;
         int t = 0;
         size_t row = 0;
-        qrow[q] = (p < 64 && tile_row(R, it, 2 * p + (lane >> 4), t, row)) ? static_cast<int>(row) : -1;
+        qrow[q] = (p < 64 && tile_row<GQ>(R, it, 2 * p + (lane >> 4), t, row)) ? static_cast<int>(row) : -1;
     }
 }
 
@@ -463,7 +468,7 @@ __device__ __forceinline__ void gather_rows_issue(uint32_t tile, const __nv_bflo
     }
 }
 
-template <int NKV>
+template <int NKV, bool GQ>
 __global__ void __launch_bounds__(kSparseFwdThreads, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmO, const __nv_bfloat16 *__restrict__ Q,
@@ -533,7 +538,7 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
         // ---------------- gather warps: query rows of tile it into Q[it & 1] ----------------
         const int gw = warp < 12 ? warp - 8 : warp - 9;
         int tn[kGatherPairs];
-        gather_rows_load(R, 0, gw, lane, tn);
+        gather_rows_load<GQ>(R, 0, gw, lane, tn);
         for (int it = 0; it < ntiles; ++it) {
             const int qs = it % kSparseFwdQStages;
             // stage qs is free once the S MMA of tile it-3 has completed (one lane waits for the warp);
@@ -544,7 +549,7 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
             gather_rows_issue(smem_u32(smem + L::kQ + qs * 2 * kChunkBytes), Q, gw, lane, tn);
             cp_async_mbar_arrive_noinc(bar_q_full + qs);
-            if (it + 1 < ntiles) gather_rows_load(R, it + 1, gw, lane, tn);  // in flight during the next wait
+            if (it + 1 < ntiles) gather_rows_load<GQ>(R, it + 1, gw, lane, tn);  // in flight during the next wait
         }
         cp_async_wait_all();
     } else if (warp == 12) {
@@ -612,7 +617,7 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
         auto row_t = [&](int it) {
             int t = -1;
             size_t qrow;
-            return (it < ntiles && tile_row(R, it, r, t, qrow)) ? t : -1;
+            return (it < ntiles && tile_row<GQ>(R, it, r, t, qrow)) ? t : -1;
         };
         int t_n = row_t(g);
         // range exponent of the block: max |v| over V_j (bf16 in shared memory; the layout does

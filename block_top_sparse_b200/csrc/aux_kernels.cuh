@@ -171,7 +171,8 @@ __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t *__restri
 // holding o_i * 2^-e_j, where e_j >= 0 is the range exponent of key block
 // j = idx[query * k + i] (0 unless |V| in that block reaches 2^15); the word after
 // the last block's exponent is non-zero when any exponent is, and only then are
-// idx and the exponents read.  Lane i holds
+// idx and the exponents read.  For k <= 32 every slot's row is requested as soon as
+// the slot positions arrive, before the weights are known.  Lane i holds
 // slot i's position and weight (32 slots at a time), so the slots' row loads are
 // all in flight at once.  The merged fp32 row is stored as O = bf16(o) and, when
 // O_lo is given, O_lo = bf16(o - O).
@@ -184,6 +185,7 @@ __device__ __forceinline__ void half4_to_f32(uint2 u, float (&f)[4]) {
     f[3] = fb.y;
 }
 
+template <int NG>  // slot groups of 8 held in registers (k <= 8 * NG); NG = 0: any k, loads after the weights
 __global__ void __launch_bounds__(256) sparse_merge_kernel(const int32_t *__restrict__ pos,
                                                            const int32_t *__restrict__ idx,
                                                            const int32_t *__restrict__ bexp,
@@ -202,41 +204,70 @@ __global__ void __launch_bounds__(256) sparse_merge_kernel(const int32_t *__rest
     const int32_t *ps = pos + (bh * T + t) * k;
     const int32_t *js = idx + (bh * T + t) * k;
     const bool scaled = __ldg(bexp + (rows / T / G) * nb) != 0;
-    float mx = -INFINITY;
-    for (int i0 = 0; i0 < k; i0 += 32) {
-        const int p = (i0 + lane < k) ? __ldg(ps + i0 + lane) : -1;
-        if (p >= 0) mx = fmaxf(mx, __ldg(lsepart + (region + p) * G + hi));
-    }
+    auto part_row = [&](int p) {  // this lane's 4 columns of the partial at list position p
+        return __ldg(reinterpret_cast<const uint2 *>(Opart + ((region + p) * G + hi) * 128) + lane);
+    };
+    float mx = -INFINITY, wsum = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (NG > 0) {
+        // lane i holds slot i; every slot row is requested before the weights are known
+        const int p = lane < k ? __ldg(ps + lane) : -1;
+        uint2 u[8 * NG];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float wsum = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int i0 = 0; i0 < k; i0 += 32) {
-        const int p = (i0 + lane < k) ? __ldg(ps + i0 + lane) : -1;
+        for (int q = 0; q < 8 * NG; ++q) {
+            const int pq = __shfl_sync(0xffffffffu, p, q);
+            u[q] = (q < k && pq >= 0) ? part_row(pq) : make_uint2(0u, 0u);
+        }
+        const float l = p >= 0 ? __ldg(lsepart + (region + p) * G + hi) : -INFINITY;
+        mx = l;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         float w = 0.f, wo = 0.f;
         if (p >= 0) {
-            w = __expf(__ldg(lsepart + (region + p) * G + hi) - mx);
+            w = __expf(l - mx);
             // the partial's weight with its range exponent restored
-            wo = scaled ? ldexpf(w, __ldg(bexp + bh * nb + __ldg(js + i0 + lane))) : w;
+            wo = scaled ? ldexpf(w, __ldg(bexp + bh * nb + __ldg(js + lane))) : w;
         }
-        wsum += w;
-        const int n = min(32, k - i0);
-        for (int s0 = 0; s0 < n; s0 += 8) {
-            uint2 u[8];
-            float wu[8];
+        wsum = w;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int pq = __shfl_sync(0xffffffffu, p, (s0 + q) & 31);
-                wu[q] = __shfl_sync(0xffffffffu, wo, (s0 + q) & 31);
-                u[q] = (s0 + q < n && pq >= 0)
-                           ? __ldg(reinterpret_cast<const uint2 *>(Opart + ((region + pq) * G + hi) * 128) + lane)
-                           : make_uint2(0u, 0u);
+        for (int q = 0; q < 8 * NG; ++q) {
+            const float wq = __shfl_sync(0xffffffffu, wo, q);
+            float f[4];
+            half4_to_f32(u[q], f);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[c] = fmaf(wq, f[c], acc[c]);
+        }
+    } else {
+        for (int i0 = 0; i0 < k; i0 += 32) {
+            const int p = (i0 + lane < k) ? __ldg(ps + i0 + lane) : -1;
+            if (p >= 0) mx = fmaxf(mx, __ldg(lsepart + (region + p) * G + hi));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        for (int i0 = 0; i0 < k; i0 += 32) {
+            const int p = (i0 + lane < k) ? __ldg(ps + i0 + lane) : -1;
+            float w = 0.f, wo = 0.f;
+            if (p >= 0) {
+                w = __expf(__ldg(lsepart + (region + p) * G + hi) - mx);
+                wo = scaled ? ldexpf(w, __ldg(bexp + bh * nb + __ldg(js + i0 + lane))) : w;
             }
+            wsum += w;
+            const int n = min(32, k - i0);
+            for (int s0 = 0; s0 < n; s0 += 8) {
+                uint2 u[8];
+                float wu[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                float f[4];
-                half4_to_f32(u[q], f);
+                for (int q = 0; q < 8; ++q) {
+                    const int pq = __shfl_sync(0xffffffffu, p, (s0 + q) & 31);
+                    wu[q] = __shfl_sync(0xffffffffu, wo, (s0 + q) & 31);
+                    u[q] = (s0 + q < n && pq >= 0) ? part_row(pq) : make_uint2(0u, 0u);
+                }
 #pragma unroll
-                for (int c = 0; c < 4; ++c) acc[c] = fmaf(wu[q], f[c], acc[c]);
+                for (int q = 0; q < 8; ++q) {
+                    float f[4];
+                    half4_to_f32(u[q], f);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) acc[c] = fmaf(wu[q], f[c], acc[c]);
+                }
             }
         }
     }

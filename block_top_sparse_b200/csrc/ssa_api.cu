@@ -349,15 +349,17 @@ ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V,
     a.scale = S.scale;
     a.scale_log2 = S.scale * kLog2e;
     const unsigned units = static_cast<unsigned>(S.BHk * (sparse ? S.nb : (S.T + 127) / 128));
-    if (nkv == 128) {
-        const size_t sm = BwdSmem<128>::kTotal + 1024;
-        if (!set_smem(attn_bwd_kernel<128>, sm)) return SSA_ERR_CUDA;
-        attn_bwd_kernel<128><<<units, kBwdThreads, sm, st>>>(tmK, tmV, tmQ, tmdO, tmdQ, a);
-    } else {
-        const size_t sm = BwdSmem<64>::kTotal + 1024;
-        if (!set_smem(attn_bwd_kernel<64>, sm)) return SSA_ERR_CUDA;
-        attn_bwd_kernel<64><<<units, kBwdThreads, sm, st>>>(tmK, tmV, tmQ, tmdO, tmdQ, a);
-    }
+    // the grouped-head instantiations carry the group arithmetic; one query head per key head does not
+    auto run = [&](auto kernel, size_t sm) {
+        if (!set_smem(kernel, sm)) return false;
+        kernel<<<units, kBwdThreads, sm, st>>>(tmK, tmV, tmQ, tmdO, tmdQ, a);
+        return true;
+    };
+    const bool gq = S.G > 1;
+    const size_t sm128 = BwdSmem<128>::kTotal + 1024, sm64 = BwdSmem<64>::kTotal + 1024;
+    const bool launched = nkv == 128 ? (gq ? run(attn_bwd_kernel<128, true>, sm128) : run(attn_bwd_kernel<128, false>, sm128))
+                                     : (gq ? run(attn_bwd_kernel<64, true>, sm64) : run(attn_bwd_kernel<64, false>, sm64));
+    if (!launched) return SSA_ERR_CUDA;
     if (!g32) {
         const size_t n = S.rows * S.d;
         acc_to_out_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, st>>>(dQacc, (__nv_bfloat16 *)dQ, n, acc);
@@ -482,24 +484,31 @@ ssa_status_t ssa_sparse_attn_fwd(const ssa_dims_t *dims, const void *Q, const vo
         return SSA_ERR_CUDA;
     const unsigned units = static_cast<unsigned>(S.BHk * S.nb);
     const float sl2 = S.scale * kLog2e;
-    if (S.s == 128) {
-        const size_t sm = SparseFwdSmem<128>::kTotal + 1024;
-        if (!set_smem(sparse_fwd_kernel<128>, sm)) return SSA_ERR_CUDA;
-        sparse_fwd_kernel<128><<<units, kSparseFwdThreads, sm, st>>>(tmK, tmV, tmO, (const __nv_bfloat16 *)Q,
-                                                                      W.entries, W.lstart, W.llen, lsepart, bexp,
-                                                                      static_cast<int>(S.BHk), S.T, S.k, S.nb, S.G,
-                                                                      sl2);
-    } else {
-        const size_t sm = SparseFwdSmem<64>::kTotal + 1024;
-        if (!set_smem(sparse_fwd_kernel<64>, sm)) return SSA_ERR_CUDA;
-        sparse_fwd_kernel<64><<<units, kSparseFwdThreads, sm, st>>>(tmK, tmV, tmO, (const __nv_bfloat16 *)Q,
-                                                                     W.entries, W.lstart, W.llen, lsepart, bexp,
-                                                                     static_cast<int>(S.BHk), S.T, S.k, S.nb, S.G,
-                                                                     sl2);
-    }
-    sparse_merge_kernel<<<static_cast<unsigned>((S.rows + 7) / 8), 256, 0, st>>>(
-        W.pos, idx, bexp, Opart, lsepart, (__nv_bfloat16 *)O, (__nv_bfloat16 *)O_lo, lse, S.rows, S.T, S.k, S.nb,
-        S.G);
+    auto run = [&](auto kernel, size_t sm) {
+        if (!set_smem(kernel, sm)) return false;
+        kernel<<<units, kSparseFwdThreads, sm, st>>>(tmK, tmV, tmO, (const __nv_bfloat16 *)Q, W.entries, W.lstart,
+                                                     W.llen, lsepart, bexp, static_cast<int>(S.BHk), S.T, S.k, S.nb,
+                                                     S.G, sl2);
+        return true;
+    };
+    const bool gq = S.G > 1;
+    const size_t sm128 = SparseFwdSmem<128>::kTotal + 1024, sm64 = SparseFwdSmem<64>::kTotal + 1024;
+    const bool launched = S.s == 128 ? (gq ? run(sparse_fwd_kernel<128, true>, sm128) : run(sparse_fwd_kernel<128, false>, sm128))
+                                     : (gq ? run(sparse_fwd_kernel<64, true>, sm64) : run(sparse_fwd_kernel<64, false>, sm64));
+    if (!launched) return SSA_ERR_CUDA;
+    const unsigned mg = static_cast<unsigned>((S.rows + 7) / 8);
+    auto merge = [&](auto kernel) {
+        kernel<<<mg, 256, 0, st>>>(W.pos, idx, bexp, Opart, lsepart, (__nv_bfloat16 *)O, (__nv_bfloat16 *)O_lo, lse,
+                                   S.rows, S.T, S.k, S.nb, S.G);
+    };
+    if (S.k <= 8)
+        merge(sparse_merge_kernel<1>);
+    else if (S.k <= 16)
+        merge(sparse_merge_kernel<2>);
+    else if (S.k <= 32)
+        merge(sparse_merge_kernel<4>);
+    else
+        merge(sparse_merge_kernel<0>);
     return launch_status();
 }
 
