@@ -9,8 +9,9 @@
 // memory and the transposed accumulators dV_j^T, dK_j^T stay in tensor memory
 // for the whole unit.  Per query tile:
 //   S = Q K^T, dP = dO V^T                      (M = 128 query rows)
-//   P = exp(scale S - lse), dS = P o (dP - D)   -> shared memory, bf16
-//   dV^T += dO^T P, dK^T += Q^T dS              (M = head dim 128)
+//   P = exp(scale S - lse)                       -> shared memory, bf16; then
+//   dV^T += dO^T P  while  dS = P o (dP - D)     -> shared memory, bf16
+//   dK^T += Q^T dS                               (M = head dim 128)
 //   dQ = dS K, * scale                           -> added into an fp32 accumulator
 // Paper: section 4.2 (keys outside S(t) get no gradient; the selection is a
 // constant), FlashAttention-2 style recomputation of P from the saved lse.
@@ -29,9 +30,9 @@
 //                the staging buffer;
 //   warp 12      MMA issuer (one thread);
 //   warp 13      TMA producer (K_j, V_j; contiguous Q / dO tiles of the full stream);
-//   warps 14-19  sparse stream: gather the next tile's Q and dO rows with
-//                cp.async (a half-warp per 256-byte row) once the dV / dK MMAs
-//                of the current tile have consumed the buffers.
+//   warps 14-19  sparse stream: gather the next tile's dO rows once the dV MMAs
+//                of the current tile have read dO, then its Q rows once the dK
+//                MMAs have read Q, with cp.async (a half-warp per 256-byte row).
 //
 // Shared memory: Q 32 KB | dO 32 KB | K, V NKV*256 B each | P, dS (NKV/64)*16 KB each |
 //                dQ staging 32 KB
@@ -61,10 +62,50 @@ struct BwdArgs {
     float *dQacc;  // sparse stream: fp32 dQ accumulator [B*H*T, 128] (the full stream adds through tmdQ)
     void *dK, *dV;  // bf16, or fp32 when grad_fp32
     const int32_t *entries, *lstart, *llen;  // sparse only
+    const int32_t *order;                    // sparse: launch order of the (head, block) units
     int BH, T, k, nb, sparse, accumulate, grad_fp32;
     int G;  // query heads per key/value head; BH counts key/value heads
     float scale, scale_log2;
 };
+
+// Four consecutive gradient values of one key row of dV and dK (fp32 in registers) to the
+// caller's dV, dK at element offset `off`: bf16 or fp32, added to the existing values in fp32
+// first when accumulating (one rounding).
+__device__ __forceinline__ void write_grad4(const BwdArgs &a, size_t off, float4 v4, float4 k4) {
+    if (a.grad_fp32) {
+        float4 *dv4 = reinterpret_cast<float4 *>(static_cast<float *>(a.dV) + off);
+        float4 *dk4 = reinterpret_cast<float4 *>(static_cast<float *>(a.dK) + off);
+        if (a.accumulate) {
+            const float4 ov = *dv4, ok4 = *dk4;
+            v4.x += ov.x;
+            v4.y += ov.y;
+            v4.z += ov.z;
+            v4.w += ov.w;
+            k4.x += ok4.x;
+            k4.y += ok4.y;
+            k4.z += ok4.z;
+            k4.w += ok4.w;
+        }
+        *dv4 = v4;
+        *dk4 = k4;
+        return;
+    }
+    uint2 *dv2 = reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.dV) + off);
+    uint2 *dk2 = reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.dK) + off);
+    if (a.accumulate) {
+        const uint2 ov = *dv2, ok2 = *dk2;
+        v4.x += __uint_as_float(ov.x << 16);
+        v4.y += __uint_as_float(ov.x & 0xFFFF0000u);
+        v4.z += __uint_as_float(ov.y << 16);
+        v4.w += __uint_as_float(ov.y & 0xFFFF0000u);
+        k4.x += __uint_as_float(ok2.x << 16);
+        k4.y += __uint_as_float(ok2.x & 0xFFFF0000u);
+        k4.z += __uint_as_float(ok2.y << 16);
+        k4.w += __uint_as_float(ok2.y & 0xFFFF0000u);
+    }
+    *dv2 = make_uint2(pack_bf16x2(v4.x, v4.y), pack_bf16x2(v4.z, v4.w));
+    *dk2 = make_uint2(pack_bf16x2(k4.x, k4.y), pack_bf16x2(k4.z, k4.w));
+}
 
 // 640 threads launched with 96 registers each (61,440); setmaxnreg moves them to
 // softmax 2 x 144, flush 96, MMA / producer / gather 2 x 48: 128 * 480 = 61,440.
@@ -87,18 +128,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint64_t *bar_f_staged = bars + 8, *bar_f_free = bars + 9;  // dQ staging buffer handshakes
     uint64_t *bar_p_free = bars + 12;  // the P region's dQ half has been read by the flush
     uint64_t *bar_epi = bars + 13;     // the dV / dK staging of the epilogue is complete
-    // full stream: dO has its own load / release barriers (released after the dV MMAs, before
-    // Q, which the dK MMAs still read); the sparse gather brings Q and dO together on bar_qdo_full
+    // dO has its own load / release barriers (released after the dV MMAs, before Q, which the dK
+    // MMAs still read), so that the next tile's dO arrives and its dP runs during dK / dQ
     uint64_t *bar_do_full = bars + 14, *bar_do_free = bars + 15;
+    uint64_t *bar_ds_full = bars + 16;  // dS stored (bar_pds_full: P stored)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 11);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = a.T;
-    // Head-major unit order: the query rows and the dQ accumulator of the head
-    // being worked on stay in L2.
-    const int units_per_head = a.sparse ? a.nb : (a.T + NKV - 1) / NKV;
+    // Unit order: sparse, the index's (heaviest units first, then head-major); full, head-major
+    // with each head's longest unit first.  Head-major keeps the query rows and the dQ
+    // accumulator of the head being worked on in L2.
     int bh, kb;  // key/value head, key tile (block)
-    unit_order(blockIdx.x, a.BH, units_per_head, bh, kb);
+    if (a.order) {
+        const int u = __ldg(a.order + blockIdx.x);
+        bh = u / a.nb;
+        kb = u - bh * a.nb;
+    } else {
+        unit_order(blockIdx.x, a.BH, (a.T + NKV - 1) / NKV, bh, kb);
+    }
     const int kv0 = kb * NKV;
     const size_t head_rows = static_cast<size_t>(bh) * T;  // key/value rows of this head
     const bool sparse = a.sparse != 0;
@@ -134,8 +182,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(bar_qdo_full, sparse ? 32 * kBwdGatherWarps : 1);
         mbar_init(bar_sdp_full, 1);
         mbar_init(bar_pds_full, 256);
+        mbar_init(bar_ds_full, 256);
         mbar_init(bar_qdo_free, 1);
-        mbar_init(bar_do_full, 1);
+        mbar_init(bar_do_full, sparse ? 32 * kBwdGatherWarps : 1);
         mbar_init(bar_do_free, 1);
         mbar_init(bar_dq_full, 1);
         mbar_init(bar_dq_empty, 128);
@@ -175,12 +224,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         tn[q] = (p < 64 && tile_row<GQ>(R, it, 2 * p + (lane >> 4), t, row)) ? static_cast<int>(row) : -1;
                     }
                 };
-                load_rows(0);
-                for (int it = 0; it < ntiles; ++it) {
-                    // Q / dO are free once the dV / dK MMAs of the previous tile have completed
-                    bool ok = true;
-                    if (lane == 0 && it > 0) ok = mbar_wait(bar_qdo_free, (it - 1) & 1, abort_flag, 0x312);
-                    if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+                // this lane's rows of one 256-byte-row tensor into a 2-chunk swizzled tile
+                auto gather = [&](uint32_t tile, const __nv_bfloat16 *src) {
 #pragma unroll
                     for (int q = 0; q < kBwdGatherPairs; ++q) {
                         const int p = gw + kBwdGatherWarps * q;
@@ -188,13 +233,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                             const int r = 2 * p + (lane >> 4);
                             const uint32_t off = (u >> 3) * kChunkBytes + r * 128 + ((((u & 7) ^ (r & 7)) & 7) << 4);
                             const bool valid = tn[q] >= 0;
-                            const size_t src = static_cast<size_t>(valid ? tn[q] : 0) * kD + u * 8;
-                            cp_async_16(sQ + off, a.Q + src, valid ? 16u : 0u);
-                            cp_async_16(sdO + off, a.dO + src, valid ? 16u : 0u);
+                            cp_async_16_row(tile + off, src + u * 8, valid ? static_cast<uint32_t>(tn[q]) : 0u,
+                                            valid ? 16u : 0u);
                         }
                     }
-                    cp_async_mbar_arrive_noinc(bar_qdo_full);
-                    if (it + 1 < ntiles) load_rows(it + 1);  // in flight during the next wait
+                };
+                load_rows(0);
+                bool ok = true;
+                for (int it = 0; ok && it < ntiles; ++it) {
+                    // dO is free once the dV MMAs of the previous tile have completed, Q once its dK MMAs
+                    // have: dO comes first, so that dP of this tile can run while dK, dQ of the previous
+                    // one do.  (One wait site for both: the loop runs twice per tile.)
+#pragma unroll 1
+                    for (int ph = 0; ph < 2; ++ph) {
+                        if (lane == 0 && it > 0)
+                            ok = mbar_wait(ph == 0 ? bar_do_free : bar_qdo_free, (it - 1) & 1, abort_flag, 0x312 + ph);
+                        ok = __shfl_sync(0xffffffffu, ok, 0);
+                        if (!ok) break;
+                        gather(ph == 0 ? sdO : sQ, ph == 0 ? a.dO : a.Q);
+                        cp_async_mbar_arrive_noinc(ph == 0 ? bar_do_full : bar_qdo_full);
+                    }
+                    if (ok && it + 1 < ntiles) load_rows(it + 1);  // in flight during the next wait
                 }
                 cp_async_wait_all();
             }
@@ -239,24 +298,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 for (int it = 0; ok && it < ntiles; ++it) {
                     // dP first (its columns are free once the previous tile's P/dS were formed), then S,
                     // which overwrites the previous tile's dQ once the flush has taken it out
-                    if (!mbar_wait(sparse ? bar_qdo_full : bar_do_full, it & 1, abort_flag, 0x302)) break;
+                    if (!mbar_wait(bar_do_full, it & 1, abort_flag, 0x302)) break;
                     if (sparse) fence_proxy_async_smem();  // cp.async-written rows -> tensor-core reads
                     tc_fence_after();
                     mma_k128_kmajor(tdP, sdO, sV, NKV * 128, idS);
-                    if (!sparse && !mbar_wait(bar_qdo_full, it & 1, abort_flag, 0x315)) break;
+                    if (!mbar_wait(bar_qdo_full, it & 1, abort_flag, 0x315)) break;
+                    if (sparse) fence_proxy_async_smem();
                     if (it > 0 && !mbar_wait(bar_dq_empty, (it - 1) & 1, abort_flag, 0x303)) break;
                     tc_fence_after();
                     mma_k128_kmajor(tS, sQ, sK, NKV * 128, idS);
                     mma_commit(bar_sdp_full);
+                    // dV^T[d x kv] += dO^T P as soon as P is stored (while dS is formed); then
+                    // dK^T[d x kv] += Q^T dS   (K = 128 query rows)
                     if (!mbar_wait(bar_pds_full, it & 1, abort_flag, 0x304)) break;
                     tc_fence_after();
-                    // dV^T[d x kv] += dO^T P ; dK^T[d x kv] += Q^T dS   (K = 128 query rows)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         mma_bf16_ss(tdV, smem_desc_sw128(sdO + kk * 2048, kChunkBytes),
                                     smem_desc_sw128(sP + kk * 2048, kChunkBytes), idT, (it > 0 || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(bar_do_free);
+                    if (!mbar_wait(bar_ds_full, it & 1, abort_flag, 0x316)) break;
+                    tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
                         mma_bf16_ss(tdK, smem_desc_sw128(sQ + kk * 2048, kChunkBytes),
@@ -436,11 +499,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int lim = valid ? t - kv0 - h * HALF : -1;
             const uint64_t sl2 = f2_pack(a.scale_log2, a.scale_log2), nl2 = f2_pack(-lse2, -lse2),
                            nD = f2_pack(-Dt, -Dt);
+            // P = 2^(s * scale_log2 - lse2) first, stored so that the dV MMAs start while dS is formed
+            float p[HALF];
 #pragma unroll
             for (int c = 0; c < HALF / 32; ++c) {
-                uint32_t sraw[32], draw[32];
+                uint32_t sraw[32];
                 tmem_ld32_async(tS + lane_off + h * HALF + 32 * c, sraw);
-                tmem_ld32_async(tdP + lane_off + h * HALF + 32 * c, draw);
                 tmem_ld_wait();
                 // masked scores become -inf (only warps holding a masked column pay for it)
                 if (!__all_sync(0xffffffffu, lim >= 32 * c + 31)) {
@@ -448,27 +512,41 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     for (int i = 0; i < 32; ++i)
                         if (32 * c + i > lim) sraw[i] = 0xff800000u;
                 }
-                // p = 2^(s * scale_log2 - lse2), ds = p * (dp - D), in packed pairs
-                float sv[32], dp[32];
+                float sv[32];
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
                     float x0, x1;
                     f2_unpack(ffma2(f2_pack(__uint_as_float(sraw[i]), __uint_as_float(sraw[i + 1])), sl2, nl2), x0, x1);
                     sv[i] = fast_exp2(x0);
                     sv[i + 1] = fast_exp2(x1);
-                    f2_unpack(fmul2(f2_pack(sv[i], sv[i + 1]),
-                                    fadd2(f2_pack(__uint_as_float(draw[i]), __uint_as_float(draw[i + 1])), nD)),
-                              dp[i], dp[i + 1]);
+                    p[32 * c + i] = sv[i];
+                    p[32 * c + i + 1] = sv[i + 1];
                 }
                 // full stream: the previous tile's dQ staged over P (and dS for 64-key units) has been read
                 if (!sparse && c == 0 && it > 0) ok = mbar_wait(bar_p_free, (it - 1) & 1, abort_flag, 0x30d);
                 store_row32_bf16(sP, kChunkBytes, r, h * HALF + 32 * c, sv);
-                store_row32_bf16(sdS, kChunkBytes, r, h * HALF + 32 * c, dp);
             }
             if (!ok) break;
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(bar_pds_full);
+            // dS = P o (dP - D), in packed pairs
+#pragma unroll
+            for (int c = 0; c < HALF / 32; ++c) {
+                uint32_t draw[32];
+                tmem_ld32_async(tdP + lane_off + h * HALF + 32 * c, draw);
+                tmem_ld_wait();
+                float dp[32];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2)
+                    f2_unpack(fmul2(f2_pack(p[32 * c + i], p[32 * c + i + 1]),
+                                    fadd2(f2_pack(__uint_as_float(draw[i]), __uint_as_float(draw[i + 1])), nD)),
+                              dp[i], dp[i + 1]);
+                store_row32_bf16(sdS, kChunkBytes, r, h * HALF + 32 * c, dp);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar_ds_full);
         }
         // Epilogue.  dV^T / dK^T (thread <-> head-dim row r, key columns of its half) are restaged in
         // fp32 as [key][dim] rows over the idle operand buffers (dV over Q/dO, dK over K/V, NKV rows of
@@ -508,40 +586,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                              : "=f"(k4.x), "=f"(k4.y), "=f"(k4.z), "=f"(k4.w)
                              : "r"(sdk + kr * 512 + lane * 16));
                 const size_t off = (head_rows + kv0 + kr) * kD + 4 * lane;
-                if (a.grad_fp32) {
-                    // fp32 gradients: 16 bytes per lane, added to the existing values when asked
-                    float4 *dv4 = reinterpret_cast<float4 *>(static_cast<float *>(a.dV) + off);
-                    float4 *dk4 = reinterpret_cast<float4 *>(static_cast<float *>(a.dK) + off);
-                    if (a.accumulate) {
-                        const float4 ov = *dv4, ok4 = *dk4;
-                        v4.x += ov.x;
-                        v4.y += ov.y;
-                        v4.z += ov.z;
-                        v4.w += ov.w;
-                        k4.x += ok4.x;
-                        k4.y += ok4.y;
-                        k4.z += ok4.z;
-                        k4.w += ok4.w;
-                    }
-                    *dv4 = v4;
-                    *dk4 = k4;
-                    continue;
-                }
-                uint2 *dv2 = reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.dV) + off);
-                uint2 *dk2 = reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.dK) + off);
-                if (a.accumulate) {
-                    const uint2 ov = *dv2, ok2 = *dk2;
-                    v4.x += __uint_as_float(ov.x << 16);
-                    v4.y += __uint_as_float(ov.x & 0xFFFF0000u);
-                    v4.z += __uint_as_float(ov.y << 16);
-                    v4.w += __uint_as_float(ov.y & 0xFFFF0000u);
-                    k4.x += __uint_as_float(ok2.x << 16);
-                    k4.y += __uint_as_float(ok2.x & 0xFFFF0000u);
-                    k4.z += __uint_as_float(ok2.y << 16);
-                    k4.w += __uint_as_float(ok2.y & 0xFFFF0000u);
-                }
-                *dv2 = make_uint2(pack_bf16x2(v4.x, v4.y), pack_bf16x2(v4.z, v4.w));
-                *dk2 = make_uint2(pack_bf16x2(k4.x, k4.y), pack_bf16x2(k4.z, k4.w));
+                write_grad4(a, off, v4, k4);
             }
         }
     }

@@ -394,8 +394,9 @@ __global__ void __launch_bounds__(kFullFwdThreads, 1)
 
 // ---------------------------------------------------------------------------
 // Sparse forward, block-major, two warpgroups in ping-pong.
-// grid = (B*Hkv*nb): unit u -> key/value head bh = u / nb, block j = u % nb
-// (head-major, so the head's query rows stay in L2); a tile holds 128 / G list
+// grid = (B*Hkv*nb): CTA i takes unit u = order[i] of the index, key/value head
+// bh = u / nb, block j = u % nb (the heaviest units first, the rest head-major so
+// that the head's query rows stay in L2); a tile holds 128 / G list
 // entries for each of the G query heads reading the key head.  block = 512 threads:
 //   warpgroup g (warps 4g .. 4g+3) owns the query tiles it = g, g+2, ... of the
 //   block's list: masked softmax over the block's NKV keys, P written back over
@@ -412,8 +413,10 @@ __global__ void __launch_bounds__(kFullFwdThreads, 1)
 //   half-warp per 256-byte row (a gather's cost is set by the number of warp
 //   instructions in flight, so seven warps share it; completion on an mbarrier);
 //   warp 12 loads K_j, V_j (TMA) and issues each S(it) as soon as its query
-//   rows have landed and each PV(it) as soon as its P is ready (polling both,
-//   S(it) never ahead of PV(it-2), whose P it overwrites), so that one
+//   rows have landed and each PV(it) as soon as its P is ready (polling both
+//   with the non-suspending test_wait, so that a barrier that is not ready
+//   cannot hold up the other; S(it) never ahead of PV(it-2), whose P it
+//   overwrites), so that one
 //   warpgroup's softmax overlaps the other's MMAs and epilogue.
 // smem: Q[3] 32 KB each | K, V NKV*256 each | O staging[2] 32 KB each | barriers
 // tmem: S/P[2] at 0 / 128, O[2] at 256 / 384 (512 allocated).
@@ -473,7 +476,8 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
     sparse_fwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmO, const __nv_bfloat16 *__restrict__ Q,
                       const int32_t *__restrict__ entries, const int32_t *__restrict__ lstart,
-                      const int32_t *__restrict__ llen, float *__restrict__ lsepart, int32_t *__restrict__ bexp,
+                      const int32_t *__restrict__ llen, const int32_t *__restrict__ order,
+                      float *__restrict__ lsepart, int32_t *__restrict__ bexp,
                       int BH, int T, int k, int nb, int G, float scale_log2) {
     using L = SparseFwdSmem<NKV>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -491,8 +495,12 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
     uint32_t *vmax_part = reinterpret_cast<uint32_t *>(bars + 24);  // [8] per softmax warp, |v| bits
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int bh, j;  // key/value head, key block
-    unit_order(blockIdx.x, BH, nb, bh, j);
+    int bh, j;  // key/value head, key block, in the index's launch order (heaviest units first)
+    {
+        const int u = __ldg(order + blockIdx.x);
+        bh = u / nb;
+        j = u - bh * nb;
+    }
     const int kv0 = j * NKV;
     const size_t head_rows = static_cast<size_t>(bh) * T;  // key/value rows of this head
     // this block's list starts at list position obase; its partial-output rows at obase * G
@@ -568,7 +576,7 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
             uint64_t t_idle = globaltimer_ns();
             while (ok && ip < ntiles) {
                 bool progressed = false;
-                if (ip < is && mbar_try_wait(bar_p_full + (ip & 1), (ip >> 1) & 1)) {
+                if (ip < is && mbar_test_wait(bar_p_full + (ip & 1), (ip >> 1) & 1)) {
                     const int g = ip & 1;
                     tc_fence_after();
                     // O_g = P_g V : A = P from tensor memory (bf16 pairs over S_g), B = V [NKV x d] MN-major
@@ -581,7 +589,7 @@ __global__ void __launch_bounds__(kSparseFwdThreads, 1)
                     progressed = true;
                 }
                 if (is < ntiles && is < ip + 2 &&
-                    mbar_try_wait(bar_q_full + is % kSparseFwdQStages, (is / kSparseFwdQStages) & 1)) {
+                    mbar_test_wait(bar_q_full + is % kSparseFwdQStages, (is / kSparseFwdQStages) & 1)) {
                     const int g = is & 1;
                     fence_proxy_async_smem();  // cp.async-written rows -> tensor-core reads
                     tc_fence_after();

@@ -1,6 +1,7 @@
 // aux_kernels.cuh -- bandwidth-bound helpers of the attention path:
 //   * inverse selection index (key block -> list of (query, slot) entries,
-//     ascending in query position), built deterministically in three passes;
+//     ascending in query position), built deterministically in three passes,
+//     and the launch order of the block-major units (heaviest first);
 //   * merge of the block-major sparse forward's per-slot partial outputs;
 //   * backward pre/post-processing (D = rowsum(dO o (O + O_lo)), dQ accumulator -> dQ);
 //   * bidirectional SmoothL1 alignment loss forward/backward (paper section 5);
@@ -160,6 +161,95 @@ __global__ void __launch_bounds__(128) index_fill_kernel(const int32_t *__restri
             }
         }
         __syncwarp();
+    }
+}
+
+// Pass 4 (one CTA): launch order of the (head, key block) units of the block-major
+// attention kernels.  A unit's work is its number of query tiles, ceil(len / per_tile),
+// and the lists are very uneven (early blocks and attention-sink blocks are chosen by
+// many queries), so units of at least 5/4 of the mean come first, heaviest first (in
+// kOrdHeavy buckets of equal width between the threshold and the maximum); the rest
+// follow in head-major order, which keeps the head being worked on in L2.  A stable
+// counting sort (ranks from warp match masks, per-warp bucket counts scanned in
+// shared memory), so the order is deterministic.
+constexpr int kOrdHeavy = 63;            // buckets of heavy units; bucket kOrdHeavy holds the rest
+constexpr int kOrdBuckets = kOrdHeavy + 1;
+
+__global__ void __launch_bounds__(1024) unit_order_kernel(const int *__restrict__ llen, int32_t *__restrict__ order,
+                                                          int units, int per_tile) {
+    __shared__ int wcnt[32][kOrdBuckets];  // per-warp bucket counts of the current chunk, then their offsets
+    __shared__ int start[kOrdBuckets];     // running write position of every bucket
+    __shared__ unsigned long long red_tot[32];
+    __shared__ int red_max[32];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    auto tiles_of = [&](int u) { return (__ldg(llen + u) + per_tile - 1) / per_tile; };
+    // total and largest work
+    unsigned long long tot = 0;
+    int mx = 0;
+    for (int u = tid; u < units; u += blockDim.x) {
+        const int t = tiles_of(u);
+        tot += static_cast<unsigned long long>(t);
+        mx = max(mx, t);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (lane == 0) {
+        red_tot[warp] = tot;
+        red_max[warp] = mx;
+    }
+    __syncthreads();
+    tot = 0;
+    mx = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
+        tot += red_tot[w];
+        mx = max(mx, red_max[w]);
+    }
+    const int thr = max(2, static_cast<int>((5 * tot + 4ull * units - 1) / (4ull * units)));
+    auto bucket_of = [&](int u) {
+        const int t = tiles_of(u);
+        if (t < thr) return kOrdHeavy;
+        return mx > thr ? static_cast<int>(static_cast<long long>(mx - t) * (kOrdHeavy - 1) / (mx - thr)) : 0;
+    };
+    // bucket sizes -> first position of every bucket
+    for (int b = tid; b < kOrdBuckets; b += blockDim.x) start[b] = 0;
+    __syncthreads();
+    for (int u = tid; u < units; u += blockDim.x) atomicAdd(&start[bucket_of(u)], 1);
+    __syncthreads();
+    if (tid == 0) {
+        int acc = 0;
+        for (int b = 0; b < kOrdBuckets; ++b) {
+            const int c = start[b];
+            start[b] = acc;
+            acc += c;
+        }
+    }
+    __syncthreads();
+    // stable scatter, one unit per thread per chunk
+    const int nw = blockDim.x >> 5;
+    for (int u0 = 0; u0 < units; u0 += blockDim.x) {
+        const int u = u0 + tid;
+        const int b = u < units ? bucket_of(u) : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, b);
+        const int rank = __popc(same & ((1u << lane) - 1u));
+        for (int i = lane; i < kOrdBuckets; i += 32) wcnt[warp][i] = 0;
+        __syncwarp();
+        if (b >= 0 && rank == 0) wcnt[warp][b] = __popc(same);
+        __syncthreads();
+        for (int i = tid; i < kOrdBuckets; i += blockDim.x) {  // exclusive scan over warps, per bucket
+            int acc = start[i];
+            for (int w = 0; w < nw; ++w) {
+                const int c = wcnt[w][i];
+                wcnt[w][i] = acc;
+                acc += c;
+            }
+            start[i] = acc;
+        }
+        __syncthreads();
+        if (b >= 0) order[wcnt[warp][b] + rank] = u;
+        __syncthreads();
     }
 }
 

@@ -69,6 +69,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe of phase `parity` (mbarrier.test_wait never suspends the thread, unlike
+// try_wait): for a thread that polls several barriers and must act on whichever completes first.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait on phase `parity`.  Returns false (and records the site) when the
 // phase did not complete within limit_ns or when another thread of the CTA
 // already aborted (abort flag in shared memory).
@@ -121,6 +135,19 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void *src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes)
                  : "memory");
+}
+
+// 16-byte cp.async of row `row` of a tensor with 256-byte rows: source = base + row * 256, the
+// address formed inside the instruction block so that gathers of several tensors from the same rows
+// keep only the 32-bit row indices live (not one 64-bit address per row and tensor).
+__device__ __forceinline__ void cp_async_16_row(uint32_t dst_smem, const void *base, uint32_t row, uint32_t src_bytes) {
+    asm volatile(
+        "{\n\t.reg .u64 a;\n\t"
+        "mul.wide.u32 a, %2, 256;\n\t"
+        "add.u64 a, a, %1;\n\t"
+        "cp.async.cg.shared.global [%0], [a], 16, %3;\n\t}" ::"r"(dst_smem),
+        "l"(base), "r"(row), "r"(src_bytes)
+        : "memory");
 }
 
 // Arrive on `bar` once every cp.async this thread issued so far has landed; the

@@ -85,13 +85,14 @@ struct IndexWs {
     int *cnt, *lstart, *llen;
     int32_t *entries;  // per head: list_stride(T, k, nb) entries, block lists on 128-entry boundaries
     int32_t *pos;      // [B*H*T, k] list position of every (query, slot), -1 when unused
+    int32_t *order;    // [B*Hk*nb] launch order of the (head, block) units, heaviest first
     int nch;
 };
 
 size_t index_bytes(const Shape &S) {
     if (!S.tc) return 0;
     const size_t nch = (S.T + kIdxChunk - 1) / kIdxChunk;
-    return align_up(S.BHk * nch * S.nb * 4) + 2 * align_up(S.BHk * S.nb * 4) +
+    return align_up(S.BHk * nch * S.nb * 4) + 3 * align_up(S.BHk * S.nb * 4) +
            align_up(S.BHk * list_stride(S.T, S.k, S.nb) * 4) + align_up(S.krows * S.k * 4);
 }
 
@@ -108,6 +109,8 @@ IndexWs carve_index(const Shape &S, const void *base) {
     W.entries = reinterpret_cast<int32_t *>(p);
     p += align_up(S.BHk * list_stride(S.T, S.k, S.nb) * 4);
     W.pos = reinterpret_cast<int32_t *>(p);
+    p += align_up(S.krows * S.k * 4);
+    W.order = reinterpret_cast<int32_t *>(p);
     return W;
 }
 
@@ -241,6 +244,7 @@ ssa_status_t build_index(const Shape &S, const int32_t *idx, const IndexWs &W, c
     if (!set_smem(index_fill_kernel, wbytes * wpc)) return SSA_ERR_CUDA;
     index_fill_kernel<<<dim3((W.nch + wpc - 1) / wpc, S.BHk), 32 * wpc, wbytes * wpc, st>>>(
         idx, W.cnt, W.entries, W.pos, S.T, S.k, S.nb, W.nch);
+    unit_order_kernel<<<1, 1024, 0, st>>>(W.llen, W.order, static_cast<int>(S.BHk) * S.nb, kTileQ / S.G);
     return launch_status();
 }
 
@@ -338,6 +342,7 @@ ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V,
     a.entries = W.entries;
     a.lstart = W.lstart;
     a.llen = W.llen;
+    a.order = sparse ? W.order : nullptr;
     a.BH = static_cast<int>(S.BHk);
     a.G = S.G;
     a.T = S.T;
@@ -349,13 +354,13 @@ ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V,
     a.scale = S.scale;
     a.scale_log2 = S.scale * kLog2e;
     const unsigned units = static_cast<unsigned>(S.BHk * (sparse ? S.nb : (S.T + 127) / 128));
+    const bool gq = S.G > 1;
     // the grouped-head instantiations carry the group arithmetic; one query head per key head does not
     auto run = [&](auto kernel, size_t sm) {
         if (!set_smem(kernel, sm)) return false;
         kernel<<<units, kBwdThreads, sm, st>>>(tmK, tmV, tmQ, tmdO, tmdQ, a);
         return true;
     };
-    const bool gq = S.G > 1;
     const size_t sm128 = BwdSmem<128>::kTotal + 1024, sm64 = BwdSmem<64>::kTotal + 1024;
     const bool launched = nkv == 128 ? (gq ? run(attn_bwd_kernel<128, true>, sm128) : run(attn_bwd_kernel<128, false>, sm128))
                                      : (gq ? run(attn_bwd_kernel<64, true>, sm64) : run(attn_bwd_kernel<64, false>, sm64));
@@ -487,7 +492,7 @@ ssa_status_t ssa_sparse_attn_fwd(const ssa_dims_t *dims, const void *Q, const vo
     auto run = [&](auto kernel, size_t sm) {
         if (!set_smem(kernel, sm)) return false;
         kernel<<<units, kSparseFwdThreads, sm, st>>>(tmK, tmV, tmO, (const __nv_bfloat16 *)Q, W.entries, W.lstart,
-                                                     W.llen, lsepart, bexp, static_cast<int>(S.BHk), S.T, S.k, S.nb,
+                                                     W.llen, W.order, lsepart, bexp, static_cast<int>(S.BHk), S.T, S.k, S.nb,
                                                      S.G, sl2);
         return true;
     };
