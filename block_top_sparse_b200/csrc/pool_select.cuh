@@ -335,12 +335,17 @@ constexpr int kSelTcRows = 128;
 constexpr int kSelTcThreads = 512;
 constexpr int kSelTcMaxBlocks = 256;
 
+constexpr int kSelList = 16;  // register top list per thread (k - 1 <= kSelList)
+
 struct SelTcSmem {
     static constexpr int kQ = 0;                      // 128 rows x 128 bf16: 2 swizzled 16 KB chunks
-    static constexpr int kB = 2 * 16384;              // hi / mid / lo: 3 x (64 blocks x 128 bf16), 16 KB each
-    static constexpr int kCnt = kB + 3 * 16384;       // [2 steps][4 column groups][128 rows] partial counts
+    static constexpr int kB = 2 * 16384;              // [2 buffers] hi / mid / lo: 3 x (64 blocks x 128 bf16)
+    static constexpr int kBBuf = 3 * 16384;
+    static constexpr int kCnt = kB + 2 * kBBuf;       // [2 steps][4 column groups][128 rows] partial counts
     static constexpr int kMask = kCnt + 2 * 4 * 128 * 4;  // [8 chunks][128 rows] x {above, equal} masks
-    static constexpr int kBar = kMask + 2 * 8 * 128 * 4;
+    static constexpr int kList = kMask + 2 * 8 * 128 * 4;  // [4 column groups][128 rows][kSelList] top lists
+    static constexpr int kThr = kList + 4 * 128 * kSelList * 4;  // [128 rows] thresholds
+    static constexpr int kBar = kThr + 128 * 4;
     static constexpr int kTotal = kBar + 64;
 };
 
@@ -369,6 +374,8 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
     int *cnt_sm = reinterpret_cast<int *>(smem + L::kCnt);          // [2][4][128]
     uint32_t *gt_sm = reinterpret_cast<uint32_t *>(smem + L::kMask);  // [8][128]
     uint32_t *eq_sm = gt_sm + 8 * 128;                                // [8][128]
+    float *list_sm = reinterpret_cast<float *>(smem + L::kList);      // [4][128][kSelList]
+    float *thr_sm = reinterpret_cast<float *>(smem + L::kThr);        // [128]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.y, t0 = blockIdx.x * kSelTcRows;
     const size_t head_rows = static_cast<size_t>(bh) * T_len;
@@ -406,9 +413,9 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
     int phase = 0;  // completed MMA batches (bar_mma phases)
-    for (int gi = 0; gi < ngroups && ok; ++gi) {
-        // Kbar rows 64gi .. 64gi+63 -> hi / mid / lo tiles (K-major, swizzled); rows >= nbc are zero.
-        // Lane c4 of a warp takes dims 4c4 .. 4c4+3 of one row: two 128-byte row halves per store.
+    // Kbar rows 64gi .. 64gi+63 -> hi / mid / lo tiles (K-major, swizzled) of buffer sBb; rows >= nbc are
+    // zero.  Lane c4 of a warp takes dims 4c4 .. 4c4+3 of one row: two 128-byte row halves per store.
+    auto convert = [&](int gi, uint32_t sBb) {
         const int c4 = lane;
         for (int jj = warp; jj < 64; jj += kSelTcThreads / 32) {
             const int j = 64 * gi + jj;
@@ -421,30 +428,55 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
             const uint32_t l01 = pack_bf16x2(r0 - __uint_as_float(m01 << 16), r1 - __uint_as_float(m01 & 0xFFFF0000u));
             const uint32_t l23 = pack_bf16x2(r2 - __uint_as_float(m23 << 16), r3 - __uint_as_float(m23 & 0xFFFF0000u));
             const uint32_t off = (c4 >> 4) * 8192 + jj * 128 + (((((c4 & 15) >> 1) ^ (jj & 7)) & 7) << 4) + (c4 & 1) * 8;
-            st_shared_v2(sB + off, h01, h23);
-            st_shared_v2(sB + 16384 + off, m01, m23);
-            st_shared_v2(sB + 2 * 16384 + off, l01, l23);
+            st_shared_v2(sBb + off, h01, h23);
+            st_shared_v2(sBb + 16384 + off, m01, m23);
+            st_shared_v2(sBb + 2 * 16384 + off, l01, l23);
         }
         fence_proxy_async_smem();  // generic-proxy tile writes -> tensor-core reads
-        // with grouped query heads the group's tiles are added one after another into the same scores
-        for (int hi = 0; hi < G && ok; ++hi) {
-            if (G > 1) load_q(hi);  // the previous batch's MMAs have read the tile (waited below)
-            __syncthreads();
-            if (tid == 0) {
-                tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 64, false, false);
+    };
+    // S[:, 64gi ..] (+)= Q [hi | mid | lo]^T, issued by one thread, completion on bar_mma
+    auto issue = [&](int gi, uint32_t sBb, bool acc0) {
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 64, false, false);
 #pragma unroll
-                for (int sp = 0; sp < 3; ++sp)
+            for (int sp = 0; sp < 3; ++sp)
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16_ss(tmem + 64 * gi, smem_desc_sw128(sQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
-                                    smem_desc_sw128(sB + sp * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32, 16), id,
-                                    (hi > 0 || sp > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(bar_mma);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16_ss(tmem + 64 * gi, smem_desc_sw128(sQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16),
+                                smem_desc_sw128(sBb + sp * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32, 16), id,
+                                (acc0 || sp > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(bar_mma);
+        }
+    };
+    if (G == 1) {
+        // the split of group gi is written while the MMAs of group gi-1 run (two buffers: buffer gi & 1
+        // was last read by the MMAs of group gi-2, which completed before group gi-1 was issued)
+        for (int gi = 0; gi < ngroups && ok; ++gi) {
+            convert(gi, sB + (gi & 1) * L::kBBuf);
+            if (gi > 0) {
+                if (!mbar_wait(bar_mma, phase & 1, abort_flag, 0x501)) ok = false;
+                ++phase;
             }
-            // the split tiles and the query tile are rewritten only after these MMAs have read them
+            __syncthreads();
+            issue(gi, sB + (gi & 1) * L::kBBuf, false);
+        }
+        if (ok && ngroups > 0) {
             if (!mbar_wait(bar_mma, phase & 1, abort_flag, 0x501)) ok = false;
             ++phase;
+        }
+    } else {
+        for (int gi = 0; gi < ngroups && ok; ++gi) {
+            convert(gi, sB);
+            // with grouped query heads the group's tiles are added one after another into the same scores
+            for (int hi = 0; hi < G && ok; ++hi) {
+                load_q(hi);  // the previous batch's MMAs have read the tile (waited below)
+                __syncthreads();
+                issue(gi, sB, hi > 0);
+                // the split tiles and the query tile are rewritten only after these MMAs have read them
+                if (!mbar_wait(bar_mma, phase & 1, abort_flag, 0x501)) ok = false;
+                ++phase;
+            }
         }
     }
     // one verdict for the whole CTA: the loads below are warp-collective and the row groups meet on
@@ -496,29 +528,89 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
         }
         return c;
     };
-    // the row group's four warps meet on named barrier 1 + rg (128 threads)
     const bool search = ok && want > 0 && want < n;  // uniform over the row group
-    uint32_t tau = 0u;
-    bool exact = false;
-    if (search) {
-        bool done = false;
-        int step = 0;
-        for (int b = 31; b >= 0; --b, ++step) {
-            const uint32_t cand = tau | (1u << b);
-            const int part = count_ge(key_value(cand));
-            int *cs = cnt_sm + (step & 1) * 512;
-            cs[cg * 128 + r] = part;
-            named_barrier(1 + rg, 128);
-            const int tot = cs[r] + cs[128 + r] + cs[256 + r] + cs[384 + r];
-            if (!done && tot >= want) {
-                tau = cand;
-                if (tot == want) exact = done = true;
+    float ft = 0.f;     // threshold: the want-th largest score of the row
+    bool exact = false;  // exactly want scores at or above ft (otherwise: above ft, then ties lowest first)
+    if (k - 1 <= kSelList) {
+        // Each thread keeps the kSelList largest of its candidates in registers (a descending list,
+        // each candidate passed down a compare-exchange chain: branch-free, no barrier); thread cg = 0
+        // of each row then merges the four threads' lists in shared memory up to the want-th value.
+        float lst[kSelList];
+#pragma unroll
+        for (int q = 0; q < kSelList; ++q) lst[q] = -INFINITY;
+        auto insert = [&](float v) {
+            v = (v == v) ? v : -INFINITY;  // non-candidates (NaN) never enter
+#pragma unroll
+            for (int q = 0; q < kSelList; ++q) {
+                const float hi = fmaxf(lst[q], v);
+                v = fminf(lst[q], v);
+                lst[q] = hi;
             }
-            if (__all_sync(0xffffffffu, done)) break;  // the same rows and counts in all four warps
+        };
+        if (search) {
+            if (mych > 0) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) insert(x[0][e]);
+            }
+            if (mych > 1) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) insert(x[1][e]);
+            }
+            float4 *dst = reinterpret_cast<float4 *>(list_sm + (cg * 128 + r) * kSelList);
+#pragma unroll
+            for (int q = 0; q < kSelList / 4; ++q)
+                dst[q] = make_float4(lst[4 * q], lst[4 * q + 1], lst[4 * q + 2], lst[4 * q + 3]);
         }
+        if (search) named_barrier(1 + rg, 128);
+        if (search && cg == 0) {
+            const float *l0 = list_sm + r * kSelList, *l1 = l0 + 128 * kSelList, *l2 = l1 + 128 * kSelList,
+                        *l3 = l2 + 128 * kSelList;
+            int p0 = 0, p1 = 0, p2 = 0, p3 = 0;
+            float h0 = l0[0], h1 = l1[0], h2 = l2[0], h3 = l3[0], t = -INFINITY;
+            for (int q = 0; q < want; ++q) {
+                const float m01 = fmaxf(h0, h1), m23 = fmaxf(h2, h3);
+                t = fmaxf(m01, m23);
+                if (h0 == t) {
+                    ++p0;
+                    h0 = p0 < kSelList ? l0[p0] : -INFINITY;
+                } else if (h1 == t) {
+                    ++p1;
+                    h1 = p1 < kSelList ? l1[p1] : -INFINITY;
+                } else if (h2 == t) {
+                    ++p2;
+                    h2 = p2 < kSelList ? l2[p2] : -INFINITY;
+                } else {
+                    ++p3;
+                    h3 = p3 < kSelList ? l3[p3] : -INFINITY;
+                }
+            }
+            thr_sm[r] = t;
+        }
+        if (search) named_barrier(1 + rg, 128);
+        if (search) ft = thr_sm[r];
+    } else {
+        // the row group's four warps meet on named barrier 1 + rg (128 threads)
+        uint32_t tau = 0u;
+        if (search) {
+            bool done = false;
+            int step = 0;
+            for (int b = 31; b >= 0; --b, ++step) {
+                const uint32_t cand = tau | (1u << b);
+                const int part = count_ge(key_value(cand));
+                int *cs = cnt_sm + (step & 1) * 512;
+                cs[cg * 128 + r] = part;
+                named_barrier(1 + rg, 128);
+                const int tot = cs[r] + cs[128 + r] + cs[256 + r] + cs[384 + r];
+                if (!done && tot >= want) {
+                    tau = cand;
+                    if (tot == want) exact = done = true;
+                }
+                if (__all_sync(0xffffffffu, done)) break;  // the same rows and counts in all four warps
+            }
+        }
+        ft = key_value(tau);
     }
-    // chosen columns of this warp's chunks: above tau (at or above when exact), and the ties
-    const float ft = key_value(tau);
+    // chosen columns of this warp's chunks: above ft (at or above when exact), and the ties
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
         const int c = cg + 4 * i;
