@@ -39,9 +39,10 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse-attn fwd+bwd TFLOP/s & tokens/s at 32K ctx; % of bf16 tensor peak"
 WORKLOAD = "long"
 K_SEL = 16
-# DRAM bytes (read + write) of one attn_bwd_kernel launch of the full stream on the 4-head case of the
-# 32K workload, from an ncu capture of the current kernel; None until one exists.
-FULL_BWD_DRAM_BYTES_H4 = None
+# DRAM bytes (read + write) per head of one attn_bwd_kernel launch of the full stream at the 32K
+# workload: ncu dram__bytes_read.sum + dram__bytes_write.sum of the 8-head launch (509,917,696 +
+# 413,089,536 B) divided by 8.  Set to None whenever the kernel changes until it is captured again.
+FULL_BWD_DRAM_BYTES_PER_HEAD = 923007232 / 8
 
 
 def flops(B, H, T, d, s, k):
@@ -502,10 +503,10 @@ def ours(args, rank, world, local_rank):
     full_ms = op_ms["full_fwd"] + op_ms["full_bwd"]
     op_flops = {"full_fwd": ff, "full_bwd": fb, "sparse_fwd": sf, "sparse_bwd": sb}
     # Dominant call of the step: the full-attention backward.  DRAM bytes per launch of its kernel from
-    # one ncu capture of this build on the 4-head case of the same workload (heads are independent units
-    # of the grid, so the traffic scales by 32/4 to the benchmarked launch); None when no capture of the
-    # current kernel exists.
-    traffic = FULL_BWD_DRAM_BYTES_H4 * (wl.H / 4) if FULL_BWD_DRAM_BYTES_H4 else None
+    # one ncu capture of this build on an 8-head case of the same workload (heads are independent units
+    # of the grid, so the traffic scales by the head count to the benchmarked launch); None when no
+    # capture of the current kernel exists.
+    traffic = FULL_BWD_DRAM_BYTES_PER_HEAD * wl.H if FULL_BWD_DRAM_BYTES_PER_HEAD else None
     roof = {"kernel": "ssa_full_attn_bwd call (attn_bwd_kernel, prep, dQ conversion)", "bound": "tensor",
             "achieved": fb / (op_ms["full_bwd"] / 1e3) / 1e12, "peak": peak_sust,
             "unit": "TFLOP/s", "traffic": traffic, "traffic_unit": "DRAM bytes per launch (ncu)",
