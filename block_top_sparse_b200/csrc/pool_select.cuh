@@ -479,7 +479,7 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
             }
         }
     }
-    // one verdict for the whole CTA: the loads below are warp-collective and the row groups meet on
+    // one decision for the whole CTA: the loads below are warp-collective and the row groups meet on
     // named barriers, so every thread must take the same branch
     ok = __syncthreads_and(ok ? 1 : 0) != 0;
     tc_fence_after();
