@@ -543,7 +543,7 @@ def ours(args, rank, world, local_rank):
                 "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in out_host.values()),
                 "path": "pool, select, index, sparse fwd, sparse bwd with Q, K, V, dO copied in and O, dQ, dK, dV "
                         "copied out every step"},
-        "gpu_launches": args.steps * (ops.SSAStep.KERNELS_FWD + ops.SSAStep.KERNELS_BWD),
+        "gpu_launches": args.steps * (ops.SSAStep.KERNELS_FWD + steps[0].kernels_bwd()),
         "clocks": clocks,
     }
     if not args.no_cpu_baseline:

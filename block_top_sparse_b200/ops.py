@@ -150,9 +150,16 @@ class SSAStep:
         shared = torch.empty(need, dtype=torch.uint8, device=device) if need else None
         self.ws[L.SSA_OP_SPARSE_FWD] = self.ws[L.SSA_OP_SPARSE_BWD] = shared
 
-    # Number of libssa kernel launches per forward / backward (bf16, d = 128).
-    KERNELS_FWD = 1 + 1 + 3 + 1 + (1 + 1) + 2  # pool, select, index x3, full, sparse(fwd, merge), align x2
-    KERNELS_BWD = 1 + (1 + 1 + 1) + (1 + 1 + 1)  # align, full(prep, bwd, dq), sparse(prep, bwd, dq)
+    # Number of libssa kernel launches per forward (bf16, d = 128): pool, select, index (count, scan, fill,
+    # launch order), full, sparse (kernel, merge), align (partial, final).
+    KERNELS_FWD = 1 + 1 + 4 + 1 + (1 + 1) + 2
+
+    def kernels_bwd(self) -> int:
+        """libssa kernel launches per backward (bf16, d = 128): align, then per stream the prep and the
+        attention kernel, plus the dQ conversion unless the gradients are fp32; with rotary positions the
+        two passes that turn dQ and dK back."""
+        per_stream = 2 if self.grad_fp32 else 3
+        return 1 + 2 * per_stream + (2 if self.rope else 0)
 
     def _rotated(self, Q, K, stream=None):
         if not self.rope:
