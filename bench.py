@@ -318,27 +318,13 @@ def extras(args):
     del st, dev, Q, K, V
     torch.cuda.empty_cache()
     # ---- sparse decoding: 64 sequences, caches of 32768 tokens, new tokens at random lengths
-    Bd, Hd, Hk, Td = 64, 32, 8, 32768
-    ddims = L.make_dims(Bd, Hd, Td, d, s, k, Hkv=Hk)
-    rng = np.random.default_rng(5)
-    lens = torch.from_numpy(rng.integers(Td // 2, Td, size=Bd).astype(np.int32)).cuda()
-    Kc = torch.randn((Bd, Hk, Td, d), device="cuda").mul_(d ** -0.25).to(torch.bfloat16)
-    Vc = torch.randn((Bd, Hk, Td, d), device="cuda").mul_(d ** -0.25).to(torch.bfloat16)
-    q = torch.randn((Bd, Hd, d), device="cuda").mul_(d ** -0.25).to(torch.bfloat16)
-    Kbar = ops.block_pool(ddims, Kc)
-    idx = torch.empty((Bd, Hk, k), dtype=torch.int32, device="cuda")
-    o = torch.empty((Bd, Hd, d), dtype=torch.bfloat16, device="cuda")
-    lse = torch.empty((Bd, Hd), dtype=torch.float32, device="cuda")
-    ws = ops._ws(ddims, L.SSA_OP_DECODE, "cuda")
-    ms = _time(lambda: L.ssa_sparse_decode(ddims, lens, q, Kc, Vc, Kbar, idx, o, lse, ws), args.steps, args.warmup)
-    Ls = lens.cpu().numpy().astype(np.int64)
-    # bytes a decode step must read: pooled keys of the complete blocks and the selected blocks' keys and values
-    nbytes = float(sum(Hk * ((L_ // s) * d * 4 + min(k * s, L_ + 1) * d * 2 * 2) for L_ in Ls))
-    print(json.dumps({"extra": "sparse decode", "sequences": Bd, "H": Hd, "Hkv": Hk, "cache": Td, "k": k,
-                      "ms": ms, "tokens_per_s": Bd / (ms / 1e3), "gbs": nbytes / (ms / 1e3) / 1e9,
-                      "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / hbm, "device_error": L.ssa_get_device_error()}),
-          flush=True)
-    del Kc, Vc, Kbar
+    Bd = 64
+    call, nbytes, wl = decode_workload(Bd, d, s, k)
+    ms = _time(call, args.steps, args.warmup)
+    print(json.dumps({"extra": "sparse decode", **wl, "ms": ms, "tokens_per_s": Bd / (ms / 1e3),
+                      "gbs": nbytes / (ms / 1e3) / 1e9, "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / hbm,
+                      "device_error": L.ssa_get_device_error()}), flush=True)
+    del call
     torch.cuda.empty_cache()
     # ---- rotary positions on Q of the 32K workload (one read and one write)
     X = torch.randn((B, H, T, d), device="cuda").to(torch.bfloat16)
@@ -560,6 +546,34 @@ def ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def decode_workload(Bd, d=128, s=128, k=16, Hd=32, Hk=8, Td=32768, seed=5):
+    """Sparse decoding over key/value caches: Bd sequences with caches of Td tokens (Hk key/value heads, Hd
+    query heads), the new token at a random length in [Td/2, Td).  Returns the decode call, the bytes it must
+    read (the pooled keys of the complete blocks and the selected blocks' keys and values) and the workload's
+    description."""
+    import torch
+    from block_top_sparse_b200 import _lib as L
+    from block_top_sparse_b200 import ops
+
+    ddims = L.make_dims(Bd, Hd, Td, d, s, k, Hkv=Hk)
+    rng = np.random.default_rng(seed)
+    lens = torch.from_numpy(rng.integers(Td // 2, Td, size=Bd).astype(np.int32)).cuda()
+    Kc = torch.randn((Bd, Hk, Td, d), device="cuda").mul_(d ** -0.25).to(torch.bfloat16)
+    Vc = torch.randn((Bd, Hk, Td, d), device="cuda").mul_(d ** -0.25).to(torch.bfloat16)
+    q = torch.randn((Bd, Hd, d), device="cuda").mul_(d ** -0.25).to(torch.bfloat16)
+    Kbar = ops.block_pool(ddims, Kc)
+    idx = torch.empty((Bd, Hk, k), dtype=torch.int32, device="cuda")
+    o = torch.empty((Bd, Hd, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((Bd, Hd), dtype=torch.float32, device="cuda")
+    ws = ops._ws(ddims, L.SSA_OP_DECODE, "cuda")
+    Ls = lens.cpu().numpy().astype(np.int64)
+    nbytes = float(sum(Hk * ((L_ // s) * d * 4 + min(k * s, L_ + 1) * d * 2 * 2) for L_ in Ls))
+
+    def call():
+        L.ssa_sparse_decode(ddims, lens, q, Kc, Vc, Kbar, idx, o, lse, ws)
+    return call, nbytes, {"sequences": Bd, "H": Hd, "Hkv": Hk, "cache": Td, "k": k}
+
+
 def single_op(args):
     """One library call at a chosen size, timed with CUDA events (for profiling runs)."""
     import torch
@@ -567,6 +581,12 @@ def single_op(args):
     from block_top_sparse_b200 import build, inputs, ops
 
     build.build()
+    if args.op == "decode":  # args.sequences sequences over caches of 32768 tokens (8 key/value heads, G = 4)
+        call, nbytes, wl = decode_workload(args.sequences)
+        ms = _time(call, args.steps, args.warmup)
+        print(json.dumps({"op": "decode", **wl, "ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9,
+                          "device_error": L.ssa_get_device_error()}), flush=True)
+        return
     wl = inputs.WORKLOADS[args.workload]
     g = inputs.generate(wl, H=args.H or wl.H, T=args.T or wl.T, with_dO=True)
     w = g["wl"]
@@ -626,12 +646,13 @@ def main():
     ap.add_argument("--union", action="store_true",
                     help="size of the union of a 128-query tile's selected blocks, per workload (one line each)")
     ap.add_argument("--op", default=None,
-                    choices=["pool", "select", "index", "full_fwd", "sparse_fwd", "full_bwd", "sparse_bwd"],
+                    choices=["pool", "select", "index", "full_fwd", "sparse_fwd", "full_bwd", "sparse_bwd", "decode"],
                     help="time one library call instead of the whole step (profiling)")
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--T", type=int, default=0)
     ap.add_argument("--H", type=int, default=0)
     ap.add_argument("--k", type=int, default=0)
+    ap.add_argument("--sequences", type=int, default=64, help="sequences of --op decode")
     args = ap.parse_args()
     if args.sweep:
         sweep(args)

@@ -656,6 +656,18 @@ ssa_status_t noalloc_scratch(void **out) {
     *out = p;
     return SSA_OK;
 }
+
+// One slot's block of the decode against the G query heads, for G padded to GP.
+template <int GP>
+bool launch_decode_attend(const Shape &S, cudaStream_t st, const int32_t *cache_len, const void *q, const void *Kc,
+                          const void *Vc, const int32_t *idx, float *opart, float *lsepart) {
+    const size_t sm = dec_attend_smem(S.s, GP);
+    if (!set_smem(decode_attend_kernel<GP>, sm)) return false;
+    decode_attend_kernel<GP><<<dim3(static_cast<unsigned>(S.BHk), S.k), kDecThreads, sm, st>>>(
+        cache_len, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)Kc, (const __nv_bfloat16 *)Vc, idx, opart, lsepart,
+        S.Hk, S.G, S.T, S.s, S.k, S.scale);
+    return true;
+}
 }  // namespace
 
 extern "C" {
@@ -683,19 +695,35 @@ ssa_status_t ssa_sparse_decode(const ssa_dims_t *dims, const int32_t *cache_len,
     if (e != SSA_OK) return e;
     if (!cache_len || !q || !Kcache || !Vcache || !Kbar_cache || !idx || !o || !lse) return SSA_ERR_INVALID_ARG;
     if (S.dtype != SSA_DT_BF16 || S.d != 128 || S.nb > kDecMaxBlocks || S.G > kDecMaxGroup) return SSA_ERR_UNSUPPORTED;
+    // the selected blocks are bulk-copied and the query rows read in 16-byte units: 16-byte aligned bases
+    if ((reinterpret_cast<uintptr_t>(Kcache) | reinterpret_cast<uintptr_t>(Vcache) | reinterpret_cast<uintptr_t>(q)) &
+        15u)
+        return SSA_ERR_INVALID_ARG;
     if ((e = check_ws(S, SSA_OP_DECODE, ws, ws_bytes)) != SSA_OK) return e;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     float *opart = static_cast<float *>(ws);
     float *lsepart = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + align_up(S.BH * S.k * S.d * 4));
     const unsigned bhk = static_cast<unsigned>(S.BHk);
     const size_t sm = (128 + (S.nb > 256 ? S.nb : 256)) * sizeof(float);
-    decode_select_kernel<<<bhk, kDecThreads, sm, st>>>(cache_len, (const __nv_bfloat16 *)q,
-                                                       (const __nv_bfloat16 *)Kcache, Kbar_cache, idx, S.Hk, S.G, S.T,
-                                                       S.s, S.k, S.nb);
-    decode_attend_kernel<<<dim3(bhk, S.k), kDecThreads, 0, st>>>(cache_len, (const __nv_bfloat16 *)q,
-                                                                (const __nv_bfloat16 *)Kcache,
-                                                                (const __nv_bfloat16 *)Vcache, idx, opart, lsepart,
-                                                                S.Hk, S.G, S.T, S.s, S.k, S.scale);
+    // the warp search holds ceil(nb / 32) scores per lane (8, 16 or 32)
+    auto sel = S.nb <= 256 ? decode_select_kernel<8> : S.nb <= 512 ? decode_select_kernel<16> : decode_select_kernel<32>;
+    sel<<<bhk, kDecThreads, sm, st>>>(cache_len, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)Kcache, Kbar_cache,
+                                      idx, S.Hk, S.G, S.T, S.s, S.k, S.nb);
+    if (S.s == 128) {  // tensor-core attend: blocks brought in by TMA, both products on tcgen05
+        CUtensorMap tmK, tmV;
+        if (!make_tmap(&tmK, Kcache, S.krows, 128) || !make_tmap(&tmV, Vcache, S.krows, 128)) return SSA_ERR_CUDA;
+        if (!set_smem(decode_attend_tc_kernel, DecTcSmem::kTotal)) return SSA_ERR_CUDA;
+        decode_attend_tc_kernel<<<dim3(bhk, S.k), 128, DecTcSmem::kTotal, st>>>(
+            tmK, tmV, cache_len, (const __nv_bfloat16 *)q, idx, opart, lsepart, S.Hk, S.G, S.T, S.k,
+            S.scale * 1.4426950408889634f);
+    } else {  // blocks of 64 keys: CUDA-core attend, the group padded to a power of two
+        auto launch = S.G <= 1   ? launch_decode_attend<1>
+                      : S.G <= 2 ? launch_decode_attend<2>
+                      : S.G <= 4 ? launch_decode_attend<4>
+                      : S.G <= 8 ? launch_decode_attend<8>
+                                 : launch_decode_attend<16>;
+        if (!launch(S, st, cache_len, q, Kcache, Vcache, idx, opart, lsepart)) return SSA_ERR_CUDA;
+    }
     const unsigned rows = static_cast<unsigned>(S.BH);
     decode_combine_kernel<<<(rows + kDecThreads / 32 - 1) / (kDecThreads / 32), kDecThreads, 0, st>>>(
         opart, lsepart, (__nv_bfloat16 *)o, lse, static_cast<int>(rows), S.k);

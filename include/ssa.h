@@ -305,6 +305,8 @@ ssa_status_t ssa_get_device_error(ssa_stream_t stream);
  *   cache_len   in   [B] int32, device
  *   q           in   [B, H, d] bf16
  *   Kcache, Vcache in [B, Hkv, T, d] bf16
+ *               q, Kcache and Vcache need 16-byte aligned base addresses (the selected
+ *               blocks are bulk-copied; SSA_ERR_INVALID_ARG otherwise)
  *   Kbar_cache  in/out [B, Hkv, T/s, d] fp32: rows j < b(L) are read, row b(L)
  *               is written when the token completes it
  *   idx         out  [B, Hkv, k] int32

@@ -151,6 +151,10 @@ def test_null_pointers_and_workspace(lib):
     assert _call("ssa_align_loss_bwd", d, p, p, 0, ctypes.c_float(1.0), ctypes.c_float(1), ctypes.c_float(1), None,
                  p, p, 0, None) == L.SSA_ERR_INVALID_ARG
     assert _call("ssa_dropped_mass", d, p, None, p, None) == L.SSA_ERR_INVALID_ARG
+    # the decode bulk-copies cache blocks: a cache base off a 16-byte boundary is refused
+    odd = ctypes.c_void_p(24)
+    assert _call("ssa_sparse_decode", d, p, p, odd, p, p, p, p, p, p, 1 << 40, None) == L.SSA_ERR_INVALID_ARG
+    assert _call("ssa_sparse_decode", d, p, p, p, odd, p, p, p, p, p, 1 << 40, None) == L.SSA_ERR_INVALID_ARG
 
 
 def test_binding_raises_on_error(lib):

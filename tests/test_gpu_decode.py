@@ -25,10 +25,14 @@ def _build():
     ora.build()
 
 
-@pytest.mark.parametrize("H,Hkv,s,k", [(2, 2, 128, 4), (8, 2, 64, 6)])
-def test_decode_matches_oracle(H, Hkv, s, k):
-    B, T, d = 4, 2048, 128
-    lens = np.array([0, 700, 2047, 3 * s - 1], dtype=np.int32)  # the last one completes block 2
+# groups of 1, 2, 4, 8 and 16 query heads per key/value head; blocks of 128 and 64 keys; caches of 16, 32,
+# 512 and 1024 blocks (the selection's warp search holds 8, 16 or 32 scores per lane)
+@pytest.mark.parametrize("H,Hkv,s,k,T", [(2, 2, 128, 4, 2048), (4, 2, 128, 5, 2048), (8, 2, 64, 6, 2048),
+                                         (16, 2, 64, 4, 2048), (16, 1, 128, 3, 2048), (2, 1, 64, 8, 32768),
+                                         (2, 1, 64, 8, 65536)])
+def test_decode_matches_oracle(H, Hkv, s, k, T):
+    B, d = 4, 128
+    lens = np.array([0, 700, T - 1, 3 * s - 1], dtype=np.int32)  # the last one completes block 2
     g = inputs.group_kv(inputs.generate(inputs.WORKLOADS["long"], B=B, H=H, T=T), Hkv)
     Kc, Vc = to_device(g["K"], "bf16"), to_device(g["V"], "bf16")
     qraw = inputs.random_tensor((B, H, d), "bf16", seed=21, std=d ** -0.25)
@@ -36,6 +40,13 @@ def test_decode_matches_oracle(H, Hkv, s, k):
     dims = L.make_dims(B, H, T, d, s, k, Hkv=Hkv)
     # pooled-key cache: every block pooled once, then the rows the call may write set to a marker
     Kbar = ops.block_pool(dims, Kc)
+    # cache rows past each sequence's new token hold NaN on the device (a cache's unwritten rows may hold
+    # anything): the current block's keys and values past L must not reach the output, not even with
+    # weight 0; the oracle reads the clean rows up to L only
+    Kc4, Vc4 = Kc.view(B, Hkv, T, d), Vc.view(B, Hkv, T, d)
+    for b, Lb in enumerate(lens):
+        Kc4[b, :, Lb + 1:] = float("nan")
+        Vc4[b, :, Lb + 1:] = float("nan")
     marker = -7.0
     for b, Lb in enumerate(lens):
         Kbar[b, :, Lb // s] = marker
