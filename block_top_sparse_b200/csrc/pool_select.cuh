@@ -362,6 +362,46 @@ __device__ __forceinline__ float key_value(uint32_t key) {
     return -INFINITY;
 }
 
+// Compare-exchange: a keeps the larger value, b the smaller.
+__device__ __forceinline__ void ce_desc(float &a, float &b) {
+    const float hi = fmaxf(a, b);
+    b = fminf(a, b);
+    a = hi;
+}
+
+// Sorts 16 values descending: the bitonic network (sorted runs of 2, 4, 8, 16, alternately descending
+// and ascending until the last merge), 10 stages of 8 compare-exchanges.
+__device__ __forceinline__ void sort16_desc(float (&a)[16]) {
+#pragma unroll
+    for (int size = 2; size <= 16; size <<= 1)
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int j = i ^ stride;
+                if (j > i) {
+                    if ((i & size) == 0)
+                        ce_desc(a[i], a[j]);
+                    else
+                        ce_desc(a[j], a[i]);
+                }
+            }
+}
+
+// a <- the 16 largest of a and b, descending (both descending): max(a[i], b[15 - i]) is a bitonic
+// sequence holding them, which one bitonic merge (4 stages of 8 compare-exchanges) sorts.
+__device__ __forceinline__ void merge_top16_desc(float (&a)[16], const float (&b)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a[i] = fmaxf(a[i], b[15 - i]);
+#pragma unroll
+    for (int stride = 8; stride > 0; stride >>= 1)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int j = i ^ stride;
+            if (j > i) ce_desc(a[i], a[j]);
+        }
+}
+
 __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_bfloat16 *__restrict__ Q,
                                                            const float *__restrict__ Kbar, int32_t *__restrict__ idx,
                                                            int T_len, int s, int k, int nb, int G) {
@@ -532,29 +572,36 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
     float ft = 0.f;     // threshold: the want-th largest score of the row
     bool exact = false;  // exactly want scores at or above ft (otherwise: above ft, then ties lowest first)
     if (k - 1 <= kSelList) {
-        // Each thread keeps the kSelList largest of its candidates in registers (a descending list,
-        // each candidate passed down a compare-exchange chain: branch-free, no barrier); thread cg = 0
-        // of each row then merges the four threads' lists in shared memory up to the want-th value.
+        // Each thread forms the kSelList largest of its candidates in registers (a descending list):
+        // groups of 16 sorted by a bitonic network, each merged into the running list by keeping the
+        // larger of a[i] and b[15-i] (a bitonic sequence holding the 16 largest) and one bitonic merge
+        // (880 min/max per 64 candidates, against 2,048 for passing each candidate down a 16-long
+        // compare-exchange chain); thread cg = 0 of each row then merges the four threads' lists in
+        // shared memory up to the want-th value.
         float lst[kSelList];
-#pragma unroll
-        for (int q = 0; q < kSelList; ++q) lst[q] = -INFINITY;
-        auto insert = [&](float v) {
-            v = (v == v) ? v : -INFINITY;  // non-candidates (NaN) never enter
-#pragma unroll
-            for (int q = 0; q < kSelList; ++q) {
-                const float hi = fmaxf(lst[q], v);
-                v = fminf(lst[q], v);
-                lst[q] = hi;
-            }
-        };
         if (search) {
-            if (mych > 0) {
+            float g[kSelList];
+            auto take = [&](const float (&src)[32], int half, float (&dst)[kSelList]) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) insert(x[0][e]);
+                for (int e = 0; e < kSelList; ++e) {
+                    const float v = src[half * kSelList + e];
+                    dst[e] = (v == v) ? v : -INFINITY;  // non-candidates (NaN) never enter
+                }
+                sort16_desc(dst);
+            };
+            if (mych > 0) {
+                take(x[0], 0, lst);
+                take(x[0], 1, g);
+                merge_top16_desc(lst, g);
+            } else {
+#pragma unroll
+                for (int q = 0; q < kSelList; ++q) lst[q] = -INFINITY;
             }
             if (mych > 1) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) insert(x[1][e]);
+                take(x[1], 0, g);
+                merge_top16_desc(lst, g);
+                take(x[1], 1, g);
+                merge_top16_desc(lst, g);
             }
             float4 *dst = reinterpret_cast<float4 *>(list_sm + (cg * 128 + r) * kSelList);
 #pragma unroll
