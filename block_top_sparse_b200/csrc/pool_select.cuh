@@ -455,12 +455,25 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
     int phase = 0;  // completed MMA batches (bar_mma phases)
     // Kbar rows 64gi .. 64gi+63 -> hi / mid / lo tiles (K-major, swizzled) of buffer sBb; rows >= nbc are
     // zero.  Lane c4 of a warp takes dims 4c4 .. 4c4+3 of one row: two 128-byte row halves per store.
-    auto convert = [&](int gi, uint32_t sBb) {
+    // The split of a group of 64 pooled keys: every warp takes 4 rows, one float4 per lane.  The rows are
+    // loaded into registers first (load_rows), then split and stored (split_store); the stores are asm with
+    // a memory clobber, so a load issued after one would wait for it: one L2 round trip per row.
+    constexpr int kRowsPerWarp = 64 / (kSelTcThreads / 32);
+    static_assert(64 % (kSelTcThreads / 32) == 0, "64 pooled keys per group over the CTA's warps");
+    auto load_rows = [&](int gi, float4 (&vr)[kRowsPerWarp]) {
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i) {
+            const int j = 64 * gi + warp + i * (kSelTcThreads / 32);
+            vr[i] = j < nbc ? __ldg(reinterpret_cast<const float4 *>(Kbar + (static_cast<size_t>(bh) * nb + j) * 128) + lane)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    auto split_store = [&](const float4 (&vr)[kRowsPerWarp], uint32_t sBb) {
         const int c4 = lane;
-        for (int jj = warp; jj < 64; jj += kSelTcThreads / 32) {
-            const int j = 64 * gi + jj;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (j < nbc) v = __ldg(reinterpret_cast<const float4 *>(Kbar + (static_cast<size_t>(bh) * nb + j) * 128) + c4);
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i) {
+            const int jj = warp + i * (kSelTcThreads / 32);
+            const float4 v = vr[i];
             const uint32_t h01 = pack_bf16x2(v.x, v.y), h23 = pack_bf16x2(v.z, v.w);
             const float r0 = v.x - __uint_as_float(h01 << 16), r1 = v.y - __uint_as_float(h01 & 0xFFFF0000u);
             const float r2 = v.z - __uint_as_float(h23 << 16), r3 = v.w - __uint_as_float(h23 & 0xFFFF0000u);
@@ -492,8 +505,13 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
     if (G == 1) {
         // the split of group gi is written while the MMAs of group gi-1 run (two buffers: buffer gi & 1
         // was last read by the MMAs of group gi-2, which completed before group gi-1 was issued)
+        // the next group's rows are loaded right after this group's split is stored: in flight while the
+        // previous group's MMAs complete and this group's are issued
+        float4 vr[kRowsPerWarp];
+        if (ngroups > 0) load_rows(0, vr);
         for (int gi = 0; gi < ngroups && ok; ++gi) {
-            convert(gi, sB + (gi & 1) * L::kBBuf);
+            split_store(vr, sB + (gi & 1) * L::kBBuf);
+            if (gi + 1 < ngroups) load_rows(gi + 1, vr);
             if (gi > 0) {
                 if (!mbar_wait(bar_mma, phase & 1, abort_flag, 0x501)) ok = false;
                 ++phase;
@@ -507,7 +525,11 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
         }
     } else {
         for (int gi = 0; gi < ngroups && ok; ++gi) {
-            convert(gi, sB);
+            {
+                float4 vr[kRowsPerWarp];
+                load_rows(gi, vr);
+                split_store(vr, sB);
+            }
             // with grouped query heads the group's tiles are added one after another into the same scores
             for (int hi = 0; hi < G && ok; ++hi) {
                 load_q(hi);  // the previous batch's MMAs have read the tile (waited below)
@@ -663,39 +685,57 @@ __global__ void __launch_bounds__(kSelTcThreads, 1) select_tc_kernel(const __nv_
         const int c = cg + 4 * i;
         if (c < nch) {
             uint32_t gm = 0u, em = 0u;
+            if (!search) {  // every candidate (non-candidates are NaN)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const float v = x[i][e];
-                const bool above = search ? (exact ? v >= ft : v > ft) : (v == v);  // no search: every candidate
-                gm |= (above ? 1u : 0u) << e;
-                em |= ((search && !exact && v == ft) ? 1u : 0u) << e;
+                for (int e = 0; e < 32; ++e) gm |= (x[i][e] == x[i][e] ? 1u : 0u) << e;
+            } else if (exact) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) gm |= (x[i][e] >= ft ? 1u : 0u) << e;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    gm |= (x[i][e] > ft ? 1u : 0u) << e;
+                    em |= (x[i][e] == ft ? 1u : 0u) << e;
+                }
             }
             gt_sm[c * 128 + r] = gm;
             eq_sm[c * 128 + r] = em;
         }
     }
     __syncthreads();
-    if (cg == 0 && valid_row && ok) {
-        // need_eq: keys equal to tau taken in ascending block order until want are chosen
-        int above = 0;
-        for (int c = 0; c < nch; ++c) above += __popc(gt_sm[c * 128 + r]);
-        int need = search ? want - above : 0;
+    if (valid_row && ok) {
+        // Each of the row's four threads writes the chosen columns of its own chunks, ascending: a chunk's
+        // first position is the count of columns above the threshold in the chunks before it plus the ties
+        // taken there (ties go lowest column first until want are chosen).
+        int above = 0, ab[2] = {0, 0}, eb[2] = {0, 0};
+        for (int c = 0; c < nch; ++c) {
+            const int pa = __popc(gt_sm[c * 128 + r]), pe = __popc(eq_sm[c * 128 + r]);
+            above += pa;
+            if (c < cg) ab[0] += pa, eb[0] += pe;
+            if (c < cg + 4) ab[1] += pa, eb[1] += pe;
+        }
+        const int need = search ? want - above : 0;  // ties to take
         int32_t *out = idx + (head_rows + t) * k;
-        int pos = 0;
-        for (int c = 0; c < nch && pos < want; ++c) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int c = cg + 4 * i;
+            if (c >= nch) continue;
             uint32_t m = gt_sm[c * 128 + r], e = eq_sm[c * 128 + r];
-            while (e != 0u && need > 0) {
+            const int ties_before = min(need, eb[i]);
+            for (int take = need - ties_before; take > 0 && e != 0u; --take) {
                 m |= e & (~e + 1u);  // lowest equal column
                 e &= e - 1u;
-                --need;
             }
+            int pos = ab[i] + ties_before;
             while (m != 0u && pos < want) {
                 out[pos++] = 32 * c + __ffs(m) - 1;
                 m &= m - 1u;
             }
         }
-        out[pos++] = bt;
-        for (; pos < k; ++pos) out[pos] = -1;
+        if (cg == 0) {
+            out[want] = bt;
+            for (int pos = want + 1; pos < k; ++pos) out[pos] = -1;
+        }
     }
 }
 
