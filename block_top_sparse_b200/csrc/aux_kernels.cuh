@@ -398,6 +398,46 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const T *__restrict__ dO,
     if (lane == 0) Dvec[row] = acc;
 }
 
+// The same for bf16 rows of d = 128 (the tensor-core path): a warp takes 4 consecutive rows, lane l the
+// elements 4l .. 4l+3 of each (8-byte loads), so that the rows' twelve loads are in flight together; the fp32
+// accumulator rows are zeroed with 16-byte stores.
+constexpr int kPrepRows = 4;  // rows per warp
+__global__ void __launch_bounds__(256) bwd_prep_bf16_kernel(const __nv_bfloat16 *__restrict__ dO,
+                                                            const __nv_bfloat16 *__restrict__ O,
+                                                            const __nv_bfloat16 *__restrict__ O_lo,
+                                                            float *__restrict__ Dvec, float *__restrict__ dQacc,
+                                                            size_t rows) {
+    const size_t row0 = ((static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5) * kPrepRows;
+    const int lane = threadIdx.x & 31;
+    uint2 g[kPrepRows], o[kPrepRows], lo[kPrepRows];
+#pragma unroll
+    for (int i = 0; i < kPrepRows; ++i) {
+        const size_t row = row0 + i;
+        const bool in = row < rows;
+        g[i] = in ? __ldg(reinterpret_cast<const uint2 *>(dO + row * 128) + lane) : make_uint2(0u, 0u);
+        o[i] = in ? __ldg(reinterpret_cast<const uint2 *>(O + row * 128) + lane) : make_uint2(0u, 0u);
+        lo[i] = (in && O_lo) ? __ldg(reinterpret_cast<const uint2 *>(O_lo + row * 128) + lane) : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < kPrepRows; ++i) {
+        const uint32_t gw[2] = {g[i].x, g[i].y}, ow[2] = {o[i].x, o[i].y}, lw[2] = {lo[i].x, lo[i].y};
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            acc += __uint_as_float(gw[w] << 16) * (__uint_as_float(ow[w] << 16) + __uint_as_float(lw[w] << 16));
+            acc += __uint_as_float(gw[w] & 0xFFFF0000u) *
+                   (__uint_as_float(ow[w] & 0xFFFF0000u) + __uint_as_float(lw[w] & 0xFFFF0000u));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        const size_t row = row0 + i;
+        if (row < rows) {
+            if (lane == 0) Dvec[row] = acc;
+            if (dQacc) reinterpret_cast<float4 *>(dQacc + row * 128)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+}
+
 // out = (accumulate ? out : 0) + acc, rounded once to T.
 template <typename T>
 __global__ void __launch_bounds__(256) acc_to_out_kernel(const float *__restrict__ acc, T *__restrict__ out,

@@ -322,10 +322,16 @@ ssa_status_t tc_bwd(const Shape &S, const void *Q, const void *K, const void *V,
     // With fp32 gradients the caller's dQ is the accumulator itself (zeroed unless accumulating).
     const bool acc = (accumulate & SSA_BWD_ACCUMULATE) != 0, g32 = (accumulate & SSA_BWD_GRAD_FP32) != 0;
     float *dQacc = g32 ? static_cast<float *>(dQ) : reinterpret_cast<float *>(p);
-    const unsigned g = static_cast<unsigned>((S.rows + 7) / 8);
-    bwd_prep_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16 *)dO, (const __nv_bfloat16 *)O,
-                                                       (const __nv_bfloat16 *)O_lo, Dvec,
-                                                       (g32 && acc) ? nullptr : dQacc, S.rows, S.d);
+    float *zero_acc = (g32 && acc) ? nullptr : dQacc;
+    if (((reinterpret_cast<uintptr_t>(O) | reinterpret_cast<uintptr_t>(O_lo)) & 7u) == 0) {  // 8-byte row loads
+        const unsigned g = static_cast<unsigned>((S.rows + 8 * kPrepRows - 1) / (8 * kPrepRows));
+        bwd_prep_bf16_kernel<<<g, 256, 0, st>>>((const __nv_bfloat16 *)dO, (const __nv_bfloat16 *)O,
+                                                (const __nv_bfloat16 *)O_lo, Dvec, zero_acc, S.rows);
+    } else {
+        const unsigned g = static_cast<unsigned>((S.rows + 7) / 8);
+        bwd_prep_kernel<__nv_bfloat16><<<g, 256, 0, st>>>((const __nv_bfloat16 *)dO, (const __nv_bfloat16 *)O,
+                                                           (const __nv_bfloat16 *)O_lo, Dvec, zero_acc, S.rows, S.d);
+    }
     const int nkv = sparse ? S.s : 128;
     CUtensorMap tmK, tmV, tmQ, tmdO, tmdQ;
     if (!make_tmap(&tmK, K, S.krows, nkv) || !make_tmap(&tmV, V, S.krows, nkv) || !make_tmap(&tmQ, Q, S.rows, 128) ||
