@@ -25,9 +25,18 @@ __global__ void __launch_bounds__(256) index_count_kernel(const int32_t *__restr
     const int t0 = c * kIdxChunk;
     const int n = min(kIdxChunk, T - t0) * k;
     const int32_t *src = idx + (static_cast<size_t>(bh) * T + t0) * k;
-    for (int e = threadIdx.x; e < n; e += blockDim.x) {
-        const int j = __ldg(src + e);
-        if (j >= 0 && j < nb) atomicAdd(&hcount[j], 1);
+    // 16 loads in flight before their shared-memory atomics (a load after an atomic would wait for it)
+    constexpr int U = 16;
+    for (int e0 = threadIdx.x; e0 < n; e0 += U * blockDim.x) {
+        int jv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int e = e0 + u * blockDim.x;
+            jv[u] = e < n ? __ldg(src + e) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (jv[u] >= 0 && jv[u] < nb) atomicAdd(&hcount[jv[u]], 1);
     }
     __syncthreads();
     for (int j = threadIdx.x; j < nb; j += blockDim.x) cnt[(static_cast<size_t>(bh) * nch + c) * nb + j] = hcount[j];
@@ -45,12 +54,20 @@ __global__ void __launch_bounds__(1024) index_scan_kernel(int *__restrict__ cnt,
     __syncthreads();
     for (int j0 = 0; j0 < nb; j0 += blockDim.x) {
         const int j = j0 + threadIdx.x;
+        // chunk counts -> exclusive offsets within the block, 16 chunks' loads in flight at a time (a load
+        // after a store to the same array would wait for it)
+        constexpr int U = 16;
         int total = 0;
         if (j < nb) {
-            for (int c = 0; c < nch; ++c) {
-                const int v = base[static_cast<size_t>(c) * nb + j];
-                base[static_cast<size_t>(c) * nb + j] = total;
-                total += v;
+            for (int c0 = 0; c0 < nch; c0 += U) {
+                int v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) v[u] = c0 + u < nch ? base[static_cast<size_t>(c0 + u) * nb + j] : 0;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    if (c0 + u < nch) base[static_cast<size_t>(c0 + u) * nb + j] = total;
+                    total += v[u];
+                }
             }
         }
         // exclusive scan over j of the totals rounded up to whole 128-entry tiles
@@ -79,7 +96,14 @@ __global__ void __launch_bounds__(1024) index_scan_kernel(int *__restrict__ cnt,
         if (j < nb) {
             lstart[bh * nb + j] = start;
             llen[bh * nb + j] = total;
-            for (int c = 0; c < nch; ++c) base[static_cast<size_t>(c) * nb + j] += start;
+            for (int c0 = 0; c0 < nch; c0 += U) {
+                int v[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) v[u] = c0 + u < nch ? base[static_cast<size_t>(c0 + u) * nb + j] : 0;
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    if (c0 + u < nch) base[static_cast<size_t>(c0 + u) * nb + j] = v[u] + start;
+            }
         }
         __syncthreads();
         if (threadIdx.x == blockDim.x - 1) carry = start + padded;
