@@ -39,6 +39,7 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse-attn fwd+bwd TFLOP/s & tokens/s at 32K ctx; % of bf16 tensor peak"
 WORKLOAD = "long"
 K_SEL = 16
+E2E_GROUPS = 8  # head groups of the end-to-end pipeline (copy in / sparse path / copy out on three streams)
 # DRAM bytes (read + write) per head of one attn_bwd_kernel launch of the full stream at the 32K
 # workload: ncu dram__bytes_read.sum + dram__bytes_write.sum of the 8-head launch (509,917,696 +
 # 413,089,536 B) divided by 8.  Set to None whenever the kernel changes until it is captured again.
@@ -448,31 +449,75 @@ def ours(args, rank, world, local_rank):
 
     # ---- end to end, through the same calls with host buffers: each step copies Q, K, V, dO from pinned
     # host memory, runs the sparse path (pool, select, index, sparse forward, sparse backward) and copies
-    # its results O, dQ, dK, dV back to pinned host memory ----
-    out_host = {"O": torch.empty_like(host["Q"]).pin_memory()}
-    out_host.update({key: torch.empty(host["Q"].shape, dtype=torch.float32).pin_memory() for key in ("dQ", "dK", "dV")})
-    st0 = steps[1]
+    # its results O, dQ, dK, dV back to pinned host memory.  Heads are independent through the whole path,
+    # so the step runs over E2E_GROUPS groups of heads on three streams: a group's inputs are copied in on
+    # one, its sparse path runs on the second, its results leave on the third, and the copies of one group
+    # overlap the work and the copies of the others (events keep a group's inputs until its path has read
+    # them and its results until they have left) ----
+    BH = wl.B * wl.H
+    ng = E2E_GROUPS if BH % E2E_GROUPS == 0 else 1
+    hg = BH // ng
+    gdims = L.make_dims(1, hg, wl.T, wl.d, wl.s, K_SEL, dtype="bf16")
+    gst = ops.SSAStep(gdims, device=dev, main="sparse", grad_fp32=True)  # a group's scratch, reused in turn
+    flat = lambda t: t.view(BH, wl.T, wl.d)  # noqa: E731
+    dev_in = {key: flat(d[key]) for key in ("Q", "K", "V", "dO")}
+    dev_out = {"O": flat(torch.empty_like(d["Q"]))}
+    dev_out.update({key: flat(torch.empty(d["Q"].shape, dtype=torch.float32, device=dev)) for key in ("dQ", "dK", "dV")})
+    host_in = {key: flat(host[key]) for key in dev_in}
+    host_out = {"O": flat(torch.empty_like(host["Q"]).pin_memory())}
+    host_out.update({key: flat(torch.empty(host["Q"].shape, dtype=torch.float32).pin_memory())
+                     for key in ("dQ", "dK", "dV")})
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(ng)] for _ in range(3))
+
+    def e2e_step():
+        for g in range(ng):
+            sl = slice(g * hg, (g + 1) * hg)
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_comp[g])  # the previous step's path has read this group's inputs
+                for key in dev_in:
+                    dev_in[key][sl].copy_(host_in[key][sl], non_blocking=True)
+                ev_in[g].record(s_in)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(ev_in[g])
+                s_comp.wait_event(ev_out[g])  # the previous step's results of this group have left
+                Q, K, V, dO = (dev_in[key][sl] for key in ("Q", "K", "V", "dO"))
+                O, dQ, dK, dV = (dev_out[key][sl] for key in ("O", "dQ", "dK", "dV"))
+                L.ssa_block_pool(gdims, K, gst.Kbar)
+                L.ssa_block_select(gdims, Q, gst.Kbar, gst.idx)
+                L.ssa_sparse_index(gdims, gst.idx, gst.index)
+                L.ssa_sparse_attn_fwd(gdims, Q, K, V, gst.idx, O, gst.lse_s, gst.ws[L.SSA_OP_SPARSE_FWD],
+                                      O_lo=gst.Os_lo, index=gst.index)
+                L.ssa_sparse_attn_bwd(gdims, Q, K, V, O, gst.lse_s, dO, gst.idx, dQ, dK, dV, G32,
+                                      gst.ws[L.SSA_OP_SPARSE_BWD], O_lo=gst.Os_lo, index=gst.index)
+                ev_comp[g].record(s_comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[g])
+                for key in dev_out:
+                    host_out[key][sl].copy_(dev_out[key][sl], non_blocking=True)
+                ev_out[g].record(s_out)
+
+    e2e_step()  # untimed: first use of the streams and the group's buffers
+    torch.cuda.synchronize(dev)
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
     e_start.record(stream)
+    for s_ in (s_in, s_comp, s_out):
+        s_.wait_event(e_start)
     for i in range(args.steps):
-        for key in ("Q", "K", "V", "dO"):
-            d[key].copy_(host[key], non_blocking=True)
-        dd = st0.dims
-        L.ssa_block_pool(dd, d["K"], st0.Kbar)
-        L.ssa_block_select(dd, d["Q"], st0.Kbar, st0.idx)
-        L.ssa_sparse_index(dd, st0.idx, st0.index)
-        L.ssa_sparse_attn_fwd(dd, d["Q"], d["K"], d["V"], st0.idx, st0.Os, st0.lse_s, st0.ws[L.SSA_OP_SPARSE_FWD],
-                              O_lo=st0.Os_lo, index=st0.index)
-        L.ssa_sparse_attn_bwd(dd, d["Q"], d["K"], d["V"], st0.Os, st0.lse_s, d["dO"], st0.idx, st0.dQ, st0.dK,
-                              st0.dV, G32, st0.ws[L.SSA_OP_SPARSE_BWD], O_lo=st0.Os_lo, index=st0.index)
-        for key, src in (("O", st0.Os), ("dQ", st0.dQ), ("dK", st0.dK), ("dV", st0.dV)):
-            out_host[key].copy_(src, non_blocking=True)
+        e2e_step()
+    for s_ in (s_in, s_comp, s_out):
+        done = torch.cuda.Event()
+        done.record(s_)
+        stream.wait_event(done)
     e_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     e_ms = e_start.elapsed_time(e_end)
+    # the pipelined path's sparse output must equal the timed steps' (the forward is deterministic per head): a
+    # missing dependency between the streams would show here
+    e2e_o_diff = (dev_out["O"].float() - flat(steps[1].Os).float()).abs().max().item()
     if L.ssa_get_device_error() != L.SSA_OK:
         raise RuntimeError("device error during timing")
 
@@ -526,9 +571,11 @@ def ours(args, rank, world, local_rank):
         "roofline": roof,
         "e2e": {"value": whole_job_tokens_per_s(wl.B * wl.T, world, e_ms / args.steps), "unit": "tokens/s",
                 "h2d_bytes_per_step": sum(host[k].numel() * 2 for k in host),
-                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in out_host.values()),
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in host_out.values()),
                 "path": "pool, select, index, sparse fwd, sparse bwd with Q, K, V, dO copied in and O, dQ, dK, dV "
-                        "copied out every step"},
+                        "copied out every step, over %d head groups on three streams (copy in, sparse path, "
+                        "copy out)" % ng,
+                "o_max_abs_diff_vs_timed_steps": e2e_o_diff},
         "gpu_launches": args.steps * (ops.SSAStep.KERNELS_FWD + steps[0].kernels_bwd()),
         "clocks": clocks,
     }
