@@ -176,3 +176,40 @@ def test_product_does_not_import_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in txt and "from oracle" not in txt and "ssa_oracle" not in txt, f
+
+
+def test_decode_argument_validation(lib):
+    """ssa_sparse_decode refuses what its kernels do not cover before enqueueing anything."""
+    p = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    big = 1 << 40
+
+    def call(d, cache_len=p, q=p, kc=p, vc=p, kbar=p, idx=p, o=p, lse=p, ws=p, ws_bytes=big):
+        return _call("ssa_sparse_decode", d, cache_len, q, kc, vc, kbar, idx, o, lse, ws, ws_bytes, None)
+
+    ok = L.make_dims(2, 8, 4096, 128, 128, 4, Hkv=2)
+    assert call(L.make_dims(2, 8, 4096, 64, 64, 4)) == L.SSA_ERR_UNSUPPORTED                  # d = 64
+    assert call(L.make_dims(2, 8, 4096, 128, 128, 4, dtype="fp32")) == L.SSA_ERR_UNSUPPORTED   # fp32 caches
+    assert call(L.make_dims(1, 32, 4096, 128, 128, 4, Hkv=1)) == L.SSA_ERR_UNSUPPORTED         # group of 32
+    assert call(L.make_dims(1, 2, 128 * 1025, 128, 128, 4)) == L.SSA_ERR_UNSUPPORTED           # 1025 blocks
+    for name in ("cache_len", "q", "kc", "vc", "kbar", "idx", "o", "lse"):
+        assert call(ok, **{name: None}) == L.SSA_ERR_INVALID_ARG, name
+    assert call(ok, q=ctypes.c_void_p(24)) == L.SSA_ERR_INVALID_ARG                            # q off 16 B
+    need = L.ssa_workspace_size(ok, L.SSA_OP_DECODE)
+    assert call(ok, ws_bytes=need - 1) == L.SSA_ERR_WORKSPACE
+    assert call(ok, ws=None, ws_bytes=need) == L.SSA_ERR_WORKSPACE
+
+
+def test_rope_argument_validation(lib):
+    """ssa_rope refuses a bad base, factor, head count or start position before enqueueing anything."""
+    p = ctypes.c_void_p(16)
+    d = L.make_dims(1, 4, 1024, 128, 128, 1)
+    f = ctypes.c_float
+
+    def call(X=p, heads=4, pos0=0, base=10000.0, factor=1.0, dims=d):
+        return _call("ssa_rope", dims, X, heads, pos0, f(base), f(factor), 0, None)
+
+    for over in (dict(X=None), dict(heads=0), dict(pos0=-1), dict(base=1.0), dict(base=float("nan")),
+                 dict(base=float("inf")), dict(factor=0.0), dict(factor=-4.0), dict(factor=float("inf"))):
+        assert call(**over) == L.SSA_ERR_INVALID_ARG, over
+    # B * heads * T rows beyond int32
+    assert call(dims=L.make_dims(1, 1, 1 << 22, 128, 128, 1), heads=1024) == L.SSA_ERR_UNSUPPORTED
