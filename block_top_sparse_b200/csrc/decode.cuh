@@ -36,7 +36,7 @@
 namespace ssa {
 
 constexpr int kDecThreads = 256;
-constexpr int kDecMaxBlocks = 1024;  // the warp search holds 32 keys per lane
+constexpr int kDecMaxBlocks = 1024;  // the warp search holds at most 32 scores per lane
 constexpr int kDecMaxGroup = 16;     // query heads per key head
 
 enum : unsigned { ERR_BAD_INPUT = 6u };
