@@ -163,7 +163,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Untiled bulk copy of `bytes` contiguous bytes global -> this CTA's shared memory, completing on `bar`
-// (both addresses 16-byte aligned, bytes a multiple of 16).  No multicast.
+// (both addresses 16-byte aligned, bytes a multiple of 16); the copy lands in this CTA only.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
